@@ -1,0 +1,9 @@
+"""fp64 CPU oracle of the routed MoE layer forward -- test infrastructure.
+
+Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package.  It shares no code with the CUDA
+library and never receives a value computed by it.
+"""
+
+from .moe_oracle import *  # noqa: F401,F403
+from .moe_oracle import __all__  # noqa: F401

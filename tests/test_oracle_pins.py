@@ -1,0 +1,339 @@
+"""Pins for the fp64 oracle, against things other than the oracle itself.
+
+Each check compares the oracle with a hand-worked example, a closed form, a
+library routine doing a special case, an invariant, exact rational arithmetic
+or brute force on tiny inputs.  The planted-mistake tests at the bottom plant
+plausible bugs into the oracle (on the CPU) and confirm a pin catches each.
+"""
+
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from routing_dispatch_expert_softmax_b200 import workloads as wl
+
+
+def _np(t):
+    return t.float().numpy().astype(np.float64) if t is not None else None
+
+
+# ---------------------------------------------------------------- selection
+def test_topk_hand_worked_examples(golden):
+    for case in golden["topk"]:
+        L = np.array([case["logits"]], dtype=np.float32)
+        k = case["k"]
+        got = oracle.topk_select(L, k)[0].tolist()
+        assert got == case["idx"], case["why"]
+        assert oracle.topk_select_sorted(L, k)[0].tolist() == case["idx"]
+        L64 = np.array([case["logits"]], dtype=np.float64)
+        w = oracle.gate_weights(L64, np.array([case["idx"]]))[0]
+        want = [eval(expr, {"exp": math.exp}) for expr in case["gates"]]
+        np.testing.assert_allclose(w, want, rtol=0, atol=1e-12, err_msg=case["why"])
+
+
+def _lexmax_topk(row, k):
+    """Brute force over all ordered k-subsets: the selection is the
+    lexicographically greatest sequence of (value, -index) pairs."""
+    best = None
+    for combo in itertools.permutations(range(len(row)), k):
+        key = tuple((float(row[e]) + 0.0, -e) for e in combo)
+        if best is None or key > best[0]:
+            best = (key, combo)
+    return list(best[1])
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "const"])
+def test_topk_brute_force_tiny(kind):
+    L = wl.make_logits(40, 6, seed=3, kind=kind).numpy()
+    for k in (1, 2, 3, 6):
+        a = oracle.topk_select(L, k)
+        b = oracle.topk_select_sorted(L, k)
+        np.testing.assert_array_equal(a, b)
+        for t in range(0, 40, 7):
+            assert a[t].tolist() == _lexmax_topk(L[t], k)
+
+
+def test_topk_forms_agree_tie_heavy_wide():
+    L = wl.make_logits(200, 16, seed=5, kind="ties").numpy()
+    for k in (1, 4, 8, 16):
+        np.testing.assert_array_equal(oracle.topk_select(L, k),
+                                      oracle.topk_select_sorted(L, k))
+
+
+def test_topk_signed_zero_ties():
+    L = np.array([[-0.0, 0.0, -0.0, 0.0]], dtype=np.float32)
+    assert oracle.topk_select(L, 2)[0].tolist() == [0, 1]
+    L = np.array([[0.0, -0.0, -1.0, -0.0]], dtype=np.float32)
+    assert oracle.topk_select_sorted(L, 3)[0].tolist() == [0, 1, 3]
+
+
+def test_topk_rejects_bad_k():
+    L = np.zeros((2, 4), np.float32)
+    for k in (0, 5):
+        with pytest.raises(ValueError):
+            oracle.topk_select(L, k)
+
+
+# ---------------------------------------------------------------- gates
+def test_gates_sum_to_one_and_k_equals_E_is_softmax():
+    L = wl.make_logits(64, 12, seed=1).numpy().astype(np.float64) * 3.0
+    for k in (1, 2, 5, 12):
+        idx = oracle.topk_select_sorted(L, k)
+        w = oracle.gate_weights(L, idx)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+        assert np.all(w > 0)
+        assert np.all(np.diff(w, axis=1) <= 1e-15)  # slots in descending order
+    idx = oracle.topk_select_sorted(L, 12)
+    w = oracle.gate_weights(L, idx)
+    ref = scipy.special.softmax(L, axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(ref, idx.astype(np.int64), 1),
+                               rtol=1e-13, atol=0)
+
+
+def test_gates_k2_closed_form_is_logistic():
+    L = wl.make_logits(50, 7, seed=2).numpy().astype(np.float64) * 2.0
+    idx = oracle.topk_select_sorted(L, 2)
+    w = oracle.gate_weights(L, idx)
+    a = np.take_along_axis(L, idx[:, :1].astype(np.int64), 1)[:, 0]
+    b = np.take_along_axis(L, idx[:, 1:2].astype(np.int64), 1)[:, 0]
+    np.testing.assert_allclose(w[:, 0], scipy.special.expit(a - b), rtol=1e-13)
+    np.testing.assert_allclose(w[:, 1], scipy.special.expit(b - a), rtol=1e-12)
+
+
+def test_gates_shift_invariant_and_large_logits_finite():
+    L = wl.make_logits(16, 8, seed=4).numpy().astype(np.float64)
+    idx = oracle.topk_select_sorted(L, 3)
+    w0 = oracle.gate_weights(L, idx)
+    w1 = oracle.gate_weights(L + 700.0, idx)  # exp(700+) would overflow unshifted
+    np.testing.assert_allclose(w0, w1, rtol=1e-10)
+    assert np.all(np.isfinite(w1))
+
+
+# ---------------------------------------------------------------- counts / rows
+def test_dispatch_hand_worked_example(golden):
+    g = golden["dispatch"]
+    idx = np.array(g["idx"], dtype=np.int32)
+    counts = oracle.expert_counts(idx, g["E"])
+    assert counts.tolist() == g["counts"]
+    assert oracle.expert_offsets(counts).tolist() == g["offsets"]
+    perm, row_of = oracle.dispatch_rows(idx, g["E"])
+    assert perm.tolist() == g["perm"]
+    assert row_of.tolist() == g["row_of"]
+    S, ro = oracle.virtual_ep_layout(idx, g["E"], g["R"])
+    assert S.tolist() == g["send_counts"]
+    assert ro.tolist() == g["rank_offsets"]
+
+
+def test_imbalance_hand_worked_example(golden):
+    g = golden["imbalance"]
+    assert oracle.imbalance_factor(np.array(g["counts"]), g["R"]) == pytest.approx(g["factor"])
+
+
+@pytest.mark.parametrize("T,E,k,R", [(1, 8, 2, 2), (37, 16, 4, 4), (300, 32, 8, 8),
+                                     (5, 4, 4, 2)])
+def test_counts_offsets_perm_invariants(T, E, k, R):
+    L = wl.make_logits(T, E, seed=T + E).numpy()
+    idx = oracle.topk_select_sorted(L, k)
+    counts = oracle.expert_counts(idx, E)
+    # library routines for the special cases
+    np.testing.assert_array_equal(counts, np.bincount(idx.reshape(-1), minlength=E))
+    assert counts.sum() == T * k
+    assert counts.mean() == pytest.approx(T * k / E)  # mean load B*k/E
+    offsets = oracle.expert_offsets(counts)
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    perm, row_of = oracle.dispatch_rows(idx, E)
+    P = T * k
+    assert sorted(row_of.reshape(-1).tolist()) == list(range(P))  # bijection
+    for t in range(T):
+        for j in range(k):
+            r = row_of[t, j]
+            assert perm[r] == t
+            e = idx[t, j]
+            assert offsets[e] <= r < offsets[e + 1]
+    # rows equal a stable library sort of the pairs by (expert, token)
+    flat_e = idx.reshape(-1)
+    flat_t = np.repeat(np.arange(T), k)
+    order = np.lexsort((flat_t, flat_e))
+    np.testing.assert_array_equal(perm, flat_t[order])
+    S, ro = oracle.virtual_ep_layout(idx, E, R)
+    assert S.sum() == P
+    chunk = -(-T // R)
+    per_src = np.array([min(T, (s + 1) * chunk) - min(T, s * chunk) for s in range(R)])
+    np.testing.assert_array_equal(S.sum(axis=1), per_src * k)
+    np.testing.assert_array_equal(S.sum(axis=0), np.diff(ro))
+    assert ro[0] == 0 and ro[-1] == P
+
+
+def test_dispatch_then_combine_is_identity():
+    T, d, E = 33, 24, 8
+    x = np.random.default_rng(0).standard_normal((T, d))
+    L = wl.make_logits(T, E, seed=9).numpy()
+    # k = 1 with unit gates: bit-exact identity
+    idx = oracle.topk_select_sorted(L, 1)
+    perm, row_of = oracle.dispatch_rows(idx, E)
+    y = oracle.combine(x[perm], row_of, np.ones((T, 1)))
+    np.testing.assert_array_equal(y, x)
+    # k = 3 with gates summing to 1: identity up to rounding
+    idx = oracle.topk_select_sorted(L, 3)
+    perm, row_of = oracle.dispatch_rows(idx, E)
+    w = oracle.gate_weights(L, idx)
+    y = oracle.combine(x[perm], row_of, w)
+    np.testing.assert_allclose(y, x, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- FFN / layer
+def test_silu_against_library():
+    z = np.linspace(-30, 30, 1001)
+    np.testing.assert_allclose(oracle.silu(z), z * scipy.special.expit(z), rtol=1e-14)
+
+
+def test_router_logits_exact_rational():
+    rng = np.random.default_rng(1)
+    x = rng.integers(-8, 8, (3, 5)) / 8.0
+    W = rng.integers(-8, 8, (5, 4)) / 16.0
+    b = rng.integers(-4, 4, 4) / 4.0
+    L = oracle.router_logits(x, W, b)
+    for t in range(3):
+        for e in range(4):
+            exact = sum(Fraction(x[t, i]) * Fraction(W[i, e]) for i in range(5)) + Fraction(b[e])
+            assert L[t, e] == float(exact)
+
+
+def _small_layer(T, d, E, k, f, seed=0, zipf=None):
+    cfg = wl.MoEConfig("pin", T=T, d=d, E=E, k=k, f=f, zipf_s=zipf)
+    t = wl.make_layer(cfg, "cpu", seed)
+    return cfg, {n: _np(v) for n, v in t.items()}
+
+
+def test_single_expert_k1_is_plain_swiglu_ffn():
+    cfg, t = _small_layer(T=9, d=32, E=1, k=1, f=48)
+    out = oracle.moe_forward(t["x"], t["w_g"], None, t["w13"], t["w2"], k=1)
+    x = torch.tensor(t["x"], dtype=torch.float64)
+    Wg = torch.tensor(t["w13"][0, :48], dtype=torch.float64)
+    Wu = torch.tensor(t["w13"][0, 48:], dtype=torch.float64)
+    Wd = torch.tensor(t["w2"][0], dtype=torch.float64)
+    ref = torch.nn.functional.linear(
+        torch.nn.functional.silu(torch.nn.functional.linear(x, Wg))
+        * torch.nn.functional.linear(x, Wu), Wd)
+    np.testing.assert_allclose(out["y"], ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.all(out["w"] == 1.0)
+
+
+def test_k_equals_E_is_dense_gate_weighted_sum():
+    cfg, t = _small_layer(T=11, d=32, E=4, k=4, f=16)
+    out = oracle.moe_forward(t["x"], t["w_g"], None, t["w13"], t["w2"], k=4)
+    x = torch.tensor(t["x"], dtype=torch.float64)
+    p = torch.softmax(x @ torch.tensor(t["w_g"], dtype=torch.float64), dim=1)
+    y = torch.zeros_like(x)
+    for e in range(4):
+        W = torch.tensor(t["w13"][e], dtype=torch.float64)
+        Wd = torch.tensor(t["w2"][e], dtype=torch.float64)
+        h = torch.nn.functional.silu(x @ W[:16].T) * (x @ W[16:].T)
+        y += p[:, e:e + 1] * (h @ Wd.T)
+    np.testing.assert_allclose(out["y"], y.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_layer_per_token_brute_force_with_bias():
+    cfg, t = _small_layer(T=13, d=32, E=8, k=3, f=16, zipf=1.0)
+    out = oracle.moe_forward(t["x"], t["w_g"], t["bias"], t["w13"], t["w2"], k=3)
+    for tok in range(13):
+        xt = t["x"][tok]
+        L = xt @ t["w_g"] + t["bias"]
+        L32 = L.astype(np.float32)
+        order = sorted(range(8), key=lambda e: (-float(L32[e]), e))[:3]
+        assert out["idx"][tok].tolist() == order
+        ex = np.exp(L[order] - L.max())
+        gates = ex / ex.sum()
+        acc = np.zeros(32)
+        for g, e in zip(gates, order):
+            W = t["w13"][e]
+            h = (xt @ W[:16].T) / (1 + np.exp(-(xt @ W[:16].T))) * (xt @ W[16:].T)
+            acc += g * (h @ t["w2"][e].T)
+        np.testing.assert_allclose(out["y"][tok], acc, rtol=1e-11, atol=1e-12)
+
+
+def test_bias_skews_popularity_toward_low_rank():
+    cfg = wl.MoEConfig("skew", T=4000, d=64, E=16, k=1, f=8, zipf_s=1.0)
+    w_g, bias = wl.make_router(cfg, "cpu", 0)
+    x = wl.make_hidden(cfg, "cpu", 0)
+    L = oracle.router_logits(_np(x), _np(w_g), _np(bias))
+    counts = oracle.expert_counts(oracle.topk_select_sorted(L, 1), 16)
+    hottest = int(np.argmax(_np(bias)))
+    assert counts[hottest] == counts.max()
+    assert counts.max() > 3 * cfg.T / 16
+
+
+def test_weight_bytes_match_memory_sizing():
+    # Expert memory = N_experts * P_per_expert * bytes ("Expert Parallelism
+    # for MoE Models", memory sizing), P_per_expert = 3*d*f for SwiGLU.
+    assert wl.DEEPSEEK_V3_ROUTED.expert_bytes() * 256 == pytest.approx(22.55e9, rel=1e-3)
+    assert wl.QWEN3_30B_A3B_DECODE.expert_bytes() * 128 == pytest.approx(1.208e9, rel=1e-3)
+    assert wl.MIXTRAL_8X7B.expert_bytes() * 8 == pytest.approx(2.818e9, rel=1e-3)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def _pins_fail(monkeypatch, name, bad, golden):
+    monkeypatch.setattr(oracle.moe_oracle, name, bad)
+    monkeypatch.setattr(oracle, name, bad)
+    failures = 0
+    for fn in (lambda: test_topk_hand_worked_examples(golden),
+               lambda: test_dispatch_hand_worked_example(golden),
+               lambda: test_single_expert_k1_is_plain_swiglu_ffn(),
+               lambda: test_k_equals_E_is_dense_gate_weighted_sum(),
+               lambda: test_layer_per_token_brute_force_with_bias(),
+               lambda: test_gates_k2_closed_form_is_logistic(),
+               lambda: test_counts_offsets_perm_invariants(37, 16, 4, 4)):
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            failures += 1
+    return failures
+
+
+def test_planted_tie_break_to_higher_index_is_caught(monkeypatch, golden):
+    def bad(L, k):
+        L = np.asarray(L)
+        return (L.shape[1] - 1 - np.argsort(-L[:, ::-1], axis=1, kind="stable")[:, :k]).astype(np.int32)
+    assert _pins_fail(monkeypatch, "topk_select_sorted", bad, golden) > 0
+
+
+def test_planted_missing_renormalisation_is_caught(monkeypatch, golden):
+    def bad(L, idx):
+        L = np.asarray(L, dtype=np.float64)
+        p = scipy.special.softmax(L, axis=1)
+        return np.take_along_axis(p, np.asarray(idx, dtype=np.int64), axis=1)
+    assert _pins_fail(monkeypatch, "gate_weights", bad, golden) > 0
+
+
+def test_planted_swapped_gate_up_is_caught(monkeypatch, golden):
+    def bad(X, w13_e, w2_e):
+        f = w13_e.shape[0] // 2
+        X = np.asarray(X, np.float64)
+        g = X @ np.asarray(w13_e[f:], np.float64).T
+        u = X @ np.asarray(w13_e[:f], np.float64).T
+        return (g / (1 + np.exp(-g)) * u) @ np.asarray(w2_e, np.float64).T
+    assert _pins_fail(monkeypatch, "swiglu_ffn", bad, golden) > 0
+
+
+def test_planted_token_descending_rows_are_caught(monkeypatch, golden):
+    real = oracle.moe_oracle.dispatch_rows
+
+    def bad(idx, E):
+        idx = np.asarray(idx)
+        perm, row_of = real(idx[::-1], E)
+        T = idx.shape[0]
+        return (T - 1 - perm).astype(np.int32), row_of[::-1].copy()
+    assert _pins_fail(monkeypatch, "dispatch_rows", bad, golden) > 0
+
+
+def test_planted_wrong_silu_sign_is_caught(monkeypatch, golden):
+    def bad(z):
+        z = np.asarray(z, np.float64)
+        return z / (1.0 + np.exp(z))
+    assert _pins_fail(monkeypatch, "silu", bad, golden) > 0
