@@ -1,0 +1,183 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed mixture-of-experts layer forward.
+ *
+ * The operation is the routed MoE layer the expert-parallel serving pages
+ * describe, on one GPU:
+ *   - "Wide Expert Parallelism" (llm-d), section "What is an MoE layer?": a
+ *     routing gate scores every token and sends it to a few experts (8 of 256
+ *     in the DeepSeek example);
+ *   - "Serving MoE models with expert parallelism on 8xH200", section "Tensor
+ *     parallel vs expert parallel": tokens are dispatched to the holders of
+ *     their experts, run through full-size expert GEMMs, and returned by a
+ *     second exchange.  On one GPU both exchanges become local permutations;
+ *   - same page, section "Routing imbalance": per-expert token counts;
+ *   - "Expert Parallelism for MoE Models" (apxml), section "Mechanics of Token
+ *     Routing and All-to-All Communication": token representations travel to
+ *     the expert and the output travels back.
+ * The pages leave the arithmetic open; this library computes softmax scoring
+ * of linear router logits, top-k selection (ties to the lower expert index,
+ * slots in descending logit order), gates renormalised over the k selected,
+ * SwiGLU experts h = silu(x Wg) * (x Wu), z = h Wd, and the gate-weighted sum.
+ *
+ * Conventions for every entry point
+ *   - Pointers named x, w_g, ... are DEVICE pointers, 16-byte aligned, owned by
+ *     the caller.  The library never allocates, frees or synchronises (except
+ *     moe_check) and writes only the outputs named in each call plus `ws`.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on it.
+ *   - bf16 tensors are passed as raw 16-bit patterns (moe_bf16).  All matrices
+ *     are row-major and densely packed.
+ *   - The return value is a moe_status.  Argument errors are detected on the
+ *     host before anything is launched.  Errors found on the device (an expert
+ *     index out of range, inconsistent offsets, a bounded wait that ran out) are
+ *     recorded in the workspace's error word and reported by moe_check.
+ *   - There is no CPU fallback: a call that would launch work returns
+ *     MOE_ERR_CUDA when no CUDA device is usable and MOE_ERR_UNSUPPORTED when
+ *     the current device is not an sm_100 GPU.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16; /* raw bfloat16 bits */
+
+/* Problem statement: T tokens of hidden size d routed to k of E experts, each
+ * a SwiGLU FFN with intermediate size f; R virtual expert-parallel ranks. */
+typedef struct moe_shape {
+  int32_t T; /* tokens in the batch, 0 <= T <= 1<<20 (T = 0 is a no-op)      */
+  int32_t d; /* hidden size, a multiple of 64, 64 <= d <= 16384               */
+  int32_t E; /* routed experts, 1 <= E <= 1024                                */
+  int32_t k; /* experts per token, 1 <= k <= min(E, 32)                       */
+  int32_t f; /* expert intermediate size, a multiple of 64, 64 <= f <= 32768  */
+  int32_t R; /* virtual EP ranks: 0 or 1 = none; otherwise R divides E, R<=64 */
+} moe_shape;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, shape out of range  */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but unsupported (no sm_100 device, ...)  */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed           */
+  MOE_ERR_TIMEOUT = 4,      /* a bounded device wait ran out (moe_check)      */
+  MOE_ERR_DEVICE_CHECK = 5  /* a device-side consistency check failed         */
+} moe_status;
+
+/* Human-readable name of a moe_status. Never NULL. */
+MOE_API const char* moe_error_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+MOE_API int moe_version(void);
+
+/* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
+ * need for shape *s (enough for all three).  Returns 0 if *s is invalid.
+ * The workspace must be 256-byte aligned.  Its first 64 bytes hold the
+ * device error word: zero them once before the first call (moe_check clears
+ * them after reporting an error); the rest needs no initialisation. */
+MOE_API size_t moe_workspace_size(const moe_shape* s);
+
+/* Router gate ("What is an MoE layer?": the gate scores each token).
+ *   x      [T, d] bf16          hidden states
+ *   w_g    [d, E] fp32          router weight
+ *   bias   [E] fp32 or NULL     per-expert additive bias
+ *   logits [T, E] fp32 out      logits[t,e] = sum_i x[t,i] w_g[i,e] + bias[e],
+ *                               accumulated in fp32 in a fixed order.       */
+MOE_API int moe_router(const moe_bf16* x, const float* w_g, const float* bias,
+               const moe_shape* s, float* logits, void* stream);
+
+/* Expert selection and gates ("What is an MoE layer?": 8 of 256 experts per
+ * token; "Batching ...": top-8 over 256).
+ *   logits [T, E] fp32 in (finite values; NaN/Inf behaviour unspecified)
+ *   idx    [T, k] int32 out     idx[t,j] = expert in slot j; slots ordered by
+ *                               descending logit, ties to the lower index
+ *   w      [T, k] fp32 out      w[t,j] = exp(L[idx[t,j]] - L[idx[t,0]]) /
+ *                               sum_j' exp(L[idx[t,j']] - L[idx[t,0]]), i.e. the
+ *                               softmax over E renormalised over the k chosen. */
+MOE_API int moe_topk(const float* logits, const moe_shape* s, int32_t* idx, float* w,
+             void* stream);
+
+/* Dispatch: the local form of the token exchange ("Tensor parallel vs expert
+ * parallel"; "Mechanics of Token Routing ...").  Rows of the expert-major
+ * buffer are ordered by (expert, token) ascending.
+ *   idx          [T, k] int32 in   expert ids; each in [0, E), distinct per token
+ *   x            [T, d] bf16 in
+ *   counts       [E] int32 out     rows per expert ("Routing imbalance")
+ *   offsets      [E+1] int32 out   exclusive prefix sum, offsets[E] = T*k
+ *   perm         [T*k] int32 out   perm[row] = token
+ *   row_of       [T, k] int32 out  row_of[t,j] = row of (t, j)
+ *   x_perm       [T*k, d] bf16 out x_perm[row] = x[perm[row]]
+ *   send_counts  [R, R] int32 out or NULL (needs R > 1): S[s][r] = rows that
+ *                source rank s = t / ceil(T/R) sends to the rank r = e/(E/R)
+ *                owning the expert ("Expert Parallelism: keep specialists
+ *                whole": contiguous expert blocks per device)
+ *   rank_offsets [R+1] int32 out or NULL: first row of each rank; rank r's
+ *                buffer is x_perm[rank_offsets[r] : rank_offsets[r+1]]
+ *   ws           workspace of moe_workspace_size(s) bytes
+ * An out-of-range expert id is recorded as MOE_ERR_DEVICE_CHECK.           */
+MOE_API int moe_dispatch(const int32_t* idx, const moe_bf16* x, const moe_shape* s,
+                 int32_t* counts, int32_t* offsets, int32_t* perm,
+                 int32_t* row_of, moe_bf16* x_perm, int32_t* send_counts,
+                 int32_t* rank_offsets, void* ws, void* stream);
+
+/* Expert FFNs over the expert-major rows ("full-size expert GEMMs"):
+ * for the rows r in [offsets[e], offsets[e+1]) of expert e,
+ *   h = silu(x_perm[r] Wg_e) * (x_perm[r] Wu_e)   (fp32 accumulate, h in bf16)
+ *   z[r] = h Wd_e                                  (fp32 accumulate, bf16 out)
+ *   x_perm [T*k, d] bf16 in
+ *   offsets [E+1] int32 in      device-resident; monotone, offsets[E] = T*k
+ *   w13    [E, 2f, d] bf16 in   rows 0..f-1 = Wg_e^T, rows f..2f-1 = Wu_e^T
+ *   w2     [E, d, f] bf16 in    Wd_e^T
+ *   z      [T*k, d] bf16 out
+ *   ws     workspace of moe_workspace_size(s) bytes
+ * Runs on the tcgen05 tensor cores with TMA-fed operands.  Bad offsets are
+ * recorded as MOE_ERR_DEVICE_CHECK.                                        */
+MOE_API int moe_ffn(const moe_bf16* x_perm, const int32_t* offsets,
+            const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
+            moe_bf16* z, void* ws, void* stream);
+
+/* Combine: the return exchange plus the gate-weighted sum ("Tensor parallel
+ * vs expert parallel": results are sent back by a second exchange),
+ *   y[t] = sum_{j<k} w[t,j] * z[row_of[t,j]], summed in fp32 in slot order.
+ *   z [T*k, d] bf16 in; row_of [T, k] int32 in; w [T, k] fp32 in;
+ *   y [T, d] bf16 out.  Row indices out of range make y undefined. */
+MOE_API int moe_combine(const moe_bf16* z, const int32_t* row_of, const float* w,
+                const moe_shape* s, moe_bf16* y, void* stream);
+
+/* The whole layer: router, selection, dispatch, expert FFNs, combine, in one
+ * stream-ordered sequence with no host synchronisation (capturable in a CUDA
+ * graph).  Inputs as above; y [T, d] bf16 out.  idx_out [T,k], w_out [T,k]
+ * and counts_out [E] receive the routing decisions when non-NULL.  With
+ * s->R > 1 the send-count matrix and rank offsets are computed too (in the
+ * workspace).  ws: moe_workspace_size(s) bytes. */
+MOE_API int moe_forward(const moe_bf16* x, const float* w_g, const float* bias,
+                const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
+                moe_bf16* y, int32_t* idx_out, float* w_out,
+                int32_t* counts_out, void* ws, void* stream);
+
+/* Self-test of the failure path every device-side wait uses: launches one
+ * kernel that waits on a barrier nothing will ever complete, through the same
+ * bounded wait as the expert-GEMM pipeline, with a limit of limit_ns
+ * (1 .. 1e9 ns).  The wait gives up, the kernel records MOE_ERR_TIMEOUT in
+ * the error word of `ws` (at least 64 bytes, 256-byte aligned) and returns;
+ * moe_check then reports it.  Nothing hangs or traps. */
+MOE_API int moe_selftest_bounded_wait(long long limit_ns, void* ws, void* stream);
+
+/* Synchronises `stream`, returns the device error word recorded in `ws`
+ * (MOE_OK if none) and clears it. */
+MOE_API int moe_check(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

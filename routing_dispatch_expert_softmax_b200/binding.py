@@ -1,0 +1,200 @@
+"""Thin ctypes binding of ``libmoe_b200.so`` (the C ABI in ``include/moe.h``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (PyTorch supplies device memory and
+streams); the functions keep the C names and raise :class:`MoEError` on a
+non-zero status.  There is no fallback: if the library is missing or the
+device is not an sm_100 GPU, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_NAME = "libmoe_b200.so"
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), LIB_NAME)
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_CUDA = 3
+MOE_ERR_TIMEOUT = 4
+MOE_ERR_DEVICE_CHECK = 5
+
+# Every symbol include/moe.h declares.
+EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router",
+           "moe_topk", "moe_dispatch", "moe_ffn", "moe_combine", "moe_forward",
+           "moe_selftest_bounded_wait", "moe_check")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_error_string(status)}")
+
+
+class MoEShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("R", ctypes.c_int32)]
+
+    @classmethod
+    def of(cls, T, d, E, k, f, R=0) -> "MoEShape":
+        return cls(int(T), int(d), int(E), int(k), int(f), int(R))
+
+    @classmethod
+    def from_config(cls, cfg) -> "MoEShape":
+        return cls.of(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.R)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(MoEShape)
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads the library once; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{LIB_NAME} is not built (expected at {path}); run "
+            "`python -m routing_dispatch_expert_softmax_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.moe_error_string.restype = ctypes.c_char_p
+    lib.moe_error_string.argtypes = [ctypes.c_int]
+    lib.moe_version.restype = ctypes.c_int
+    lib.moe_version.argtypes = []
+    lib.moe_workspace_size.restype = ctypes.c_size_t
+    lib.moe_workspace_size.argtypes = [_S]
+    lib.moe_router.restype = ctypes.c_int
+    lib.moe_router.argtypes = [_P, _P, _P, _S, _P, _P]
+    lib.moe_topk.restype = ctypes.c_int
+    lib.moe_topk.argtypes = [_P, _S, _P, _P, _P]
+    lib.moe_dispatch.restype = ctypes.c_int
+    lib.moe_dispatch.argtypes = [_P, _P, _S, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+    lib.moe_ffn.restype = ctypes.c_int
+    lib.moe_ffn.argtypes = [_P, _P, _P, _P, _S, _P, _P, _P]
+    lib.moe_combine.restype = ctypes.c_int
+    lib.moe_combine.argtypes = [_P, _P, _P, _S, _P, _P]
+    lib.moe_forward.restype = ctypes.c_int
+    lib.moe_forward.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P]
+    lib.moe_check.restype = ctypes.c_int
+    lib.moe_check.argtypes = [_P, _P]
+    lib.moe_selftest_bounded_wait.restype = ctypes.c_int
+    lib.moe_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _P, _P]
+    _lib = lib
+    return lib
+
+
+def moe_error_string(status: int) -> str:
+    return load_library().moe_error_string(int(status)).decode()
+
+
+def moe_version() -> int:
+    return load_library().moe_version()
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def moe_workspace_size(shape: MoEShape) -> int:
+    return int(load_library().moe_workspace_size(ctypes.byref(shape)))
+
+
+def workspace(shape: MoEShape, device="cuda") -> torch.Tensor:
+    """A zeroed uint8 workspace of moe_workspace_size(shape) bytes (torch's
+    allocator returns 512-byte aligned blocks, above the 256 required)."""
+    n = moe_workspace_size(shape)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_router(x, w_g, bias, logits, shape: MoEShape, stream=None):
+    _check(load_library().moe_router(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), ctypes.byref(shape),
+        _ptr(logits, torch.float32, "logits"), _stream(stream)), "moe_router")
+
+
+def moe_topk(logits, idx, w, shape: MoEShape, stream=None):
+    _check(load_library().moe_topk(
+        _ptr(logits, torch.float32, "logits"), ctypes.byref(shape),
+        _ptr(idx, torch.int32, "idx"), _ptr(w, torch.float32, "w"), _stream(stream)),
+        "moe_topk")
+
+
+def moe_dispatch(idx, x, counts, offsets, perm, row_of, x_perm, shape: MoEShape, ws,
+                 send_counts=None, rank_offsets=None, stream=None):
+    _check(load_library().moe_dispatch(
+        _ptr(idx, torch.int32, "idx"), _ptr(x, torch.bfloat16, "x"), ctypes.byref(shape),
+        _ptr(counts, torch.int32, "counts"), _ptr(offsets, torch.int32, "offsets"),
+        _ptr(perm, torch.int32, "perm"), _ptr(row_of, torch.int32, "row_of"),
+        _ptr(x_perm, torch.bfloat16, "x_perm"),
+        _ptr(send_counts, torch.int32, "send_counts"),
+        _ptr(rank_offsets, torch.int32, "rank_offsets"),
+        _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_dispatch")
+
+
+def moe_ffn(x_perm, offsets, w13, w2, z, shape: MoEShape, ws, stream=None):
+    _check(load_library().moe_ffn(
+        _ptr(x_perm, torch.bfloat16, "x_perm"), _ptr(offsets, torch.int32, "offsets"),
+        _ptr(w13, torch.bfloat16, "w13"), _ptr(w2, torch.bfloat16, "w2"),
+        ctypes.byref(shape), _ptr(z, torch.bfloat16, "z"), _ptr(ws, torch.uint8, "ws"),
+        _stream(stream)), "moe_ffn")
+
+
+def moe_combine(z, row_of, w, y, shape: MoEShape, stream=None):
+    _check(load_library().moe_combine(
+        _ptr(z, torch.bfloat16, "z"), _ptr(row_of, torch.int32, "row_of"),
+        _ptr(w, torch.float32, "w"), ctypes.byref(shape), _ptr(y, torch.bfloat16, "y"),
+        _stream(stream)), "moe_combine")
+
+
+def moe_forward(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, idx_out=None, w_out=None,
+                counts_out=None, stream=None):
+    _check(load_library().moe_forward(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.bfloat16, "w13"),
+        _ptr(w2, torch.bfloat16, "w2"), ctypes.byref(shape), _ptr(y, torch.bfloat16, "y"),
+        _ptr(idx_out, torch.int32, "idx_out"), _ptr(w_out, torch.float32, "w_out"),
+        _ptr(counts_out, torch.int32, "counts_out"), _ptr(ws, torch.uint8, "ws"),
+        _stream(stream)), "moe_forward")
+
+
+def moe_selftest_bounded_wait(limit_ns: int, ws, stream=None):
+    _check(load_library().moe_selftest_bounded_wait(
+        int(limit_ns), _ptr(ws, torch.uint8, "ws"), _stream(stream)),
+        "moe_selftest_bounded_wait")
+
+
+def moe_check(ws, stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error word."""
+    return int(load_library().moe_check(_ptr(ws, torch.uint8, "ws"), _stream(stream)))

@@ -1,0 +1,253 @@
+// C ABI of the B200 routed MoE layer: argument checks, workspace carving and
+// the stream-ordered launch sequence.  No allocation, no host synchronisation
+// (except moe_check), no CPU fallback.
+#include <mutex>
+
+#include "moe_kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kVersion = 100;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
+bool ok4(const void* p) { return p != nullptr && aligned(p, 4); }
+
+bool shape_ok(const moe_shape* s) {
+  if (!s) return false;
+  if (s->T < 0 || s->T > (1 << 20)) return false;
+  if (s->d < 64 || s->d > 16384 || s->d % 64) return false;
+  if (s->E < 1 || s->E > kMaxE) return false;
+  if (s->k < 1 || s->k > kMaxK || s->k > s->E) return false;
+  if (s->f < 64 || s->f > 32768 || s->f % 64) return false;
+  if (s->R < 0 || s->R > kMaxR) return false;
+  if (s->R > 1 && s->E % s->R) return false;
+  return true;
+}
+
+// Current device: its SM count, and whether it is an sm_100 part.
+int device_check(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  static std::mutex mu;
+  static int cc_major[128], sms[128];
+  if (dev < 0 || dev >= 128) return MOE_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (cc_major[dev] == 0) {
+      int major = 0, n = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) !=
+              cudaSuccess ||
+          cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      cc_major[dev] = major;
+      sms[dev] = n;
+    }
+    *num_sms = sms[dev];
+    return cc_major[dev] == 10 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+  }
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_error_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null or misaligned pointer, or shape out of range";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: the current device is not an sm_100 GPU";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed or no CUDA device is usable";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait ran out";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a device-side consistency check failed";
+    default: return "unknown moe_status";
+  }
+}
+
+int moe_version(void) { return kVersion; }
+
+size_t moe_workspace_size(const moe_shape* s) {
+  if (!shape_ok(s)) return 0;
+  return ws_layout(*s, 0).total;
+}
+
+int moe_router(const moe_bf16* x, const float* w_g, const float* bias, const moe_shape* s,
+               float* logits, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(x) || !ok4(w_g) || !ok4(logits) || (bias && !aligned(bias, 4)))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  cudaError_t e = launch_router_partial(xb, w_g, *s, 1, logits, cs);
+  if (e == cudaSuccess && bias) e = launch_router_finish(logits, 1, bias, *s, logits, cs);
+  return cuda_status(e);
+}
+
+int moe_topk(const float* logits, const moe_shape* s, int32_t* idx, float* w, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok4(logits) || !ok4(idx) || !ok4(w)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_topk(logits, 1, nullptr, *s, nullptr, idx, w,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+int moe_dispatch(const int32_t* idx, const moe_bf16* x, const moe_shape* s, int32_t* counts,
+                 int32_t* offsets, int32_t* perm, int32_t* row_of, moe_bf16* x_perm,
+                 int32_t* send_counts, int32_t* rank_offsets, void* ws, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (!ok4(counts) || !ok4(offsets) || !ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  if ((send_counts || rank_offsets) && s->R <= 1) return MOE_ERR_INVALID_ARG;
+  if ((send_counts && !aligned(send_counts, 4)) || (rank_offsets && !aligned(rank_offsets, 4)))
+    return MOE_ERR_INVALID_ARG;
+  if (s->T > 0 && (!ok4(idx) || !ok16(x) || !ok4(perm) || !ok4(row_of) || !ok16(x_perm)))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*s, sms);
+  if (s->T == 0) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int) * s->E, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int) * (s->E + 1), cs);
+    if (e == cudaSuccess && send_counts)
+      e = cudaMemsetAsync(send_counts, 0, sizeof(int) * s->R * s->R, cs);
+    if (e == cudaSuccess && rank_offsets)
+      e = cudaMemsetAsync(rank_offsets, 0, sizeof(int) * (s->R + 1), cs);
+    return cuda_status(e);
+  }
+  int* send = send_counts ? send_counts : at<int>(ws, L.send);
+  int* roff = rank_offsets ? rank_offsets : at<int>(ws, L.rank_off);
+  cudaError_t e = launch_route_tables(idx, *s, L, static_cast<char*>(ws), counts, offsets,
+                                      row_of, perm, send, roff, cs);
+  if (e == cudaSuccess)
+    e = launch_gather(reinterpret_cast<const __nv_bfloat16*>(x), perm, L.P, s->T, s->d,
+                      reinterpret_cast<__nv_bfloat16*>(x_perm), at<int>(ws, L.err), cs);
+  return cuda_status(e);
+}
+
+int moe_ffn(const moe_bf16* x_perm, const int32_t* offsets, const moe_bf16* w13,
+            const moe_bf16* w2, const moe_shape* s, moe_bf16* z, void* ws, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(x_perm) || !ok4(offsets) || !ok16(w13) || !ok16(w2) || !ok16(z) || !ws ||
+      !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*s, sms);
+  char* w = static_cast<char*>(ws);
+  cudaError_t e = launch_tiles_from_offsets(offsets, *s, at<int>(ws, L.tiles),
+                                            at<int>(ws, L.err), cs);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_expert_ffn(reinterpret_cast<const __nv_bfloat16*>(x_perm), L.P,
+                           reinterpret_cast<const __nv_bfloat16*>(w13),
+                           reinterpret_cast<const __nv_bfloat16*>(w2), *s, L, w,
+                           reinterpret_cast<__nv_bfloat16*>(z), sms, cs);
+}
+
+int moe_combine(const moe_bf16* z, const int32_t* row_of, const float* w, const moe_shape* s,
+                moe_bf16* y, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(z) || !ok4(row_of) || !ok4(w) || !ok16(y)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_combine(reinterpret_cast<const __nv_bfloat16*>(z), row_of, w, *s,
+                                    reinterpret_cast<__nv_bfloat16*>(y),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const moe_bf16* w13,
+                const moe_bf16* w2, const moe_shape* s, moe_bf16* y, int32_t* idx_out,
+                float* w_out, int32_t* counts_out, void* ws, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(x) || !ok4(w_g) || (bias && !aligned(bias, 4)) || !ok16(w13) || !ok16(w2) ||
+      !ok16(y) || (idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4)) ||
+      (counts_out && !aligned(counts_out, 4)))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*s, sms);
+  char* wsb = static_cast<char*>(ws);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  float* logits = at<float>(ws, L.logits);
+  int* idx = idx_out ? idx_out : at<int>(ws, L.idx);
+  float* gw = w_out ? w_out : at<float>(ws, L.w);
+  int* counts = counts_out ? counts_out : at<int>(ws, L.counts);
+  int* offsets = at<int>(ws, L.offsets);
+  int* perm = at<int>(ws, L.perm);
+  int* row_of = at<int>(ws, L.row_of);
+  __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+  __nv_bfloat16* z = at<__nv_bfloat16>(ws, L.z);
+
+  cudaError_t e = launch_router_partial(xb, w_g, *s, 1, logits, cs);
+  if (e == cudaSuccess) e = launch_topk(logits, 1, bias, *s, nullptr, idx, gw, cs);
+  if (e == cudaSuccess)
+    e = launch_route_tables(idx, *s, L, wsb, counts, offsets, row_of, perm,
+                            at<int>(ws, L.send), at<int>(ws, L.rank_off), cs);
+  if (e == cudaSuccess)
+    e = launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  int r = launch_expert_ffn(x_perm, L.Ppad, reinterpret_cast<const __nv_bfloat16*>(w13),
+                            reinterpret_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms,
+                            cs);
+  if (r != MOE_OK) return r;
+  return cuda_status(launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs));
+}
+
+int moe_selftest_bounded_wait(long long limit_ns, void* ws, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 1000000000LL || !ws || !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_selftest_bounded_wait((unsigned long long)limit_ns,
+                                                  static_cast<int*>(ws),
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int moe_check(void* ws, void* stream) {
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (h[0] != 0) {
+    if (cudaMemsetAsync(ws, 0, 64, cs) != cudaSuccess || cudaStreamSynchronize(cs) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return h[0];
+}
+
+}  // extern "C"

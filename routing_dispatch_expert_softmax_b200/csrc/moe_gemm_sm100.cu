@@ -1,0 +1,354 @@
+// Expert FFN grouped GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// "Serving MoE models with expert parallelism on 8xH200", section "Tensor
+// parallel vs expert parallel": each expert's tokens go through full-size
+// expert GEMMs; section "Batching ...": at small batch the expert GEMM streams
+// the expert's weights from HBM for a handful of token rows.
+//
+// One persistent kernel template serves both GEMMs of the SwiGLU expert:
+//   GEMM1 (SWIGLU = true):  A = x_perm rows, B = [Wg_e^T tile ; Wu_e^T tile],
+//                           epilogue h = silu(g) * u  -> bf16 h
+//   GEMM2 (SWIGLU = false): A = h rows, B = Wd_e^T tile -> bf16 z
+// Work item = (128-row tile of one expert, BN-wide output tile).  The list of
+// row tiles is built on the device from the expert offsets, so the launch
+// needs no host synchronisation; the grid is one CTA per SM and each CTA
+// strides through the work items.
+//
+// CTA = 6 warps: warp 0 issues TMA loads (one thread), warp 1 owns TMEM and
+// issues tcgen05.mma (one thread), warps 2-5 drain the accumulator (TMEM lane
+// quarter = warp % 4).  Shared memory holds STAGES (A, B) K-slices of 64
+// elements in the 128-byte-swizzled K-major layout; TMEM holds two fp32
+// accumulators of 128 x BN so the epilogue of one tile overlaps the MMAs of
+// the next.  Every wait is bounded (error word MOE_ERR_TIMEOUT, then drain and
+// return).
+#include "moe_kernels.cuh"
+
+namespace moe {
+
+template <int BN, bool SWIGLU>
+struct GemmCfg {
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
+  static constexpr int kBBytes = BN * kGemmBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;  // double-buffered accumulator
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256;
+  static constexpr int kThreads = 192;
+};
+
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                unsigned long long limit_ns) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+template <int BN, bool SWIGLU>
+__global__ void __launch_bounds__(192, 1) k_grouped_gemm(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const int* __restrict__ tiles, int n_tiles, int K, int b_rows_per_expert,
+    int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
+    int* __restrict__ err) {
+  using C = GemmCfg<BN, SWIGLU>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_mtiles = tiles[0];
+  const int total = num_mtiles * n_tiles;
+  const int nk = K / kGemmBK;
+  const int* tl = tiles + 4;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+      const uint64_t pol_a = policy_evict_last();   // activations: reused
+      int fills[S];
+#pragma unroll
+      for (int s = 0; s < S; ++s) fills[s] = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int mt = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
+        const int row0 = tl[3 * mt + 0];
+        const int e = tl[3 * mt + 2];
+        const int brow = e * b_rows_per_expert + nt * (SWIGLU ? BN / 2 : BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = smem + stage * C::kStageBytes;
+          uint8_t* b_dst = a_dst + C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * kGemmBK, row0, pol_a);
+          if (SWIGLU) {
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * kGemmBK, brow, pol_w);
+            tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[stage], kb * kGemmBK,
+                        brow + up_offset, pol_w);
+          } else {
+            tma_load_2d(b_dst, &tmB, &full[stage], kb * kGemmBK, brow, pol_w);
+          }
+          ++fills[stage];
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        // Let every copy already issued land before the CTA leaves.
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+          if (fills[s] > 0) mbar_wait_limit(&full[s], (uint32_t)((fills[s] - 1) & 1), 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+            umma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                         sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                         (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);  // frees the smem slot when these MMAs finish
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit(&tfull[ab]);
+      }
+      if (*abort_flag) {
+        umma_commit(drain);
+        mbar_wait_limit(drain, 0, 100000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    const int r_in_tile = q * 32 + lane;
+    int it = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+      const int mt = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
+      const int row0 = tl[3 * mt + 0];
+      const int rowend = tl[3 * mt + 1];
+      const int ab = it & 1;
+      const uint32_t aph = (uint32_t)((it >> 1) & 1);
+      const bool got = mbar_wait_bounded(&tfull[ab], aph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t t_addr = tmem_base + (uint32_t)(ab * BN) + ((uint32_t)(q * 32) << 16);
+      const int row = row0 + r_in_tile;
+      const bool row_ok = row < rowend;
+      if (SWIGLU) {
+        constexpr int H = BN / 2;
+#pragma unroll 1
+        for (int c = 0; c < H; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(t_addr + c, g);
+          tmem_ld_32x32b_x32(t_addr + H + c, u);
+          tmem_ld_wait();
+          const int col = nt * H + c;
+          if (row_ok && col < n_out) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              p[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(t_addr + c, a);
+          tmem_ld_wait();
+          const int col = nt * BN + c;
+          if (row_ok && col < n_out) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              p[i] = pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0 && *abort_flag) record_error(err, MOE_ERR_TIMEOUT, 10);
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ============================================================== host side
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                    void*, const cuuint64_t*, const cuuint64_t*,
+                                    const cuuint32_t*, const cuuint32_t*,
+                                    CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix; box = 64 columns
+// (128 bytes, the swizzle span) x box_rows rows, 128-byte swizzle.
+static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kGemmBK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWIGLU>
+static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
+                                 const int* tiles, int max_work, int n_tiles, int K,
+                                 int b_rows, int up_off, int n_out, __nv_bfloat16* out,
+                                 int ld_out, int* err, int num_sms, cudaStream_t st) {
+  using C = GemmCfg<BN, SWIGLU>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<BN, SWIGLU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int grid = max_work < num_sms ? max_work : num_sms;
+  if (grid < 1) grid = 1;
+  k_grouped_gemm<BN, SWIGLU><<<grid, C::kThreads, C::kSmemBytes, st>>>(
+      ta, tb, tiles, n_tiles, K, b_rows, up_off, n_out, out, ld_out, err);
+  return cudaGetLastError();
+}
+
+// Both expert GEMMs over the rows described by the device tile list.
+//   x_rows: rows of x_perm visible to TMA (P for a caller buffer, Ppad inside
+//   the workspace); h has Ppad rows (workspace).
+int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
+                      const __nv_bfloat16* w13, const __nv_bfloat16* w2,
+                      const moe_shape& s, const WsLayout& L, char* ws,
+                      __nv_bfloat16* z, int num_sms, cudaStream_t st) {
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+  const bool wide = (L.P >= 64LL * s.E);  // many rows per expert: 256-wide tiles
+  CUtensorMap tA1, tB1, tA2, tB2;
+  const uint32_t bn = wide ? 256 : 128;
+  if (!make_tmap(&tA1, x_perm, (uint64_t)x_rows, (uint64_t)s.d, kGemmBM) ||
+      !make_tmap(&tB1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, bn / 2) ||
+      !make_tmap(&tA2, h, (uint64_t)L.Ppad, (uint64_t)s.f, kGemmBM) ||
+      !make_tmap(&tB2, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, bn))
+    return MOE_ERR_CUDA;
+  const int nt1 = (int)((s.f + bn / 2 - 1) / (bn / 2));
+  const int nt2 = (int)((s.d + bn - 1) / bn);
+  cudaError_t e;
+  if (wide) {
+    e = launch_gemm_t<256, true>(tA1, tB1, tiles, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
+                                 s.f, s.f, h, s.f, err, num_sms, st);
+    if (e == cudaSuccess)
+      e = launch_gemm_t<256, false>(tA2, tB2, tiles, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
+                                    s.d, z, s.d, err, num_sms, st);
+  } else {
+    e = launch_gemm_t<128, true>(tA1, tB1, tiles, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
+                                 s.f, s.f, h, s.f, err, num_sms, st);
+    if (e == cudaSuccess)
+      e = launch_gemm_t<128, false>(tA2, tB2, tiles, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
+                                    s.d, z, s.d, err, num_sms, st);
+  }
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

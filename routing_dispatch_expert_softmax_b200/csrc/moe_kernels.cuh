@@ -1,0 +1,35 @@
+// Internal launchers shared by the C ABI (moe_abi.cu) and the kernel files.
+#pragma once
+
+#include <algorithm>
+#include <climits>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+cudaError_t launch_router_partial(const __nv_bfloat16* x, const float* w_g,
+                                  const moe_shape& s, int split, float* part,
+                                  cudaStream_t st);
+cudaError_t launch_router_finish(const float* part, int split, const float* bias,
+                                 const moe_shape& s, float* logits, cudaStream_t st);
+cudaError_t launch_topk(const float* part, int split, const float* bias,
+                        const moe_shape& s, float* logits_out, int* idx, float* w,
+                        cudaStream_t st);
+cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayout& L,
+                                char* ws, int* counts, int* offsets, int* row_of,
+                                int* perm, int* send, int* rank_off, cudaStream_t st);
+cudaError_t launch_tiles_from_offsets(const int* offsets, const moe_shape& s,
+                                      int* tiles, int* err, cudaStream_t st);
+cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, int T,
+                          int d, __nv_bfloat16* x_perm, int* err, cudaStream_t st);
+cudaError_t launch_selftest_bounded_wait(unsigned long long limit_ns, int* err,
+                                         cudaStream_t st);
+cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const float* w,
+                           const moe_shape& s, __nv_bfloat16* y, cudaStream_t st);
+int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
+                      const __nv_bfloat16* w13, const __nv_bfloat16* w2,
+                      const moe_shape& s, const WsLayout& L, char* ws,
+                      __nv_bfloat16* z, int num_sms, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,136 @@
+"""Host-side tests of the C ABI: the library loads, exports every symbol the
+header declares, sizes workspaces, and rejects bad arguments before any
+launch.  None of these calls reaches a kernel, so they are safe anywhere."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import routing_dispatch_expert_softmax_b200 as moe
+from routing_dispatch_expert_softmax_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return B.load_library()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_what_the_binding_knows():
+    assert _declared_functions() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_error_strings(lib):
+    assert moe.moe_version() == 100
+    for code in range(6):
+        assert moe.moe_error_string(code).startswith("MOE_")
+    assert "unknown" in moe.moe_error_string(99)
+
+
+VALID = dict(T=64, d=256, E=8, k=2, f=512, R=0)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=-1), dict(T=(1 << 20) + 1), dict(d=0), dict(d=96), dict(d=16448),
+    dict(E=0), dict(E=1025), dict(k=0), dict(k=9), dict(k=33, E=64),
+    dict(f=0), dict(f=100), dict(R=-1), dict(R=3), dict(R=65),
+])
+def test_workspace_size_rejects_invalid_shapes(lib, bad):
+    s = dict(VALID, **bad)
+    assert moe.moe_workspace_size(B.MoEShape.of(**s)) == 0
+
+
+def test_workspace_size_grows_with_T(lib):
+    sizes = [moe.moe_workspace_size(B.MoEShape.of(**dict(VALID, T=t))) for t in (0, 1, 64, 4096)]
+    assert all(s > 0 for s in sizes)
+    assert sizes == sorted(sizes)
+    assert moe.moe_workspace_size(B.MoEShape.of(**dict(VALID, E=8, R=4))) > 0
+
+
+def _raw(lib, name, *args):
+    return getattr(lib, name)(*args)
+
+
+def _P(v):
+    return ctypes.c_void_p(v)
+
+
+A16 = 1 << 20          # an aligned fake address (never dereferenced)
+MIS = (1 << 20) + 2    # misaligned
+
+
+def test_bad_arguments_are_rejected_before_launch(lib):
+    s = ctypes.byref(B.MoEShape.of(**VALID))
+    bad_shape = ctypes.byref(B.MoEShape.of(**dict(VALID, k=0)))
+    INV = B.MOE_ERR_INVALID_ARG
+    # moe_router: null / misaligned x, null logits, invalid shape
+    assert _raw(lib, "moe_router", None, _P(A16), None, s, _P(A16), None) == INV
+    assert _raw(lib, "moe_router", _P(MIS), _P(A16), None, s, _P(A16), None) == INV
+    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, s, None, None) == INV
+    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, bad_shape, _P(A16), None) == INV
+    # moe_topk
+    assert _raw(lib, "moe_topk", None, s, _P(A16), _P(A16), None) == INV
+    assert _raw(lib, "moe_topk", _P(A16 + 1), s, _P(A16), _P(A16), None) == INV
+    # moe_dispatch: send_counts without R > 1, misaligned workspace
+    args = [_P(A16)] * 2
+    assert _raw(lib, "moe_dispatch", *args, s, *[_P(A16)] * 5, _P(A16), None, _P(A16),
+                None) == INV
+    assert _raw(lib, "moe_dispatch", *args, s, *[_P(A16)] * 5, None, None, _P(A16 + 16),
+                None) == INV
+    # moe_ffn: misaligned weights, null workspace
+    assert _raw(lib, "moe_ffn", _P(A16), _P(A16), _P(MIS), _P(A16), s, _P(A16), _P(A16),
+                None) == INV
+    assert _raw(lib, "moe_ffn", _P(A16), _P(A16), _P(A16), _P(A16), s, _P(A16), None,
+                None) == INV
+    # moe_combine
+    assert _raw(lib, "moe_combine", _P(A16), None, _P(A16), s, _P(A16), None) == INV
+    # moe_forward: null workspace, misaligned y
+    assert _raw(lib, "moe_forward", *[_P(A16)] * 5, s, _P(A16), None, None, None, None,
+                None) == INV
+    assert _raw(lib, "moe_forward", *[_P(A16)] * 5, s, _P(MIS), None, None, None, _P(A16),
+                None) == INV
+    # self-test limits
+    assert _raw(lib, "moe_selftest_bounded_wait", ctypes.c_longlong(0), _P(A16), None) == INV
+    assert _raw(lib, "moe_selftest_bounded_wait", ctypes.c_longlong(2 * 10 ** 9), _P(A16),
+                None) == INV
+    assert _raw(lib, "moe_check", _P(A16 + 8), None) == INV
+
+
+def test_empty_batch_is_a_no_op(lib):
+    s0 = ctypes.byref(B.MoEShape.of(**dict(VALID, T=0)))
+    # T = 0 launches nothing, so even null activation pointers are accepted.
+    assert _raw(lib, "moe_router", None, None, None, s0, None, None) == B.MOE_OK
+    assert _raw(lib, "moe_topk", None, s0, None, None, None) == B.MOE_OK
+    assert _raw(lib, "moe_combine", None, None, None, s0, None, None) == B.MOE_OK
+    assert _raw(lib, "moe_forward", *[None] * 5, s0, None, None, None, None, _P(A16),
+                None) == B.MOE_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_no_cpu_fallback_without_a_gpu(lib):
+    s = ctypes.byref(B.MoEShape.of(**VALID))
+    # Valid arguments but no device: the library refuses, it never computes on the CPU.
+    assert _raw(lib, "moe_topk", _P(A16), s, _P(A16), _P(A16), None) == B.MOE_ERR_CUDA
+    assert _raw(lib, "moe_forward", *[_P(A16)] * 5, s, _P(A16), None, None, None, _P(A16),
+                None) == B.MOE_ERR_CUDA
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.moe_combine(x, x, x, x, B.MoEShape.of(4, 64, 8, 1, 64))
