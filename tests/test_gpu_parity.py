@@ -333,7 +333,7 @@ def _check_forward(cfg, sample=None, seed=0):
     for i, t in enumerate(toks):
         ref_w = dict(zip(ref["idx"][i].tolist(), ref["w"][i].tolist()))
         for j, e in enumerate(idx_h[t].tolist()):
-            assert abs(got_w[t, j] - ref_w[e]) <= 4 * delta[i].max() + 2e-6
+            assert abs(got_w[i, j] - ref_w[e]) <= 4 * delta[i].max() + 2e-6
     rel = assert_layer_close(y[torch.from_numpy(toks).long().to(DEV)], ref["y"],
                              f"moe_forward {cfg.name}")
     return rel, flips
