@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 routed MoE layer forward.
+
+One step = one full layer forward (router, top-k, dispatch, expert SwiGLU
+GEMMs, combine) over one batch of seeded synthetic tokens, through the C ABI.
+Default workload: the Qwen3-30B-A3B-shaped decode step (T=64 concurrent
+tokens, d=2048, E=128 experts, top-8, f=768, Zipf(1.0) expert skew), the
+configuration the HBM-roofline metric is quoted on.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--T T]
+
+Device timing: W untimed steps, then K steps each bracketed by CUDA events on
+the launch stream (stage boundaries come from moe_forward_staged); L2 is
+flushed before every step, outside the events.  Under torchrun every rank runs
+its own batch with the same weights (replicas; weak scaling, no data-path
+collective); the time is the max over ranks.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; % of HBM (decode) or BF16 tensor-core (prefill) roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["routing_dispatch_expert_softmax_b200/csrc/moe_gemm_sm100.cu",
+                  "routing_dispatch_expert_softmax_b200/csrc/moe_common.cuh",
+                  "routing_dispatch_expert_softmax_b200/csrc/moe_routing.cu"]
+# Kernels one moe_forward launches (router, top-k, histogram, scan, scatter,
+# gather, GEMM1, GEMM2, combine).
+LAUNCHES_PER_FORWARD = 9
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="qwen3-30b-a3b-decode")
+    p.add_argument("--T", type=int, default=None, help="override the token count")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            pk = json.load(fh)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload_key, kernel):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, or None
+    when there is none or the kernel sources changed since it was taken."""
+    try:
+        with open(PROFILE_TRAFFIC) as fh:
+            tab = json.load(fh)
+        ent = tab[workload_key][kernel]
+        if ent.get("source_hash") != kernel_source_hash():
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def workload_config(name, T):
+    from routing_dispatch_expert_softmax_b200 import workloads as wl
+    if name not in wl.CONFIGS:
+        raise SystemExit(f"unknown workload {name!r}; choose from {sorted(wl.CONFIGS)}")
+    cfg = wl.CONFIGS[name]
+    return cfg.with_T(T) if T is not None else cfg
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            ident = self._ident()
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def _ident(self):
+        import torch
+        try:
+            u = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return str(self.dev)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.strip().split(",") for r in self.tmp.read().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(dist, value, device):
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(dist, value, device):
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((int(i.get("num_threads", 0)) for i in info), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample_run(cfg, host, tokens):
+    """One oracle pass over the given tokens of the batch (fp64, CPU)."""
+    import oracle
+    return oracle.moe_forward(host["x"][tokens], host["w_g"], host["bias"], host["w13"],
+                              host["w2"], cfg.k)
+
+
+def host_inputs_for_oracle(cfg, dev_inputs, tokens):
+    """Copies what the oracle reads to host memory before any timing: the
+    sample's hidden rows, the router, and the experts the sample touches (the
+    oracle widens them to fp64 itself, inside the timed region)."""
+    import numpy as np
+
+    import oracle
+    f32 = lambda t: None if t is None else t.float().cpu().numpy()
+    x = f32(dev_inputs["x"])
+    w_g, bias = f32(dev_inputs["w_g"]), f32(dev_inputs["bias"])
+    L = oracle.router_logits(x[tokens], w_g, bias)
+    touched = np.unique(oracle.topk_select_sorted(L.astype(np.float32), cfg.k))
+
+    class Experts(dict):
+        pass
+
+    w13, w2 = Experts(), Experts()
+    for e in touched.tolist():
+        w13[e] = f32(dev_inputs["w13"][e])
+        w2[e] = f32(dev_inputs["w2"][e])
+    return {"x": x, "w_g": w_g, "bias": bias, "w13": w13, "w2": w2}
+
+
+def cpu_baseline(cfg, dev_inputs, budget_s=12.0):
+    """The oracle as it stands, timed on this host's cores on a bounded sample
+    of the same batch (tokens/s)."""
+    import numpy as np
+    n = min(cfg.T, 16)
+    tokens = np.arange(n)
+    host = host_inputs_for_oracle(cfg, dev_inputs, tokens)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle_sample_run(cfg, host, tokens)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= 64 * n:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"first {n} tokens of the {cfg.name} T={cfg.T} batch, repeated "
+                      f"{done // n}x ({el:.1f} s); fp64 NumPy, experts widened per call"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle on the same workload, bounded
+    samples per step; rank 0 only."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+
+    from routing_dispatch_expert_softmax_b200 import workloads as wl
+    cfg = workload_config(args.workload, args.T)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inputs = wl.make_layer(cfg, dev, 0)
+    n = min(cfg.T, 8)
+    host = host_inputs_for_oracle(cfg, inputs, np.arange(cfg.T))
+    del inputs
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        oracle_sample_run(cfg, host, rng.choice(cfg.T, n, replace=False))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_run(cfg, host, rng.choice(cfg.T, n, replace=False))
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "step_sample_tokens": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} random tokens of the {cfg.name} T={cfg.T} batch "
+                                   f"per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def algorithmic(cfg, touched):
+    """Algorithmic bytes and flops of one layer call: the touched experts'
+    weights, the router weight (+bias), x read and y written; flops of the
+    expert FFN and router.  Intermediates (x_perm, h, z) are not counted."""
+    wbytes = touched * 3 * cfg.d * cfg.f * 2
+    router = cfg.d * cfg.E * 4 + (cfg.E * 4 if cfg.zipf_s is not None else 0)
+    act = cfg.T * cfg.d * 2 * 2
+    flops = 6 * cfg.P * cfg.d * cfg.f + 2 * cfg.T * cfg.d * cfg.E
+    return {"bytes": wbytes + router + act, "flops": flops,
+            "gemm1_bytes": touched * 2 * cfg.f * cfg.d * 2,
+            "gemm2_bytes": touched * cfg.f * cfg.d * 2,
+            "gemm1_flops": 4 * cfg.P * cfg.d * cfg.f, "gemm2_flops": 2 * cfg.P * cfg.d * cfg.f}
+
+
+def run_ours(args):
+    import torch
+
+    import routing_dispatch_expert_softmax_b200 as moe
+    from routing_dispatch_expert_softmax_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    moe.load_library()
+    cfg = workload_config(args.workload, args.T)
+    peaks, peak_src = load_peaks()
+
+    # Same weights on every rank (replicas), a different batch per rank.
+    w_g, bias = wl.make_router(cfg, dev, 0)
+    w13, w2 = wl.make_experts(cfg, dev, 0)
+    x = wl.make_hidden(cfg, dev, rank)
+    layer = moe.MoELayer(w_g, bias, w13, w2, cfg.k, cfg.R)
+    shape = layer.shape(cfg.T)
+    ws = moe.workspace(shape, dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events):
+        flush.zero_()  # evict L2; outside the step's events
+        moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, events, stream)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    warm = [[ev() for _ in range(moe.MOE_STAGE_EVENTS)] for _ in range(max(args.warmup, 1))]
+    for i in range(args.warmup):
+        step(warm[i])
+    torch.cuda.synchronize(dev)
+    st = moe.moe_check(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(moe.moe_error_string(st))
+
+    # ---------------- timed region (device)
+    events = [[ev() for _ in range(moe.MOE_STAGE_EVENTS)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for i in range(args.steps):
+        step(events[i])
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[-1]) for e in events]
+    stage_ms = [[e[s].elapsed_time(e[s + 1]) for s in range(moe.MOE_STAGE_EVENTS - 1)]
+                for e in events]
+    total_ms = max_over_ranks(dist, sum(step_ms), dev)
+    ms_per_step = total_ms / args.steps
+    tokens = sum_over_ranks(dist, cfg.T * args.steps, dev)
+    value = tokens / (total_ms / 1e3)
+    st = moe.moe_check(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(moe.moe_error_string(st))
+
+    # ---------------- end to end through the public API, host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    y_dev = torch.empty_like(y)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, out=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e2e_ev = [(ev(), ev()) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, out=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+        e2e_ev[i][1].synchronize()  # the host reads the result every step
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e2e_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in e2e_ev), dev)
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    # ---------------- roofline of the dominant kernel
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    layer(x, out=y_dev, counts_out=counts)
+    touched = int((counts > 0).sum().item())
+    alg = algorithmic(cfg, touched)
+    mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
+    names = ["router_topk", "dispatch_gather", "gemm1_swiglu", "gemm2", "combine"]
+    dom = max(range(len(mean_stage)), key=lambda j: mean_stage[j])
+    tokens_per_expert = cfg.P / cfg.E
+    decode = tokens_per_expert < 64
+    kern = names[dom]
+    t_kern = mean_stage[dom] / 1e3
+    if kern in ("gemm1_swiglu", "gemm2") and not decode:
+        fl = alg["gemm1_flops"] if kern == "gemm1_swiglu" else alg["gemm2_flops"]
+        achieved = fl / t_kern / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        by = {"gemm1_swiglu": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(
+            kern, cfg.T * cfg.d * 2 * 2)
+        achieved = by / t_kern / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
+    roof["kernel"] = kern
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    roof["traffic"] = profiled_traffic(f"{cfg.name}@T{cfg.T}", kern)
+    t_layer = ms_per_step / 1e3
+    layer_roof = {
+        "bytes": alg["bytes"], "flops": alg["flops"], "touched_experts": touched,
+        "hbm_frac_measured": alg["bytes"] / t_layer / (peaks["hbm_gbs"] * 1e9),
+        "hbm_frac_spec_8TBs": alg["bytes"] / t_layer / 8e12,
+        "tensor_frac_measured": alg["flops"] / t_layer / (peaks["bf16_tflops"] * 1e12),
+        "tensor_frac_spec_2250TF": alg["flops"] / t_layer / 2.25e15,
+        "bound": "hbm" if decode else "tensor",
+    }
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "R": cfg.R, "zipf_s": cfg.zipf_s,
+                   "global_batch": cfg.T * world, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+        "roofline": roof,
+        "layer_roofline": layer_roof,
+        "stage_ms": dict(zip(names, mean_stage)),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * cfg.d * 2,
+                "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+        "gpu_launches": LAUNCHES_PER_FORWARD * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, {"x": x, "w_g": w_g, "bias": bias,
+                                                  "w13": w13, "w2": w2})
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -28,7 +28,7 @@ MOE_ERR_DEVICE_CHECK = 5
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router",
            "moe_topk", "moe_dispatch", "moe_ffn", "moe_combine", "moe_forward",
-           "moe_selftest_bounded_wait", "moe_check")
+           "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check")
 
 
 class MoEError(RuntimeError):
@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_combine.argtypes = [_P, _P, _P, _S, _P, _P]
     lib.moe_forward.restype = ctypes.c_int
     lib.moe_forward.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P]
+    lib.moe_forward_staged.restype = ctypes.c_int
+    lib.moe_forward_staged.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _P, _P]
     lib.moe_check.restype = ctypes.c_int
     lib.moe_check.argtypes = [_P, _P]
     lib.moe_selftest_bounded_wait.restype = ctypes.c_int
@@ -187,6 +189,40 @@ def moe_forward(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, idx_out=None, w_o
         _ptr(idx_out, torch.int32, "idx_out"), _ptr(w_out, torch.float32, "w_out"),
         _ptr(counts_out, torch.int32, "counts_out"), _ptr(ws, torch.uint8, "ws"),
         _stream(stream)), "moe_forward")
+
+
+MOE_STAGE_EVENTS = 6
+STAGE_NAMES = ("router+topk", "dispatch+gather", "expert GEMM1+SwiGLU",
+               "expert GEMM2", "combine")
+
+
+def _event_handle(ev) -> int:
+    try:
+        return int(ev.cuda_event)
+    except Exception:
+        return 0
+
+
+def moe_forward_staged(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, events, stream=None):
+    """``events``: MOE_STAGE_EVENTS torch.cuda.Event objects (or None entries)
+    recorded at the stage boundaries on the launch stream."""
+    if len(events) != MOE_STAGE_EVENTS:
+        raise ValueError(f"need {MOE_STAGE_EVENTS} events")
+    st = torch.cuda.current_stream() if stream is None else stream
+    handles = []
+    for ev in events:
+        if ev is None:
+            handles.append(None)
+            continue
+        if not _event_handle(ev):
+            ev.record(st)  # torch creates the CUDA event at its first record
+        handles.append(ctypes.c_void_p(_event_handle(ev)))
+    arr = (ctypes.c_void_p * MOE_STAGE_EVENTS)(*handles)
+    _check(load_library().moe_forward_staged(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.bfloat16, "w13"),
+        _ptr(w2, torch.bfloat16, "w2"), ctypes.byref(shape), _ptr(y, torch.bfloat16, "y"),
+        _ptr(ws, torch.uint8, "ws"), arr, _stream(st)), "moe_forward_staged")
 
 
 def moe_selftest_bounded_wait(limit_ns: int, ws, stream=None):

@@ -181,9 +181,10 @@ int moe_combine(const moe_bf16* z, const int32_t* row_of, const float* w, const 
                                     static_cast<cudaStream_t>(stream)));
 }
 
-int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const moe_bf16* w13,
-                const moe_bf16* w2, const moe_shape* s, moe_bf16* y, int32_t* idx_out,
-                float* w_out, int32_t* counts_out, void* ws, void* stream) {
+static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
+                        const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
+                        moe_bf16* y, int32_t* idx_out, float* w_out, int32_t* counts_out,
+                        void* ws, void* stream, void* const* events) {
   if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
   if (s->T == 0) return MOE_OK;
@@ -195,6 +196,10 @@ int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const mo
   int st = device_check(&sms);
   if (st != MOE_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> cudaError_t {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), cs);
+  };
   const WsLayout L = ws_layout(*s, sms);
   char* wsb = static_cast<char*>(ws);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
@@ -208,19 +213,38 @@ int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const mo
   __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
   __nv_bfloat16* z = at<__nv_bfloat16>(ws, L.z);
 
-  cudaError_t e = launch_router_partial(xb, w_g, *s, 1, logits, cs);
+  cudaError_t e = mark(0);
+  if (e == cudaSuccess) e = launch_router_partial(xb, w_g, *s, 1, logits, cs);
   if (e == cudaSuccess) e = launch_topk(logits, 1, bias, *s, nullptr, idx, gw, cs);
+  if (e == cudaSuccess) e = mark(1);
   if (e == cudaSuccess)
     e = launch_route_tables(idx, *s, L, wsb, counts, offsets, row_of, perm,
                             at<int>(ws, L.send), at<int>(ws, L.rank_off), cs);
   if (e == cudaSuccess)
     e = launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
+  if (e == cudaSuccess) e = mark(2);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   int r = launch_expert_ffn(x_perm, L.Ppad, reinterpret_cast<const __nv_bfloat16*>(w13),
                             reinterpret_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms,
-                            cs);
+                            cs, events ? events + 3 : nullptr);
   if (r != MOE_OK) return r;
-  return cuda_status(launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs));
+  e = launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs);
+  if (e == cudaSuccess) e = mark(5);
+  return cuda_status(e);
+}
+
+int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const moe_bf16* w13,
+                const moe_bf16* w2, const moe_shape* s, moe_bf16* y, int32_t* idx_out,
+                float* w_out, int32_t* counts_out, void* ws, void* stream) {
+  return forward_impl(x, w_g, bias, w13, w2, s, y, idx_out, w_out, counts_out, ws, stream,
+                      nullptr);
+}
+
+int moe_forward_staged(const moe_bf16* x, const float* w_g, const float* bias,
+                       const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
+                       moe_bf16* y, void* ws, void* const* events, void* stream) {
+  return forward_impl(x, w_g, bias, w13, w2, s, y, nullptr, nullptr, nullptr, ws, stream,
+                      events);
 }
 
 int moe_selftest_bounded_wait(long long limit_ns, void* ws, void* stream) {

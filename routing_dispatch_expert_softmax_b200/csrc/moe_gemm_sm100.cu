@@ -320,7 +320,13 @@ static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
 int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                       const moe_shape& s, const WsLayout& L, char* ws,
-                      __nv_bfloat16* z, int num_sms, cudaStream_t st) {
+                      __nv_bfloat16* z, int num_sms, cudaStream_t st,
+                      void* const* events) {
+  // events (optional): [0] recorded after GEMM1, [1] after GEMM2.
+  auto mark = [&](int i) -> cudaError_t {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+  };
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
@@ -338,16 +344,19 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
   if (wide) {
     e = launch_gemm_t<256, true>(tA1, tB1, tiles, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
                                  s.f, s.f, h, s.f, err, num_sms, st);
+    if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_gemm_t<256, false>(tA2, tB2, tiles, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
                                     s.d, z, s.d, err, num_sms, st);
   } else {
     e = launch_gemm_t<128, true>(tA1, tB1, tiles, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
                                  s.f, s.f, h, s.f, err, num_sms, st);
+    if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_gemm_t<128, false>(tA2, tB2, tiles, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
                                     s.d, z, s.d, err, num_sms, st);
   }
+  if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

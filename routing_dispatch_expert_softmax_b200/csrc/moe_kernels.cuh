@@ -30,6 +30,7 @@ cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const floa
 int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                       const moe_shape& s, const WsLayout& L, char* ws,
-                      __nv_bfloat16* z, int num_sms, cudaStream_t st);
+                      __nv_bfloat16* z, int num_sms, cudaStream_t st,
+                      void* const* events = nullptr);
 
 }  // namespace moe
