@@ -178,6 +178,35 @@ MOE_API int moe_forward_staged(const moe_bf16* x, const float* w_g, const float*
                                const moe_shape* s, moe_bf16* y, void* ws,
                                void* const* events, void* stream);
 
+/* Dispatch without a workspace.  No counterpart in the pages: this is a
+ * library convenience for callers that cannot allocate device memory when
+ * they dispatch -- code running after a fixed memory pool has been carved
+ * out, runtimes that only hand a plugin its inputs and outputs, or hosts
+ * whose allocator may not be called from the dispatching thread.
+ * Same arguments, layout and results as moe_dispatch, minus `ws`: the
+ * per-block histograms, bases, send counts, tile list and error word live in
+ * one file-scope device array of MOE_NOALLOC_SCRATCH bytes, which every GPU
+ * that loads the library holds until the process exits.  The call allocates
+ * nothing (no cudaMalloc / cudaFree, no allocating library routine).
+ *   - A shape whose scratch would exceed MOE_NOALLOC_SCRATCH is rejected with
+ *     MOE_ERR_UNSUPPORTED before anything is launched (e.g. T = 16384,
+ *     E = 256, R = 8 needs about 160 KB; T = 1<<20 with E = 256 does not fit).
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     the error word is cleared at the start of each call and the rest is
+ *     rewritten.  Calls that overlap on the GPU (other streams, other threads)
+ *     race on it and must be serialised by the caller.
+ *   - There is no error word to read back: rejected expert ids (out of range
+ *     or repeated within a token) are not counted, so they show as
+ *     offsets[E] < T*k. */
+#define MOE_NOALLOC_SCRATCH (2u << 20)
+MOE_API int moe_dispatch_noalloc(const int32_t* idx, const moe_bf16* x, const moe_shape* s,
+                                 int32_t* counts, int32_t* offsets, int32_t* perm,
+                                 int32_t* row_of, moe_bf16* x_perm, int32_t* send_counts,
+                                 int32_t* rank_offsets, void* stream);
+
 /* Self-test of the failure path every device-side wait uses: launches one
  * kernel that waits on a barrier nothing will ever complete, through the same
  * bounded wait as the expert-GEMM pipeline, with a limit of limit_ns

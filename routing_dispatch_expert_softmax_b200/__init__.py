@@ -9,7 +9,7 @@ combine -- as hand-written CUDA kernels behind a C ABI (``include/moe.h``,
 from .binding import (EXPORTS, MOE_STAGE_EVENTS, STAGE_NAMES, MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK,  # noqa: F401
                       MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED,
                       MOE_OK, MoEError, MoEShape, load_library, moe_check,
-                      moe_combine, moe_dispatch, moe_error_string, moe_ffn,
+                      moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_error_string, moe_ffn,
                       moe_forward, moe_forward_staged, moe_router, moe_selftest_bounded_wait,
                       moe_topk, moe_version,
                       moe_workspace_size, workspace)

@@ -28,7 +28,8 @@ MOE_ERR_DEVICE_CHECK = 5
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router",
            "moe_topk", "moe_dispatch", "moe_ffn", "moe_combine", "moe_forward",
-           "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check")
+           "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check",
+           "moe_dispatch_noalloc")
 
 
 class MoEError(RuntimeError):
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_forward.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P]
     lib.moe_forward_staged.restype = ctypes.c_int
     lib.moe_forward_staged.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _P, _P]
+    lib.moe_dispatch_noalloc.restype = ctypes.c_int
+    lib.moe_dispatch_noalloc.argtypes = [_P, _P, _S, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.moe_check.restype = ctypes.c_int
     lib.moe_check.argtypes = [_P, _P]
     lib.moe_selftest_bounded_wait.restype = ctypes.c_int
@@ -163,6 +166,21 @@ def moe_dispatch(idx, x, counts, offsets, perm, row_of, x_perm, shape: MoEShape,
         _ptr(send_counts, torch.int32, "send_counts"),
         _ptr(rank_offsets, torch.int32, "rank_offsets"),
         _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_noalloc(idx, x, counts, offsets, perm, row_of, x_perm, shape: MoEShape,
+                         send_counts=None, rank_offsets=None, stream=None):
+    """moe_dispatch for callers that cannot allocate: the scratch is the
+    library's own fixed device array, so no workspace is passed (calls must
+    not overlap on the GPU)."""
+    _check(load_library().moe_dispatch_noalloc(
+        _ptr(idx, torch.int32, "idx"), _ptr(x, torch.bfloat16, "x"), ctypes.byref(shape),
+        _ptr(counts, torch.int32, "counts"), _ptr(offsets, torch.int32, "offsets"),
+        _ptr(perm, torch.int32, "perm"), _ptr(row_of, torch.int32, "row_of"),
+        _ptr(x_perm, torch.bfloat16, "x_perm"),
+        _ptr(send_counts, torch.int32, "send_counts"),
+        _ptr(rank_offsets, torch.int32, "rank_offsets"), _stream(stream)),
+        "moe_dispatch_noalloc")
 
 
 def moe_ffn(x_perm, offsets, w13, w2, z, shape: MoEShape, ws, stream=None):
