@@ -167,11 +167,14 @@ MOE_API int moe_forward(const moe_bf16* x, const float* w_g, const float* bias,
 /* moe_forward with stage timing: the same launches on the same stream, plus
  * cudaEventRecord(events[i], stream) at the stage boundaries so a caller can
  * time each stage with CUDA events inside a timed region (or a graph):
- *   events[0] before the router      events[3] after expert GEMM1 (+SwiGLU)
- *   events[1] after top-k selection  events[4] after expert GEMM2
- *   events[2] after dispatch+gather  events[5] after the combine
+ *   events[0] before the router        events[3] after expert GEMM1 (+SwiGLU)
+ *   events[1] after the router         events[4] after expert GEMM2
+ *   events[2] after top-k, dispatch    events[5] after the combine
+ *             tables and row gather
  * `events` points to MOE_STAGE_EVENTS cudaEvent_t handles (any may be NULL,
- * then it is skipped).  Routing outputs stay in the workspace. */
+ * then it is skipped).  The records use cudaEventRecordExternal, so under
+ * stream capture they become event-record nodes that fire on every replay.
+ * Routing outputs stay in the workspace. */
 #define MOE_STAGE_EVENTS 6
 MOE_API int moe_forward_staged(const moe_bf16* x, const float* w_g, const float* bias,
                                const moe_bf16* w13, const moe_bf16* w2,

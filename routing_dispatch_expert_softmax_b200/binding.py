@@ -210,7 +210,7 @@ def moe_forward(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, idx_out=None, w_o
 
 
 MOE_STAGE_EVENTS = 6
-STAGE_NAMES = ("router+topk", "dispatch+gather", "expert GEMM1+SwiGLU",
+STAGE_NAMES = ("router", "topk+dispatch+gather", "expert GEMM1+SwiGLU",
                "expert GEMM2", "combine")
 
 

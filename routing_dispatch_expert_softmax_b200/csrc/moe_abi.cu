@@ -96,9 +96,7 @@ int moe_router(const moe_bf16* x, const float* w_g, const float* bias, const moe
   if (st != MOE_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-  cudaError_t e = launch_router_partial(xb, w_g, *s, 1, logits, cs);
-  if (e == cudaSuccess && bias) e = launch_router_finish(logits, 1, bias, *s, logits, cs);
-  return cuda_status(e);
+  return cuda_status(launch_router(xb, w_g, bias, *s, logits, cs));
 }
 
 int moe_topk(const float* logits, const moe_shape* s, int32_t* idx, float* w, void* stream) {
@@ -108,8 +106,7 @@ int moe_topk(const float* logits, const moe_shape* s, int32_t* idx, float* w, vo
   int sms = 0;
   int st = device_check(&sms);
   if (st != MOE_OK) return st;
-  return cuda_status(launch_topk(logits, 1, nullptr, *s, nullptr, idx, w,
-                                 static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_topk(logits, *s, idx, w, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_dispatch(const int32_t* idx, const moe_bf16* x, const moe_shape* s, int32_t* counts,
@@ -198,7 +195,8 @@ static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
-    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), cs);
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), cs,
+                                    cudaEventRecordExternal);
   };
   const WsLayout L = ws_layout(*s, sms);
   char* wsb = static_cast<char*>(ws);
@@ -214,12 +212,20 @@ static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
   __nv_bfloat16* z = at<__nv_bfloat16>(ws, L.z);
 
   cudaError_t e = mark(0);
-  if (e == cudaSuccess) e = launch_router_partial(xb, w_g, *s, 1, logits, cs);
-  if (e == cudaSuccess) e = launch_topk(logits, 1, bias, *s, nullptr, idx, gw, cs);
+  if (e == cudaSuccess) e = launch_router(xb, w_g, bias, *s, logits, cs);
   if (e == cudaSuccess) e = mark(1);
-  if (e == cudaSuccess)
-    e = launch_route_tables(idx, *s, L, wsb, counts, offsets, row_of, perm,
-                            at<int>(ws, L.send), at<int>(ws, L.rank_off), cs);
+  if (e == cudaSuccess) {
+    if (s->T <= kFusedRouteMaxT) {
+      e = launch_route_fused(logits, *s, idx, gw, counts, offsets, at<int>(ws, L.tiles),
+                             at<int>(ws, L.send), at<int>(ws, L.rank_off), row_of, perm,
+                             at<int>(ws, L.err), cs);
+    } else {
+      e = launch_topk(logits, *s, idx, gw, cs);
+      if (e == cudaSuccess)
+        e = launch_route_tables(idx, *s, L, wsb, counts, offsets, row_of, perm,
+                                at<int>(ws, L.send), at<int>(ws, L.rank_off), cs);
+    }
+  }
   if (e == cudaSuccess)
     e = launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
   if (e == cudaSuccess) e = mark(2);

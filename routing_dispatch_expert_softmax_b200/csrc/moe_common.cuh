@@ -19,6 +19,9 @@ constexpr int kGemmBK = 64;                // K elements per pipeline stage
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 32;
 constexpr int kMaxR = 64;
+// Batches of at most this many tokens (so at most this many rows per expert)
+// run the expert GEMMs in swap-AB form.
+constexpr int kSwapMaxT = 256;
 
 // Device error word: ws[0] = first error code, ws[1] = detail (kernel id).
 enum : int { kErrSlot = 0, kErrDetail = 1 };
@@ -41,6 +44,16 @@ struct WsLayout {
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Work lists the routing kernels build for the expert GEMMs, in one int
+// buffer: [0] = number of 128-row tiles, [1] = number of touched experts,
+// then E entries (row0, row_end, expert) for the touched experts in expert
+// order, then the row tiles (row0, row_end, expert), 128 rows each.
+__host__ __device__ inline size_t tile_list_ints(int max_mtiles, int E) {
+  return 4 + 3 * ((size_t)max_mtiles + (size_t)E);
+}
+__host__ __device__ inline int* expert_entries(int* tiles) { return tiles + 4; }
+__host__ __device__ inline int* row_tile_entries(int* tiles, int E) { return tiles + 4 + 3 * E; }
 
 inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   WsLayout L{};
@@ -70,7 +83,7 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   L.rank_off = take(sizeof(int) * (R + 1));
   L.perm = take(sizeof(int) * L.P);
   L.row_of = take(sizeof(int) * L.P);
-  L.tiles = take(sizeof(int) * (4 + 3 * (size_t)L.max_mtiles));
+  L.tiles = take(sizeof(int) * tile_list_ints(L.max_mtiles, (int)E));
   L.x_perm = take(2 * (size_t)L.Ppad * d);
   L.h = take(2 * (size_t)L.Ppad * f);
   L.z = take(2 * (size_t)L.P * d);

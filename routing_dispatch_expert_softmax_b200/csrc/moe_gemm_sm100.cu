@@ -50,7 +50,7 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 template <int BN, bool SWIGLU>
 __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const int* __restrict__ tiles, int n_tiles, int K, int b_rows_per_expert,
+    const int* __restrict__ tiles, int E, int n_tiles, int K, int b_rows_per_expert,
     int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
     int* __restrict__ err) {
   using C = GemmCfg<BN, SWIGLU>;
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   const int num_mtiles = tiles[0];
   const int total = num_mtiles * n_tiles;
   const int nk = K / kGemmBK;
-  const int* tl = tiles + 4;
+  const int* tl = tiles + 4 + 3 * E;  // row tiles follow the E expert entries
 
   if (warp == 0) {
     if (lane == 0) {
@@ -256,6 +256,267 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ============================================================== small-batch kernel
+// Swap-AB form for batches of at most NMAX tokens per expert (decode): the
+// expert's weights are the M = 128 operand (128 weight rows per work item:
+// 64 gate + 64 up rows of Wg/Wu for GEMM1, 128 rows of Wd for GEMM2) and the
+// expert's n token rows are the N operand, N = 16 * ceil(n / 16) chosen per
+// item in the instruction descriptor.  Every K-stage then moves 16 KB of
+// weights and only 2 KB per 16 tokens, instead of a 128-row activation tile
+// that is mostly other experts' rows.  Work item = (touched expert, 128-row
+// weight tile).  D[weight row][token] sits in TMEM lanes x columns; GEMM1's
+// epilogue pairs gate lane j with up lane 64 + j through shared memory.
+template <int NMAX, bool SWIGLU>
+struct SwapCfg {
+  static constexpr int kStages = NMAX <= 64 ? 8 : 4;
+  static constexpr int kABytes = 128 * kGemmBK * 2;   // weights, 16 KB
+  static constexpr int kBBytes = NMAX * kGemmBK * 2;  // tokens
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * NMAX;
+  static constexpr int kXchBytes = SWIGLU ? 2 * 64 * 16 * 4 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kXchBytes + 1024 + 256;
+};
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+        "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+        "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int NMAX, bool SWIGLU>
+__global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
+    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+    const int* __restrict__ tiles, int n_tiles, int K, int w_rows_per_expert,
+    int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
+    int* __restrict__ err) {
+  using C = SwapCfg<NMAX, SWIGLU>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* xch = reinterpret_cast<float*>(smem + S * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kXchBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(&full[s2], 1);
+      mbar_init(&empty[s2], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tiles[1] * n_tiles;
+  const int nk = K / kGemmBK;
+  const int* et = tiles + 4;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int fills[S];
+#pragma unroll
+      for (int s2 = 0; s2 < S; ++s2) fills[s2] = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
+        const int row0 = et[3 * i + 0];
+        const int n = et[3 * i + 1] - row0;
+        const int e = et[3 * i + 2];
+        if (n < 1 || n > NMAX) continue;  // not a small-batch item (recorded by the epilogue)
+        const int nb = (n + 15) >> 4;
+        const int wrow = e * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
+        const uint32_t bytes = (uint32_t)(C::kABytes + nb * 16 * 128);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = smem + stage * C::kStageBytes;
+          uint8_t* b_dst = a_dst + C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          if (SWIGLU) {
+            tma_load_2d(a_dst, &tmW, &full[stage], kb * kGemmBK, wrow, pol_w);
+            tma_load_2d(a_dst + 64 * 128, &tmW, &full[stage], kb * kGemmBK, wrow + up_offset,
+                        pol_w);
+          } else {
+            tma_load_2d(a_dst, &tmW, &full[stage], kb * kGemmBK, wrow, pol_w);
+          }
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d(b_dst + b * 16 * 128, &tmX, &full[stage], kb * kGemmBK, row0 + 16 * b,
+                        pol_x);
+          ++fills[stage];
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+#pragma unroll
+        for (int s2 = 0; s2 < S; ++s2)
+          if (fills[s2] > 0)
+            mbar_wait_limit(&full[s2], (uint32_t)((fills[s2] - 1) & 1), 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
+        const int i = w / n_tiles;
+        const int n = et[3 * i + 1] - et[3 * i + 0];
+        if (n < 1 || n > NMAX) {
+          --it;  // skipped items use no accumulator buffer (same in the epilogue)
+          continue;
+        }
+        const uint32_t idesc = idesc_bf16_f32(128, ((n + 15) >> 4) * 16);
+        const int ab = it & 1;
+        const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(ab * NMAX);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk)
+            umma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                         sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit(&tfull[ab]);
+      }
+      if (*abort_flag) {
+        umma_commit(drain);
+        mbar_wait_limit(drain, 0, 100000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lanes q*32 .. q*32+31 = weight rows
+    int it = 0;
+    int chunk_parity = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+      const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
+      const int row0 = et[3 * i + 0];
+      const int n = et[3 * i + 1] - row0;
+      if (n < 1 || n > NMAX) {
+        if (threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
+        --it;  // the MMA warp skipped it too: no accumulator was used
+        continue;
+      }
+      const int ncols = ((n + 15) >> 4) * 16;
+      const int ab = it & 1;
+      const uint32_t aph = (uint32_t)((it >> 1) & 1);
+      mbar_wait_bounded(&tfull[ab], aph, abort_flag);
+      // The four epilogue warps decide together whether to go on, so none is
+      // left waiting at the exchange barrier below.
+      named_bar_sync(2, 128);
+      if (*abort_flag) break;
+      tc_fence_after();
+      const uint32_t t_addr = tmem_base + (uint32_t)(ab * NMAX) + ((uint32_t)(q * 32) << 16);
+      if (SWIGLU) {
+        // lanes 0..63: gate rows j, lanes 64..127: up rows j (j = lane & 63)
+        const int j = (q & 1) * 32 + lane;
+        const int col = nt * 64 + j;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          float* x = xch + chunk_parity * (64 * 16);
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_addr + c0, v);
+          tmem_ld_wait();
+          if (q >= 2) {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) x[cc * 64 + j] = __uint_as_float(v[cc]);
+          }
+          named_bar_sync(1, 128);
+          if (q < 2 && col < n_out) {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const int c = c0 + cc;
+              if (c < n) {
+                const float g = __uint_as_float(v[cc]);
+                const float u = x[cc * 64 + j];
+                out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(silu_f(g) * u);
+              }
+            }
+          }
+          chunk_parity ^= 1;
+        }
+      } else {
+        const int col = nt * 128 + q * 32 + lane;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_addr + c0, v);
+          tmem_ld_wait();
+          if (col < n_out) {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const int c = c0 + cc;
+              if (c < n)
+                out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0 && *abort_flag) record_error(err, MOE_ERR_TIMEOUT, 11);
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
 // ============================================================== host side
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                     void*, const cuuint64_t*, const cuuint64_t*,
@@ -295,7 +556,7 @@ static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t
 
 template <int BN, bool SWIGLU>
 static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
-                                 const int* tiles, int max_work, int n_tiles, int K,
+                                 const int* tiles, int E, int max_work, int n_tiles, int K,
                                  int b_rows, int up_off, int n_out, __nv_bfloat16* out,
                                  int ld_out, int* err, int num_sms, cudaStream_t st) {
   using C = GemmCfg<BN, SWIGLU>;
@@ -310,8 +571,72 @@ static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
   int grid = max_work < num_sms ? max_work : num_sms;
   if (grid < 1) grid = 1;
   k_grouped_gemm<BN, SWIGLU><<<grid, C::kThreads, C::kSmemBytes, st>>>(
-      ta, tb, tiles, n_tiles, K, b_rows, up_off, n_out, out, ld_out, err);
+      ta, tb, tiles, E, n_tiles, K, b_rows, up_off, n_out, out, ld_out, err);
   return cudaGetLastError();
+}
+
+template <int NMAX, bool SWIGLU>
+static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
+                                 const int* tiles, int max_work, int n_tiles, int K,
+                                 int w_rows, int up_off, int n_out, __nv_bfloat16* out,
+                                 int ld_out, int* err, int num_sms, cudaStream_t st) {
+  using C = SwapCfg<NMAX, SWIGLU>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_swap<NMAX, SWIGLU>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int grid = max_work < num_sms ? max_work : num_sms;
+  if (grid < 1) grid = 1;
+  k_expert_gemm_swap<NMAX, SWIGLU><<<grid, 192, C::kSmemBytes, st>>>(
+      tw, tx, tiles, n_tiles, K, w_rows, up_off, n_out, out, ld_out, err);
+  return cudaGetLastError();
+}
+
+// Small batches (every expert has at most 256 rows): both GEMMs in swap-AB form.
+static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
+                                  const __nv_bfloat16* w13, const __nv_bfloat16* w2,
+                                  const moe_shape& s, const WsLayout& L, char* ws,
+                                  __nv_bfloat16* z, int num_sms, cudaStream_t st,
+                                  void* const* events) {
+  auto mark = [&](int i) -> cudaError_t {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,
+                                    cudaEventRecordExternal);
+  };
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+  CUtensorMap tW1, tX1, tW2, tX2;
+  if (!make_tmap(&tW1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, 64) ||
+      !make_tmap(&tX1, x_perm, (uint64_t)x_rows, (uint64_t)s.d, 16) ||
+      !make_tmap(&tW2, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, 128) ||
+      !make_tmap(&tX2, h, (uint64_t)L.Ppad, (uint64_t)s.f, 16))
+    return MOE_ERR_CUDA;
+  const int nt1 = s.f / 64;               // 64 gate + 64 up rows per item
+  const int nt2 = (s.d + 127) / 128;      // 128 output columns per item
+  const int E = s.E;
+  cudaError_t e;
+  if (s.T <= 64) {
+    e = launch_swap_t<64, true>(tW1, tX1, tiles, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h, s.f,
+                                err, num_sms, st);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess)
+      e = launch_swap_t<64, false>(tW2, tX2, tiles, E * nt2, nt2, s.f, s.d, 0, s.d, z, s.d,
+                                   err, num_sms, st);
+  } else {
+    e = launch_swap_t<256, true>(tW1, tX1, tiles, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h,
+                                 s.f, err, num_sms, st);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess)
+      e = launch_swap_t<256, false>(tW2, tX2, tiles, E * nt2, nt2, s.f, s.d, 0, s.d, z, s.d,
+                                    err, num_sms, st);
+  }
+  if (e == cudaSuccess) e = mark(1);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // Both expert GEMMs over the rows described by the device tile list.
@@ -325,8 +650,11 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
   // events (optional): [0] recorded after GEMM1, [1] after GEMM2.
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
-    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,
+                                    cudaEventRecordExternal);
   };
+  if (s.T <= kSwapMaxT)
+    return launch_expert_ffn_swap(x_perm, x_rows, w13, w2, s, L, ws, z, num_sms, st, events);
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
@@ -342,18 +670,18 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
   const int nt2 = (int)((s.d + bn - 1) / bn);
   cudaError_t e;
   if (wide) {
-    e = launch_gemm_t<256, true>(tA1, tB1, tiles, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
+    e = launch_gemm_t<256, true>(tA1, tB1, tiles, s.E, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
                                  s.f, s.f, h, s.f, err, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
-      e = launch_gemm_t<256, false>(tA2, tB2, tiles, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
+      e = launch_gemm_t<256, false>(tA2, tB2, tiles, s.E, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
                                     s.d, z, s.d, err, num_sms, st);
   } else {
-    e = launch_gemm_t<128, true>(tA1, tB1, tiles, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
+    e = launch_gemm_t<128, true>(tA1, tB1, tiles, s.E, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
                                  s.f, s.f, h, s.f, err, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
-      e = launch_gemm_t<128, false>(tA2, tB2, tiles, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
+      e = launch_gemm_t<128, false>(tA2, tB2, tiles, s.E, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
                                     s.d, z, s.d, err, num_sms, st);
   }
   if (e == cudaSuccess) e = mark(1);

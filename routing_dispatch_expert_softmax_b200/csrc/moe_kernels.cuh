@@ -8,14 +8,16 @@
 
 namespace moe {
 
-cudaError_t launch_router_partial(const __nv_bfloat16* x, const float* w_g,
-                                  const moe_shape& s, int split, float* part,
-                                  cudaStream_t st);
-cudaError_t launch_router_finish(const float* part, int split, const float* bias,
-                                 const moe_shape& s, float* logits, cudaStream_t st);
-cudaError_t launch_topk(const float* part, int split, const float* bias,
-                        const moe_shape& s, float* logits_out, int* idx, float* w,
+cudaError_t launch_router(const __nv_bfloat16* x, const float* w_g, const float* bias,
+                          const moe_shape& s, float* logits, cudaStream_t st);
+cudaError_t launch_topk(const float* logits, const moe_shape& s, int* idx, float* w,
                         cudaStream_t st);
+// Selection + dispatch tables in one block; valid for T <= kFusedRouteMaxT.
+constexpr int kFusedRouteMaxT = 1024;
+cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
+                               int* counts, int* offsets, int* tiles, int* send,
+                               int* rank_off, int* row_of, int* perm, int* err,
+                               cudaStream_t st);
 cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayout& L,
                                 char* ws, int* counts, int* offsets, int* row_of,
                                 int* perm, int* send, int* rank_off, cudaStream_t st);

@@ -44,7 +44,7 @@ bool scratch_layout(const moe_shape& s, WsLayout* L) {
   L->blocksend = take(sizeof(int) * (size_t)L->nblocks * R * R);
   L->send = take(sizeof(int) * R * R);
   L->rank_off = take(sizeof(int) * (R + 1));
-  L->tiles = take(sizeof(int) * (4 + 3 * (size_t)L->max_mtiles));
+  L->tiles = take(sizeof(int) * tile_list_ints(L->max_mtiles, (int)E));
   L->total = o;
   return o <= kScratchBytes;
 }

@@ -8,70 +8,78 @@
 //   tile list, virtual-EP send counts) -> stable scatter (row_of, perm)
 //   -> row gather into the expert-major buffer ... expert FFNs ...
 //   -> gate-weighted combine.
+#include <cooperative_groups.h>
+
 #include "moe_kernels.cuh"
 
 namespace moe {
 
 // ============================================================== router GEMM
-// logit_part[s][t][e] = sum over the s-th K slice of x[t,i] * w_g[i,e].
-// Block: 16 tokens x 32 experts, 256 threads; thread = (2 tokens, 1 expert).
-constexpr int kRtT = 16, kRtE = 32, kRtK = 64;
+// logits[t,e] = sum_i x[t,i] * w_g[i,e] (+ bias[e]), fp32.
+// A thread-block cluster of CS CTAs owns a 32-token x 32-expert tile; CTA r
+// of the cluster accumulates the K slice [r*d/CS, (r+1)*d/CS) in fp32 FMA
+// order, the partial tiles meet in distributed shared memory, and CTA r then
+// sums output slice r over the CS partials in rank order 0..CS-1.  The order
+// is fixed, so every call with the same d gives the same bits, and nothing
+// leaves the SMs but the logits.
+constexpr int kRtT = 32, kRtE = 32, kRtKC = 128;
 
-__global__ void __launch_bounds__(256) k_router_partial(
-    const __nv_bfloat16* __restrict__ x, const float* __restrict__ w_g, int T,
-    int d, int E, int k_per_split, float* __restrict__ part) {
-  __shared__ float xs[kRtT][kRtK + 1];
-  __shared__ float ws[kRtK][kRtE];
-  const int t0 = blockIdx.x * kRtT;
-  const int e0 = blockIdx.y * kRtE;
-  const int split = blockIdx.z;
-  const int kbeg = split * k_per_split;
-  const int kend = min(d, kbeg + k_per_split);
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // ty in 0..7
-  float acc0 = 0.f, acc1 = 0.f;
-  for (int kc = kbeg; kc < kend; kc += kRtK) {
-    // x tile: 16 x 64 bf16
-    for (int i = threadIdx.x; i < kRtT * kRtK; i += 256) {
-      int r = i / kRtK, c = i % kRtK;
-      int t = t0 + r;
-      xs[r][c] = (t < T) ? __bfloat162float(x[(size_t)t * d + kc + c]) : 0.f;
+__global__ void __launch_bounds__(256) k_router_cluster(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ w_g,
+    const float* __restrict__ bias, int T, int d, int E, float* __restrict__ logits) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int CS = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  __shared__ float xs[kRtT][kRtKC];
+  __shared__ float ws[kRtKC][kRtE];
+  __shared__ float part[kRtT * kRtE];
+  const int e0 = (blockIdx.x / CS) * kRtE;
+  const int t0 = blockIdx.y * kRtT;
+  const int kslice = d / CS;
+  const int kbeg = rank * kslice, kend = kbeg + kslice;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int kc = kbeg; kc < kend; kc += kRtKC) {
+    const int chunk = min(kRtKC, kend - kc);  // 64 or 128
+    const int vpr = chunk / 8;                 // 16-byte vectors per token row
+    for (int v = threadIdx.x; v < kRtT * vpr; v += 256) {
+      const int r = v / vpr, c8 = (v - r * vpr) * 8;
+      const int t = t0 + r;
+      uint4 q = make_uint4(0, 0, 0, 0);
+      if (t < T) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + kc + c8));
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        xs[r][c8 + 2 * i] = f.x;
+        xs[r][c8 + 2 * i + 1] = f.y;
+      }
     }
-    // w tile: 64 x 32 fp32
-    for (int i = threadIdx.x; i < kRtK * kRtE; i += 256) {
-      int r = i / kRtE, c = i % kRtE;
-      int e = e0 + c;
-      ws[r][c] = (e < E) ? w_g[(size_t)(kc + r) * E + e] : 0.f;
+    for (int i = threadIdx.x; i < chunk * kRtE; i += 256) {
+      const int r = i / kRtE, c = i - r * kRtE;
+      const int e = e0 + c;
+      ws[r][c] = (e < E) ? __ldg(w_g + (size_t)(kc + r) * E + e) : 0.f;
     }
     __syncthreads();
-#pragma unroll 16
-    for (int kk = 0; kk < kRtK; ++kk) {
+    for (int kk = 0; kk < chunk; ++kk) {
       const float wv = ws[kk][tx];
-      acc0 = fmaf(xs[2 * ty][kk], wv, acc0);
-      acc1 = fmaf(xs[2 * ty + 1][kk], wv, acc1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(xs[ty + 8 * i][kk], wv, acc[i]);
     }
     __syncthreads();
   }
-  const int e = e0 + tx;
-  if (e < E) {
-    const int ta = t0 + 2 * ty, tb = ta + 1;
-    float* base = part + (size_t)split * T * E;
-    if (ta < T) base[(size_t)ta * E + e] = acc0;
-    if (tb < T) base[(size_t)tb * E + e] = acc1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) part[(ty + 8 * i) * kRtE + tx] = acc[i];
+  cl.sync();
+  const int per = (kRtT * kRtE) / CS;
+  for (int o = rank * per + threadIdx.x; o < (rank + 1) * per; o += 256) {
+    float v = 0.f;
+    for (int r = 0; r < CS; ++r) v += *cl.map_shared_rank(&part[o], r);
+    const int t = t0 + o / kRtE, e = e0 + (o % kRtE);
+    if (t < T && e < E) logits[(size_t)t * E + e] = bias ? v + bias[e] : v;
   }
-}
-
-// logits[t,e] = sum_s part[s][t][e] (+ bias[e]), fixed order s = 0..S-1.
-__global__ void k_router_finish(const float* __restrict__ part, int S,
-                                const float* __restrict__ bias, int T, int E,
-                                float* __restrict__ logits) {
-  const size_t n = (size_t)T * E;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x) {
-    float v = part[i];
-    for (int s = 1; s < S; ++s) v += part[(size_t)s * n + i];
-    if (bias) v += bias[i % E];
-    logits[i] = v;
-  }
+  cl.sync();  // partial tiles stay alive until every CTA has read them
 }
 
 // ============================================================== top-k
@@ -79,31 +87,20 @@ __global__ void k_router_finish(const float* __restrict__ part, int S,
 // warp-wide arg-max under the order (value desc, index asc) pick the slots in
 // order; the winner of round j is kept by lane j.  Gates are the softmax over
 // the k selected logits (equal to the full softmax renormalised over them).
+// Shared by k_topk and the fused small-batch routing kernel so both take the
+// same decisions.
 template <int VPL>
-__global__ void __launch_bounds__(256) k_topk(
-    const float* __restrict__ part, int S, const float* __restrict__ bias,
-    int T, int E, int k, float* __restrict__ logits_out, int* __restrict__ idx,
-    float* __restrict__ w) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const size_t n = (size_t)T * E;
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k,
+                                          int lane, int* __restrict__ idx_row,
+                                          float* __restrict__ w_row) {
   float v[VPL];
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
-    float s = 0.f;
-    if (e < E) {
-      const size_t o = (size_t)t * E + e;
-      s = part[o];
-      for (int sp = 1; sp < S; ++sp) s += part[(size_t)sp * n + o];
-      if (bias) s += bias[e];
-      if (logits_out) logits_out[o] = s;
-    } else {
-      taken |= 1u << i;  // not a candidate
-    }
-    v[i] = s;
+    v[i] = 0.f;
+    if (e < E) v[i] = row[e];
+    else taken |= 1u << i;  // not a candidate
   }
   float my_v = 0.f;
   int my_e = 0;
@@ -113,10 +110,9 @@ __global__ void __launch_bounds__(256) k_topk(
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       if (taken & (1u << i)) continue;
-      const int e = lane + 32 * i;
-      if (be == INT_MAX || v[i] > bv) {  // ascending e: equal keeps lower index
+      if (be == INT_MAX || v[i] > bv) {  // ascending e: equal keeps the lower index
         bv = v[i];
-        be = e;
+        be = lane + 32 * i;
       }
     }
 #pragma unroll
@@ -137,14 +133,24 @@ __global__ void __launch_bounds__(256) k_topk(
     }
   }
   const float top = __shfl_sync(0xffffffffu, my_v, 0);
-  float ex = (lane < k) ? expf(my_v - top) : 0.f;
+  const float ex = (lane < k) ? expf(my_v - top) : 0.f;
   float sum = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
   if (lane < k) {
-    idx[(size_t)t * k + lane] = my_e;
-    w[(size_t)t * k + lane] = ex / sum;
+    idx_row[lane] = my_e;
+    w_row[lane] = ex / sum;
   }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, int T, int E,
+                                              int k, int* __restrict__ idx,
+                                              float* __restrict__ w) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  warp_topk<VPL>(logits + (size_t)t * E, E, k, threadIdx.x & 31, idx + (size_t)t * k,
+                 w + (size_t)t * k);
 }
 
 // ============================================================== histogram
@@ -211,6 +217,31 @@ __device__ int block_exclusive_scan_1024(int v, int* scratch /*[32]*/, int* tota
   return r;
 }
 
+// The expert GEMMs' work lists (layout in tile_list_ints): every thread of a
+// 1024-thread block calls this; thread e < E passes expert e's row count c
+// and first row off.
+__device__ void write_work_lists(int e, int E, int c, int off, int* tiles, int* scratch,
+                                 int* total) {
+  const int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
+  const int tb = block_exclusive_scan_1024(nt, scratch, total);
+  if (threadIdx.x == 0) tiles[0] = *total;
+  int* rt = row_tile_entries(tiles, E);
+  for (int i = 0; i < nt; ++i) {
+    rt[3 * (tb + i) + 0] = off + i * kGemmBM;
+    rt[3 * (tb + i) + 1] = off + c;
+    rt[3 * (tb + i) + 2] = e;
+  }
+  const int touched = (e < E && c > 0) ? 1 : 0;
+  const int eb = block_exclusive_scan_1024(touched, scratch, total);
+  if (threadIdx.x == 0) tiles[1] = *total;
+  if (touched) {
+    int* et = expert_entries(tiles);
+    et[3 * eb + 0] = off;
+    et[3 * eb + 1] = off + c;
+    et[3 * eb + 2] = e;
+  }
+}
+
 // ============================================================== scan
 // One block of 1024 threads.  counts, offsets, per-block bases, the GEMM
 // tile list (one entry per 128 rows of an expert) and the virtual-EP layout.
@@ -238,16 +269,7 @@ __global__ void __launch_bounds__(1024) k_scan(
     for (int b = 0; b < nblocks; ++b) blockbase[(size_t)b * E + e] += off;
   }
   if (e == 0) offsets[E] = P;
-  // GEMM tiles: (row0, row_end, expert) per 128-row tile of each expert.
-  const int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
-  const int tb = block_exclusive_scan_1024(nt, scratch, &total);
-  if (e == 0) tiles[0] = total;
-  int* tl = tiles + 4;
-  for (int i = 0; i < nt; ++i) {
-    tl[3 * (tb + i) + 0] = off + i * kGemmBM;
-    tl[3 * (tb + i) + 1] = off + c;
-    tl[3 * (tb + i) + 2] = e;
-  }
+  write_work_lists(e, E, c, off, tiles, scratch, &total);
   if (R > 1) {
     for (int i = threadIdx.x; i < R * R; i += blockDim.x) {
       int s = 0;
@@ -277,14 +299,79 @@ __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
       c = 0;
     }
   }
-  const int nt = (c + kGemmBM - 1) / kGemmBM;
-  const int tb = block_exclusive_scan_1024(nt, scratch, &total);
-  if (e == 0) tiles[0] = total;
-  int* tl = tiles + 4;
-  for (int i = 0; i < nt; ++i) {
-    tl[3 * (tb + i) + 0] = a + i * kGemmBM;
-    tl[3 * (tb + i) + 1] = a + c;
-    tl[3 * (tb + i) + 2] = e;
+  write_work_lists(e, E, c, a, tiles, scratch, &total);
+}
+
+// ============================================================== fused routing, T <= 1024
+// One block of 1024 threads does selection and the whole dispatch table for a
+// batch of at most 1024 tokens: top-k (warp w takes tokens w, w+32, ...),
+// histogram, scan, tile list, virtual-EP counts and the stable scatter (one
+// token per thread).  Same results as k_topk + k_hist + k_scan + k_scatter.
+template <int VPL>
+__global__ void __launch_bounds__(1024) k_route_fused(
+    const float* __restrict__ logits, int T, int E, int k, int R, int src_chunk,
+    int* __restrict__ idx, float* __restrict__ w, int* __restrict__ counts,
+    int* __restrict__ offsets, int* __restrict__ tiles, int* __restrict__ send_out,
+    int* __restrict__ rank_off, int* __restrict__ row_of, int* __restrict__ perm, int* err) {
+  extern __shared__ int sm[];
+  int* hist = sm;                                  // [E]
+  int* off_s = hist + E;                           // [E]
+  int* send = off_s + E;                           // [R*R]
+  const int RR = R > 1 ? R * R : 0;
+  uint32_t* masks = reinterpret_cast<uint32_t*>(send + RR);  // [32][E]
+  __shared__ int scratch[32];
+  __shared__ int total;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 2 * E + RR + 32 * E; i += 1024) sm[i] = 0;
+  for (int t = wid; t < T; t += 32)
+    warp_topk<VPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, w + (size_t)t * k);
+  __syncthreads();  // idx (global) is visible to the whole block after the barrier
+  const int t = threadIdx.x;
+  const bool valid = t < T;
+  int my_e[kMaxK];
+  if (valid) {
+    const int per = R > 1 ? E / R : 1;
+    const int src = R > 1 ? t / src_chunk : 0;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      bool ok = (e >= 0 && e < E);
+      for (int j2 = 0; j2 < j && ok; ++j2) ok = my_e[j2] != e;
+      my_e[j] = ok ? e : -1;
+      if (!ok) {
+        record_error(err, MOE_ERR_DEVICE_CHECK, 4);
+        continue;
+      }
+      atomicAdd(&hist[e], 1);
+      atomicOr(&masks[wid * E + e], 1u << lane);
+      if (R > 1) atomicAdd(&send[src * R + e / per], 1);
+    }
+  }
+  __syncthreads();
+  const int c = (threadIdx.x < E) ? hist[threadIdx.x] : 0;
+  const int off = block_exclusive_scan_1024(c, scratch, &total);
+  const int P = total;
+  if (threadIdx.x < E) {
+    counts[threadIdx.x] = c;
+    offsets[threadIdx.x] = off;
+    off_s[threadIdx.x] = off;
+  }
+  if (threadIdx.x == 0) offsets[E] = P;
+  write_work_lists(threadIdx.x, E, c, off, tiles, scratch, &total);
+  if (R > 1) {
+    for (int i = threadIdx.x; i < RR; i += 1024) send_out[i] = send[i];
+    if (threadIdx.x <= R) rank_off[threadIdx.x] = (threadIdx.x == R) ? P : off_s[threadIdx.x * (E / R)];
+  }
+  if (valid) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = my_e[j];
+      if (e < 0) continue;
+      int r = off_s[e];
+      for (int w2 = 0; w2 < wid; ++w2) r += __popc(masks[w2 * E + e]);
+      r += __popc(masks[wid * E + e] & lt);
+      row_of[(size_t)t * k + j] = r;
+      perm[r] = t;
+    }
   }
 }
 
@@ -344,41 +431,41 @@ __global__ void __launch_bounds__(256) k_gather_rows(
 }
 
 // ============================================================== combine
-// y[t] = sum_j w[t,j] * z[row_of[t,j]] in fp32, slot order; one warp per token.
+// y[t] = sum_j w[t,j] * z[row_of[t,j]] in fp32, slot order.  One warp per
+// (token, 256-column chunk): each lane owns 8 columns (one 16-byte vector).
 // A row index outside [0, T*k) contributes nothing (never dereferenced).
 __global__ void __launch_bounds__(256) k_combine(
     const __nv_bfloat16* __restrict__ z, const int* __restrict__ row_of,
-    const float* __restrict__ w, int T, int d, int k,
-    __nv_bfloat16* __restrict__ y) {
+    const float* __restrict__ w, int T, int d, int k, __nv_bfloat16* __restrict__ y) {
   const long long P = (long long)T * k;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const int lane = threadIdx.x & 31;
-  const int nv = d / 8;
-  for (int c = lane; c < nv; c += 32) {
-    float acc[8];
+  const int nchunk = (d + 255) / 256;
+  const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (gw >= (long long)T * nchunk) return;
+  const int t = (int)(gw / nchunk);
+  const int col = (int)(gw - (long long)t * nchunk) * 256 + (threadIdx.x & 31) * 8;
+  if (col >= d) return;
+  float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int r = row_of[(size_t)t * k + j];
-      if (r < 0 || r >= P) continue;
-      const float wj = w[(size_t)t * k + j];
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(z + (size_t)r * d) + c);
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const int r = __ldg(row_of + (size_t)t * k + j);
+    if (r < 0 || r >= P) continue;
+    const float wj = __ldg(w + (size_t)t * k + j);
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(z + (size_t)r * d + col));
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f2 = __bfloat1622float2(p[i]);
-        acc[2 * i] = fmaf(wj, f2.x, acc[2 * i]);
-        acc[2 * i + 1] = fmaf(wj, f2.y, acc[2 * i + 1]);
-      }
+    for (int i = 0; i < 4; ++i) {
+      const float2 f2 = __bfloat1622float2(p[i]);
+      acc[2 * i] = fmaf(wj, f2.x, acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wj, f2.y, acc[2 * i + 1]);
     }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(y + (size_t)t * d)[c] = o;
   }
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(y + (size_t)t * d + col) = o;
 }
 
 // ============================================================== self-test
@@ -405,45 +492,81 @@ cudaError_t launch_selftest_bounded_wait(unsigned long long limit_ns, int* err,
 }
 
 // ============================================================== launchers
-cudaError_t launch_router_partial(const __nv_bfloat16* x, const float* w_g,
-                                  const moe_shape& s, int split, float* part,
-                                  cudaStream_t st) {
-  const int kchunks = s.d / kRtK;
-  const int per = (kchunks + split - 1) / split;
-  dim3 grid((s.T + kRtT - 1) / kRtT, (s.E + kRtE - 1) / kRtE, split);
-  k_router_partial<<<grid, 256, 0, st>>>(x, w_g, s.T, s.d, s.E, per * kRtK, part);
-  return cudaGetLastError();
+static int router_cluster_size(int d) {
+  for (int cs = 8; cs > 1; cs >>= 1)
+    if (d % (64 * cs) == 0) return cs;
+  return 1;
 }
 
-cudaError_t launch_router_finish(const float* part, int split, const float* bias,
-                                 const moe_shape& s, float* logits, cudaStream_t st) {
-  const long long n = (long long)s.T * s.E;
-  const int blocks = (int)std::min<long long>((n + 255) / 256, 4096);
-  k_router_finish<<<blocks, 256, 0, st>>>(part, split, bias, s.T, s.E, logits);
-  return cudaGetLastError();
+cudaError_t launch_router(const __nv_bfloat16* x, const float* w_g, const float* bias,
+                          const moe_shape& s, float* logits, cudaStream_t st) {
+  const int cs = router_cluster_size(s.d);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(cs * ((s.E + kRtE - 1) / kRtE)), (unsigned)((s.T + kRtT - 1) / kRtT), 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_router_cluster, x, w_g, bias, s.T, s.d, s.E, logits);
 }
 
-cudaError_t launch_topk(const float* part, int split, const float* bias,
-                        const moe_shape& s, float* logits_out, int* idx, float* w,
+#define MOE_VPL_DISPATCH(VPL_VAR, CALL) \
+  do {                                  \
+    if ((VPL_VAR) <= 1) { CALL(1); }    \
+    else if ((VPL_VAR) <= 2) { CALL(2); } \
+    else if ((VPL_VAR) <= 4) { CALL(4); } \
+    else if ((VPL_VAR) <= 8) { CALL(8); } \
+    else if ((VPL_VAR) <= 16) { CALL(16); } \
+    else { CALL(32); }                  \
+  } while (0)
+
+cudaError_t launch_topk(const float* logits, const moe_shape& s, int* idx, float* w,
                         cudaStream_t st) {
   const int blocks = (s.T + 7) / 8;
   const int vpl = (s.E + 31) / 32;
-#define MOE_TOPK_CASE(V)                                                     \
-  case V:                                                                    \
-    k_topk<V><<<blocks, 256, 0, st>>>(part, split, bias, s.T, s.E, s.k,      \
-                                      logits_out, idx, w);                   \
-    break;
-  if (vpl <= 4) {
-    switch (vpl) { MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(3) MOE_TOPK_CASE(4) }
-  } else if (vpl <= 8) {
-    k_topk<8><<<blocks, 256, 0, st>>>(part, split, bias, s.T, s.E, s.k, logits_out, idx, w);
-  } else if (vpl <= 16) {
-    k_topk<16><<<blocks, 256, 0, st>>>(part, split, bias, s.T, s.E, s.k, logits_out, idx, w);
-  } else {
-    k_topk<32><<<blocks, 256, 0, st>>>(part, split, bias, s.T, s.E, s.k, logits_out, idx, w);
-  }
-#undef MOE_TOPK_CASE
+#define MOE_TOPK_CALL(V) k_topk<V><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w)
+  MOE_VPL_DISPATCH(vpl, MOE_TOPK_CALL);
+#undef MOE_TOPK_CALL
   return cudaGetLastError();
+}
+
+template <int VPL>
+static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R, int chunk,
+                                 size_t smem, int* idx, float* w, int* counts, int* offsets,
+                                 int* tiles, int* send, int* rank_off, int* row_of, int* perm,
+                                 int* err, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_route_fused<VPL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(4 * (2 * kMaxE + kMaxR * kMaxR + 32 * kMaxE)));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_route_fused<VPL><<<1, 1024, smem, st>>>(logits, s.T, s.E, s.k, R, chunk, idx, w, counts,
+                                            offsets, tiles, send, rank_off, row_of, perm, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
+                               int* counts, int* offsets, int* tiles, int* send,
+                               int* rank_off, int* row_of, int* perm, int* err,
+                               cudaStream_t st) {
+  const int R = s.R > 1 ? s.R : 0;
+  const int chunk = R ? (s.T + R - 1) / R : 1;
+  const size_t smem = sizeof(int) * (2 * s.E + (R ? R * R : 0) + 32 * s.E);
+  const int vpl = (s.E + 31) / 32;
+#define MOE_FUSED_CALL(V)                                                                 \
+  return route_fused_t<V>(logits, s, R, chunk, smem, idx, w, counts, offsets, tiles, send, \
+                          rank_off, row_of, perm, err, st)
+  MOE_VPL_DISPATCH(vpl, MOE_FUSED_CALL);
+#undef MOE_FUSED_CALL
 }
 
 cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayout& L,
@@ -488,7 +611,8 @@ cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, 
 
 cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const float* w,
                            const moe_shape& s, __nv_bfloat16* y, cudaStream_t st) {
-  const int blocks = (s.T + 7) / 8;
+  const long long warps = (long long)s.T * ((s.d + 255) / 256);
+  const unsigned blocks = (unsigned)((warps + 7) / 8);
   k_combine<<<blocks, 256, 0, st>>>(z, row_of, w, s.T, s.d, s.k, y);
   return cudaGetLastError();
 }

@@ -413,3 +413,22 @@ def test_forward_matches_router_then_topk():
     y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=DEV)
     moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, i2, g2)
     assert torch.equal(i1, i2) and torch.equal(g1, g2)
+
+
+def test_layer_graph_replay_matches_eager():
+    """MoELayer's captured-graph path gives the eager call's bits."""
+    cfg = wl.QWEN3_30B_A3B_DECODE.with_T(8)
+    t = wl.make_layer(cfg, DEV, 0)
+    layer = moe.MoELayer(t["w_g"], t["bias"], t["w13"], t["w2"], cfg.k)
+    y_eager = layer(t["x"]).clone()
+    y_graph = layer.forward_graphed(t["x"]).clone()
+    x2 = wl.make_hidden(cfg, DEV, 5)
+    y2_graph = layer.forward_graphed(x2).clone()  # replay with new contents
+    y2_eager = layer(x2)
+    x_host = t["x"].cpu().pin_memory()
+    y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+    layer.forward_host(x_host, y_host)
+    torch.cuda.synchronize()
+    assert layer.check() == moe.MOE_OK
+    assert torch.equal(y_eager, y_graph) and torch.equal(y2_eager, y2_graph)
+    assert torch.equal(y_host, y_eager.cpu())
