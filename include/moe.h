@@ -90,10 +90,16 @@ MOE_API size_t moe_workspace_size(const moe_shape* s);
  *   x      [T, d] bf16          hidden states
  *   w_g    [d, E] fp32          router weight
  *   bias   [E] fp32 or NULL     per-expert additive bias
- *   logits [T, E] fp32 out      logits[t,e] = sum_i x[t,i] w_g[i,e] + bias[e],
- *                               accumulated in fp32 in a fixed order.       */
+ *   logits [T, E] fp32 out      logits[t,e] = sum_i x[t,i] w_g[i,e] + bias[e]
+ *   ws     workspace of moe_workspace_size(s) bytes
+ * Up to 256 tokens: fp32 FMA in a fixed order (a thread-block cluster splits
+ * K; its partial sums meet in distributed shared memory in rank order).
+ * Above 256 tokens: the tcgen05 tensor cores, with w_g split into three bf16
+ * planes (hi + mid + lo = w_g to 24 significant bits) and fp32 accumulation.
+ * Both orders are fixed, and moe_forward uses the same path for the same T,
+ * so its internal logits equal this call's bit for bit. */
 MOE_API int moe_router(const moe_bf16* x, const float* w_g, const float* bias,
-               const moe_shape* s, float* logits, void* stream);
+                       const moe_shape* s, float* logits, void* ws, void* stream);
 
 /* Expert selection and gates ("What is an MoE layer?": 8 of 256 experts per
  * token; "Batching ...": top-8 over 256).

@@ -73,7 +73,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_workspace_size.restype = ctypes.c_size_t
     lib.moe_workspace_size.argtypes = [_S]
     lib.moe_router.restype = ctypes.c_int
-    lib.moe_router.argtypes = [_P, _P, _P, _S, _P, _P]
+    lib.moe_router.argtypes = [_P, _P, _P, _S, _P, _P, _P]
     lib.moe_topk.restype = ctypes.c_int
     lib.moe_topk.argtypes = [_P, _S, _P, _P, _P]
     lib.moe_dispatch.restype = ctypes.c_int
@@ -142,11 +142,12 @@ def workspace(shape: MoEShape, device="cuda") -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def moe_router(x, w_g, bias, logits, shape: MoEShape, stream=None):
+def moe_router(x, w_g, bias, logits, shape: MoEShape, ws, stream=None):
     _check(load_library().moe_router(
         _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
         _ptr(bias, torch.float32, "bias"), ctypes.byref(shape),
-        _ptr(logits, torch.float32, "logits"), _stream(stream)), "moe_router")
+        _ptr(logits, torch.float32, "logits"), _ptr(ws, torch.uint8, "ws"), _stream(stream)),
+        "moe_router")
 
 
 def moe_topk(logits, idx, w, shape: MoEShape, stream=None):

@@ -62,6 +62,18 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
 
+// Router logits: the cluster split-K kernel for small batches, the tensor
+// cores (three bf16 planes of W_g) above kRouterTcMinT tokens.  moe_router
+// and moe_forward both come here, so they give the same bits.
+cudaError_t run_router(const __nv_bfloat16* x, const float* w_g, const float* bias,
+                       const moe_shape& s, float* logits, const WsLayout& L, void* ws,
+                       int sms, cudaStream_t st) {
+  if (s.T >= kRouterTcMinT)
+    return launch_router_tc(x, w_g, bias, s, logits, at<__nv_bfloat16>(ws, L.w3),
+                            at<int>(ws, L.err), sms, st);
+  return launch_router(x, w_g, bias, s, logits, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -86,17 +98,18 @@ size_t moe_workspace_size(const moe_shape* s) {
 }
 
 int moe_router(const moe_bf16* x, const float* w_g, const float* bias, const moe_shape* s,
-               float* logits, void* stream) {
+               float* logits, void* ws, void* stream) {
   if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
   if (s->T == 0) return MOE_OK;
-  if (!ok16(x) || !ok4(w_g) || !ok4(logits) || (bias && !aligned(bias, 4)))
+  if (!ok16(x) || !ok4(w_g) || !ok4(logits) || (bias && !aligned(bias, 4)) || !ws ||
+      !aligned(ws, 256))
     return MOE_ERR_INVALID_ARG;
   int sms = 0;
   int st = device_check(&sms);
   if (st != MOE_OK) return st;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-  return cuda_status(launch_router(xb, w_g, bias, *s, logits, cs));
+  const WsLayout L = ws_layout(*s, sms);
+  return cuda_status(run_router(reinterpret_cast<const __nv_bfloat16*>(x), w_g, bias, *s,
+                                logits, L, ws, sms, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_topk(const float* logits, const moe_shape* s, int32_t* idx, float* w, void* stream) {
@@ -212,7 +225,7 @@ static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
   __nv_bfloat16* z = at<__nv_bfloat16>(ws, L.z);
 
   cudaError_t e = mark(0);
-  if (e == cudaSuccess) e = launch_router(xb, w_g, bias, *s, logits, cs);
+  if (e == cudaSuccess) e = run_router(xb, w_g, bias, *s, logits, L, ws, sms, cs);
   if (e == cudaSuccess) e = mark(1);
   if (e == cudaSuccess) {
     if (s->T <= kFusedRouteMaxT) {

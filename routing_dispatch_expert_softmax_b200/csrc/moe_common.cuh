@@ -22,6 +22,8 @@ constexpr int kMaxR = 64;
 // Batches of at most this many tokens (so at most this many rows per expert)
 // run the expert GEMMs in swap-AB form.
 constexpr int kSwapMaxT = 256;
+// Batches above this many tokens compute router logits on the tensor cores.
+constexpr int kRouterTcMinT = 257;
 
 // Device error word: ws[0] = first error code, ws[1] = detail (kernel id).
 enum : int { kErrSlot = 0, kErrDetail = 1 };
@@ -35,7 +37,7 @@ __device__ __forceinline__ void record_error(int* err, int code, int detail) {
 
 // ----------------------------------------------------------------- workspace
 struct WsLayout {
-  size_t err, logits, idx, w, counts, offsets, blockhist, blockbase,
+  size_t err, w3, logits, idx, w, counts, offsets, blockhist, blockbase,
       blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, total;
   int nblocks;      // token blocks of kTokensPerRouteBlock
   int max_mtiles;   // upper bound of 128-row expert tiles
@@ -71,6 +73,7 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
     return at;
   };
   L.err = take(64);
+  L.w3 = take(2 * 3 * (size_t)d * E);  // router weight split into 3 bf16 planes
   L.logits = take(sizeof(float) * T * E);
   L.idx = take(sizeof(int) * T * k);
   L.w = take(sizeof(float) * T * k);
@@ -179,6 +182,12 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* t
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 

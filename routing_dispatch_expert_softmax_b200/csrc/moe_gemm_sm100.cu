@@ -25,7 +25,31 @@
 
 namespace moe {
 
-template <int BN, bool SWIGLU>
+// Epilogues of the grouped GEMM.
+enum : int {
+  kEpiSwiGLU = 0,  // h = silu(gate) * up -> bf16 (columns [0,BN/2) gate, [BN/2,BN) up)
+  kEpiStore = 1,   // bf16 copy of the accumulator
+  kEpiLogits = 2   // fp32 accumulator + bias[col] (router logits)
+};
+
+struct GemmArgs {
+  const int* tiles;       // device work lists; nullptr = dense rows [0, dense_rows)
+  int E;                  // experts (the row tiles follow E expert entries)
+  int dense_rows;         // rows of A in dense mode
+  int n_tiles;            // output tiles of width BN (BN/2 for SwiGLU) per row tile
+  int K;                  // reduction length of B (multiple of 64)
+  int a_kblocks;          // A's K coordinate is (kb mod a_kblocks) * 64
+  int b_rows_per_expert;  // B rows owned by one expert
+  int up_offset;          // SwiGLU: B row offset of the up half
+  int n_out;              // valid output columns
+  void* out;
+  int ld_out;
+  const float* bias;      // kEpiLogits only (may be null)
+  int* err;
+  int weights_once;       // 1: each B tile is read by one work item (hint evict_first)
+};
+
+template <int BN, int EPI>
 struct GemmCfg {
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
@@ -47,14 +71,30 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
-template <int BN, bool SWIGLU>
+// Grouped rasterization of the work items: row tiles are taken in groups of
+// kRasterGroup; inside a group the output tile is the slow index, so the CTAs
+// running at the same time share weight tiles (each read once from DRAM and
+// reused by the group's row tiles from L2) and the group's activation tiles
+// stay in L2 while the output tiles sweep past them.
+constexpr int kRasterGroup = 16;
+
+__device__ __forceinline__ void raster(int w, int n_tiles, int num_mtiles, int& mt, int& nt) {
+  const int per_group = kRasterGroup * n_tiles;
+  const int g = w / per_group;
+  const int r = w - g * per_group;
+  const int g0 = g * kRasterGroup;
+  const int gsz = min(kRasterGroup, num_mtiles - g0);
+  nt = r / gsz;
+  mt = g0 + (r - nt * gsz);
+}
+
+template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-    const int* __restrict__ tiles, int E, int n_tiles, int K, int b_rows_per_expert,
-    int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
-    int* __restrict__ err) {
-  using C = GemmCfg<BN, SWIGLU>;
+    const GemmArgs args) {
+  using C = GemmCfg<BN, EPI>;
   constexpr int S = C::kStages;
+  constexpr bool SWIGLU = (EPI == kEpiSwiGLU);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -93,16 +133,20 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_mtiles = tiles[0];
+  const bool dense = args.tiles == nullptr;
+  const int num_mtiles = dense ? (args.dense_rows + kGemmBM - 1) / kGemmBM : args.tiles[0];
+  const int n_tiles = args.n_tiles;
   const int total = num_mtiles * n_tiles;
-  const int nk = K / kGemmBK;
-  const int* tl = tiles + 4 + 3 * E;  // row tiles follow the E expert entries
+  const int nk = args.K / kGemmBK;
+  const int* tl = dense ? nullptr : args.tiles + 4 + 3 * args.E;  // row tiles follow the expert entries
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      const uint64_t pol_w = policy_evict_first();  // weights: streamed once
-      const uint64_t pol_a = policy_evict_last();   // activations: reused
+      // Weight tiles used by a single row tile are streamed (evict first);
+      // otherwise every row tile of the expert re-reads them from L2.
+      const uint64_t pol_w = args.weights_once ? policy_evict_first() : policy_evict_normal();
+      const uint64_t pol_a = policy_evict_normal();
       int fills[S];
 #pragma unroll
       for (int s = 0; s < S; ++s) fills[s] = 0;
@@ -110,10 +154,12 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
       uint32_t phase = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int mt = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
-        const int row0 = tl[3 * mt + 0];
-        const int e = tl[3 * mt + 2];
-        const int brow = e * b_rows_per_expert + nt * (SWIGLU ? BN / 2 : BN);
+        int mt, nt;
+        raster(w, n_tiles, num_mtiles, mt, nt);
+        const int row0 = dense ? mt * kGemmBM : tl[3 * mt + 0];
+        const int e = dense ? 0 : tl[3 * mt + 2];
+        const int brow = e * args.b_rows_per_expert + nt * (SWIGLU ? BN / 2 : BN);
+        int ka = 0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -122,11 +168,12 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
           uint8_t* a_dst = smem + stage * C::kStageBytes;
           uint8_t* b_dst = a_dst + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(a_dst, &tmA, &full[stage], kb * kGemmBK, row0, pol_a);
+          tma_load_2d(a_dst, &tmA, &full[stage], ka * kGemmBK, row0, pol_a);
+          if (++ka == args.a_kblocks) ka = 0;
           if (SWIGLU) {
             tma_load_2d(b_dst, &tmB, &full[stage], kb * kGemmBK, brow, pol_w);
             tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[stage], kb * kGemmBK,
-                        brow + up_offset, pol_w);
+                        brow + args.up_offset, pol_w);
           } else {
             tma_load_2d(b_dst, &tmB, &full[stage], kb * kGemmBK, brow, pol_w);
           }
@@ -191,9 +238,10 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
     const int r_in_tile = q * 32 + lane;
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      const int mt = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
-      const int row0 = tl[3 * mt + 0];
-      const int rowend = tl[3 * mt + 1];
+      int mt, nt;
+      raster(w, n_tiles, num_mtiles, mt, nt);
+      const int row0 = dense ? mt * kGemmBM : tl[3 * mt + 0];
+      const int rowend = dense ? args.dense_rows : tl[3 * mt + 1];
       const int ab = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       const bool got = mbar_wait_bounded(&tfull[ab], aph, abort_flag);
@@ -202,8 +250,9 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
       const uint32_t t_addr = tmem_base + (uint32_t)(ab * BN) + ((uint32_t)(q * 32) << 16);
       const int row = row0 + r_in_tile;
       const bool row_ok = row < rowend;
-      if (SWIGLU) {
+      if (EPI == kEpiSwiGLU) {
         constexpr int H = BN / 2;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
 #pragma unroll 1
         for (int c = 0; c < H; c += 32) {
           uint32_t g[32], u[32];
@@ -211,7 +260,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
           tmem_ld_32x32b_x32(t_addr + H + c, u);
           tmem_ld_wait();
           const int col = nt * H + c;
-          if (row_ok && col < n_out) {
+          if (row_ok && col < args.n_out) {
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -219,28 +268,48 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
               const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
               p[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
             }
-            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * ld_out + col);
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * args.ld_out + col);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
           }
         }
-      } else {
+      } else if (EPI == kEpiStore) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t a[32];
           tmem_ld_32x32b_x32(t_addr + c, a);
           tmem_ld_wait();
           const int col = nt * BN + c;
-          if (row_ok && col < n_out) {
+          if (row_ok && col < args.n_out) {
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               p[i] = pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * ld_out + col);
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * args.ld_out + col);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+          }
+        }
+      } else {
+        float* out = static_cast<float*>(args.out);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(t_addr + c, a);
+          tmem_ld_wait();
+          const int col = nt * BN + c;
+          if (row_ok && col < args.n_out) {
+            float* dst = out + (size_t)row * args.ld_out + col;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (col + i < args.n_out) {
+                const float bv = args.bias ? __ldg(args.bias + col + i) : 0.f;
+                dst[i] = args.bias ? __uint_as_float(a[i]) + bv : __uint_as_float(a[i]);
+              }
+            }
           }
         }
       }
@@ -252,7 +321,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x == 0 && *abort_flag) record_error(err, MOE_ERR_TIMEOUT, 10);
+  if (threadIdx.x == 0 && *abort_flag) record_error(args.err, MOE_ERR_TIMEOUT, 10);
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
@@ -554,15 +623,14 @@ static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWIGLU>
+template <int BN, int EPI>
 static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
-                                 const int* tiles, int E, int max_work, int n_tiles, int K,
-                                 int b_rows, int up_off, int n_out, __nv_bfloat16* out,
-                                 int ld_out, int* err, int num_sms, cudaStream_t st) {
-  using C = GemmCfg<BN, SWIGLU>;
+                                 const GemmArgs& args, int max_work, int num_sms,
+                                 cudaStream_t st) {
+  using C = GemmCfg<BN, EPI>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<BN, SWIGLU>,
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<BN, EPI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -570,8 +638,7 @@ static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
   }
   int grid = max_work < num_sms ? max_work : num_sms;
   if (grid < 1) grid = 1;
-  k_grouped_gemm<BN, SWIGLU><<<grid, C::kThreads, C::kSmemBytes, st>>>(
-      ta, tb, tiles, E, n_tiles, K, b_rows, up_off, n_out, out, ld_out, err);
+  k_grouped_gemm<BN, EPI><<<grid, C::kThreads, C::kSmemBytes, st>>>(ta, tb, args);
   return cudaGetLastError();
 }
 
@@ -668,24 +735,74 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
     return MOE_ERR_CUDA;
   const int nt1 = (int)((s.f + bn / 2 - 1) / (bn / 2));
   const int nt2 = (int)((s.d + bn - 1) / bn);
+  GemmArgs g1{tiles, s.E, 0, nt1, s.d, s.d / kGemmBK, 2 * s.f, s.f, s.f, h, s.f, nullptr, err, 0};
+  GemmArgs g2{tiles, s.E, 0, nt2, s.f, s.f / kGemmBK, s.d, 0, s.d, z, s.d, nullptr, err, 0};
   cudaError_t e;
   if (wide) {
-    e = launch_gemm_t<256, true>(tA1, tB1, tiles, s.E, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
-                                 s.f, s.f, h, s.f, err, num_sms, st);
+    e = launch_gemm_t<256, kEpiSwiGLU>(tA1, tB1, g1, L.max_mtiles * nt1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
-      e = launch_gemm_t<256, false>(tA2, tB2, tiles, s.E, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
-                                    s.d, z, s.d, err, num_sms, st);
+      e = launch_gemm_t<256, kEpiStore>(tA2, tB2, g2, L.max_mtiles * nt2, num_sms, st);
   } else {
-    e = launch_gemm_t<128, true>(tA1, tB1, tiles, s.E, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
-                                 s.f, s.f, h, s.f, err, num_sms, st);
+    e = launch_gemm_t<128, kEpiSwiGLU>(tA1, tB1, g1, L.max_mtiles * nt1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
-      e = launch_gemm_t<128, false>(tA2, tB2, tiles, s.E, L.max_mtiles * nt2, nt2, s.f, s.d, 0,
-                                    s.d, z, s.d, err, num_sms, st);
+      e = launch_gemm_t<128, kEpiStore>(tA2, tB2, g2, L.max_mtiles * nt2, num_sms, st);
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ============================================================== router, large T
+// W_g (d x E, fp32) -> three bf16 planes W3 (E rows x 3d, K-major) with
+// W = hi + mid + lo exactly to 24 significant bits: hi = bf16(W),
+// mid = bf16(W - hi), lo = bf16(W - hi - mid) (each difference is exact in
+// fp32).  x is bf16, so x . W_g = x . [hi | mid | lo] over K = 3d on the bf16
+// tensor cores with fp32 accumulation.
+__global__ void __launch_bounds__(256) k_router_split(const float* __restrict__ w_g, int d,
+                                                      int E, __nv_bfloat16* __restrict__ w3) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int k = k0 + r, e = e0 + tx;
+    tile[r][tx] = (k < d && e < E) ? w_g[(size_t)k * E + e] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r, k = k0 + tx;
+    if (e < E && k < d) {
+      const float v = tile[tx][r];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const float r1 = v - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(mid);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+      __nv_bfloat16* row = w3 + (size_t)e * 3 * d;
+      row[k] = hi;
+      row[d + k] = mid;
+      row[2 * d + k] = lo;
+    }
+  }
+}
+
+cudaError_t launch_router_tc(const __nv_bfloat16* x, const float* w_g, const float* bias,
+                             const moe_shape& s, float* logits, __nv_bfloat16* w3,
+                             int* err, int num_sms, cudaStream_t st) {
+  dim3 g((s.d + 31) / 32, (s.E + 31) / 32);
+  k_router_split<<<g, 256, 0, st>>>(w_g, s.d, s.E, w3);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const uint32_t bn = s.E <= 128 ? 128 : 256;
+  CUtensorMap tA, tB;
+  if (!make_tmap(&tA, x, (uint64_t)s.T, (uint64_t)s.d, kGemmBM) ||
+      !make_tmap(&tB, w3, (uint64_t)s.E, (uint64_t)3 * s.d, bn))
+    return cudaErrorInvalidValue;
+  const int nt = (s.E + bn - 1) / bn;
+  GemmArgs a{nullptr, 0, s.T, nt, 3 * s.d, s.d / kGemmBK, 0, 0, s.E, logits, s.E, bias, err, 0};
+  const int work = ((s.T + kGemmBM - 1) / kGemmBM) * nt;
+  if (bn == 128) return launch_gemm_t<128, kEpiLogits>(tA, tB, a, work, num_sms, st);
+  return launch_gemm_t<256, kEpiLogits>(tA, tB, a, work, num_sms, st);
 }
 
 }  // namespace moe

@@ -24,6 +24,75 @@ namespace moe {
 // leaves the SMs but the logits.
 constexpr int kRtT = 32, kRtE = 32, kRtKC = 128;
 
+// Chunk loads of the router: every thread issues all of its 16-byte loads for
+// a 128-deep K chunk before using any of them (W: 128 x 32 fp32 = 4 float4
+// per thread; x: 32 x 128 bf16 = 2 uint4 per thread), so a chunk costs one
+// memory latency, and the next chunk's loads are in flight while this one is
+// multiplied.
+struct RouterRegs {
+  float4 w[4];
+  uint4 x[2];
+};
+
+__device__ __forceinline__ void router_load(RouterRegs& r, const __nv_bfloat16* __restrict__ x,
+                                            const float* __restrict__ w_g, int T, int d, int E,
+                                            int t0, int e0, int kc, int chunk) {
+  const int vpr = chunk / 8;  // 16-byte x vectors per token row
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int v = threadIdx.x + 256 * u;
+    r.x[u] = make_uint4(0, 0, 0, 0);
+    if (v < kRtT * vpr) {
+      const int row = v / vpr, c8 = (v - row * vpr) * 8;
+      if (t0 + row < T)
+        r.x[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + row) * d + kc + c8));
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int v = threadIdx.x + 256 * u;  // 8 float4 per K row (32 experts)
+    const int row = v >> 3, c4 = (v & 7) * 4;
+    r.w[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < chunk) {
+      const int e = e0 + c4;
+      const float* src = w_g + (size_t)(kc + row) * E + e;
+      if ((E & 3) == 0 && e + 3 < E) {
+        r.w[u] = __ldg(reinterpret_cast<const float4*>(src));
+      } else {
+        float t4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) t4[q] = (e + q < E) ? __ldg(src + q) : 0.f;
+        r.w[u] = make_float4(t4[0], t4[1], t4[2], t4[3]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void router_store(const RouterRegs& r, float (*xs)[kRtKC],
+                                             float (*ws)[kRtE], int chunk) {
+  const int vpr = chunk / 8;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int v = threadIdx.x + 256 * u;
+    if (v < kRtT * vpr) {
+      const int row = v / vpr, c8 = (v - row * vpr) * 8;
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.x[u]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        xs[row][c8 + 2 * i] = f.x;
+        xs[row][c8 + 2 * i + 1] = f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int v = threadIdx.x + 256 * u;
+    const int row = v >> 3, c4 = (v & 7) * 4;
+    if (row < chunk) *reinterpret_cast<float4*>(&ws[row][c4]) = r.w[u];
+  }
+}
+
 __global__ void __launch_bounds__(256) k_router_cluster(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ w_g,
     const float* __restrict__ bias, int T, int d, int E, float* __restrict__ logits) {
@@ -31,8 +100,8 @@ __global__ void __launch_bounds__(256) k_router_cluster(
   cg::cluster_group cl = cg::this_cluster();
   const int CS = (int)cl.num_blocks();
   const int rank = (int)cl.block_rank();
-  __shared__ float xs[kRtT][kRtKC];
-  __shared__ float ws[kRtKC][kRtE];
+  __shared__ __align__(16) float xs[kRtT][kRtKC];
+  __shared__ __align__(16) float ws[kRtKC][kRtE];
   __shared__ float part[kRtT * kRtE];
   const int e0 = (blockIdx.x / CS) * kRtE;
   const int t0 = blockIdx.y * kRtT;
@@ -40,28 +109,14 @@ __global__ void __launch_bounds__(256) k_router_cluster(
   const int kbeg = rank * kslice, kend = kbeg + kslice;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  RouterRegs regs;
+  router_load(regs, x, w_g, T, d, E, t0, e0, kbeg, min(kRtKC, kend - kbeg));
   for (int kc = kbeg; kc < kend; kc += kRtKC) {
     const int chunk = min(kRtKC, kend - kc);  // 64 or 128
-    const int vpr = chunk / 8;                 // 16-byte vectors per token row
-    for (int v = threadIdx.x; v < kRtT * vpr; v += 256) {
-      const int r = v / vpr, c8 = (v - r * vpr) * 8;
-      const int t = t0 + r;
-      uint4 q = make_uint4(0, 0, 0, 0);
-      if (t < T) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + kc + c8));
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h[i]);
-        xs[r][c8 + 2 * i] = f.x;
-        xs[r][c8 + 2 * i + 1] = f.y;
-      }
-    }
-    for (int i = threadIdx.x; i < chunk * kRtE; i += 256) {
-      const int r = i / kRtE, c = i - r * kRtE;
-      const int e = e0 + c;
-      ws[r][c] = (e < E) ? __ldg(w_g + (size_t)(kc + r) * E + e) : 0.f;
-    }
+    router_store(regs, xs, ws, chunk);
     __syncthreads();
+    if (kc + kRtKC < kend)
+      router_load(regs, x, w_g, T, d, E, t0, e0, kc + kRtKC, min(kRtKC, kend - kc - kRtKC));
     for (int kk = 0; kk < chunk; ++kk) {
       const float wv = ws[kk][tx];
 #pragma unroll
@@ -89,49 +144,56 @@ __global__ void __launch_bounds__(256) k_router_cluster(
 // the k selected logits (equal to the full softmax renormalised over them).
 // Shared by k_topk and the fused small-batch routing kernel so both take the
 // same decisions.
+// Order-preserving 32-bit key of a float: a < b  <=>  key(a) < key(b).
+// -0.0 is first turned into +0.0 so the two zeros get one key and tie.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 template <int VPL>
 __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k,
                                           int lane, int* __restrict__ idx_row,
                                           float* __restrict__ w_row) {
-  float v[VPL];
+  uint32_t key[VPL];
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
-    v[i] = 0.f;
-    if (e < E) v[i] = row[e];
+    key[i] = 0;
+    if (e < E) key[i] = order_key(row[e]);
     else taken |= 1u << i;  // not a candidate
   }
-  float my_v = 0.f;
+  uint32_t my_key = 0;
   int my_e = 0;
   for (int j = 0; j < k; ++j) {
-    float bv = 0.f;
-    int be = INT_MAX;  // INT_MAX = no candidate
+    // this lane's best remaining candidate: largest key, lowest index
+    uint32_t bk = 0;
+    int bi = -1;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       if (taken & (1u << i)) continue;
-      if (be == INT_MAX || v[i] > bv) {  // ascending e: equal keeps the lower index
-        bv = v[i];
-        be = lane + 32 * i;
+      if (bi < 0 || key[i] > bk) {  // ascending index: an equal key keeps the lower index
+        bk = key[i];
+        bi = i;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      const bool take =
-          oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be));
-      if (take) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    // Lanes with no candidate left take part with key 0 and index 0xffffffff;
+    // real keys are never 0 (0 would be the key of a negative NaN pattern).
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bi >= 0 ? bk : 0u);
+    const uint32_t cand = (bi >= 0 && bk == wk) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+    const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
+    if ((int)(we & 31) == lane) taken |= 1u << (we >> 5);
     if (lane == j) {
-      my_v = bv;
-      my_e = be;
+      my_key = wk;
+      my_e = (int)we;
     }
   }
+  const float my_v = key_value(my_key);
   const float top = __shfl_sync(0xffffffffu, my_v, 0);
   const float ex = (lane < k) ? expf(my_v - top) : 0.f;
   float sum = ex;
@@ -441,25 +503,45 @@ __global__ void __launch_bounds__(256) k_combine(
   const int nchunk = (d + 255) / 256;
   const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (gw >= (long long)T * nchunk) return;
+  const int lane = threadIdx.x & 31;
   const int t = (int)(gw / nchunk);
-  const int col = (int)(gw - (long long)t * nchunk) * 256 + (threadIdx.x & 31) * 8;
-  if (col >= d) return;
+  const int col = (int)(gw - (long long)t * nchunk) * 256 + lane * 8;
+  // lane j < k holds slot j's row and gate; broadcast them with shuffles so
+  // the k row loads below are all independent.
+  int my_r = -1;
+  float my_w = 0.f;
+  if (lane < k) {
+    my_r = __ldg(row_of + (size_t)t * k + lane);
+    my_w = __ldg(w + (size_t)t * k + lane);
+  }
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const int r = __ldg(row_of + (size_t)t * k + j);
-    if (r < 0 || r >= P) continue;
-    const float wj = __ldg(w + (size_t)t * k + j);
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(z + (size_t)r * d + col));
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    uint4 v[8];
+    float wj[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f2 = __bfloat1622float2(p[i]);
-      acc[2 * i] = fmaf(wj, f2.x, acc[2 * i]);
-      acc[2 * i + 1] = fmaf(wj, f2.y, acc[2 * i + 1]);
+    for (int jj = 0; jj < 8; ++jj) {
+      const int r = __shfl_sync(0xffffffffu, my_r, (j0 + jj) & 31);
+      wj[jj] = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
+      const bool ok = (j0 + jj < k) && r >= 0 && r < P && col < d;
+      v[jj] = ok ? __ldg(reinterpret_cast<const uint4*>(z + (size_t)r * d + col))
+                 : make_uint4(0, 0, 0, 0);
+      if (!ok) wj[jj] = 0.f;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      if (j0 + jj >= k) break;
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[jj]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __bfloat1622float2(p[i]);
+        acc[2 * i] = fmaf(wj[jj], f2.x, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj[jj], f2.y, acc[2 * i + 1]);
+      }
     }
   }
+  if (col >= d) return;
   uint4 o;
   o.x = pack_bf16x2(acc[0], acc[1]);
   o.y = pack_bf16x2(acc[2], acc[3]);

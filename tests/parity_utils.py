@@ -47,6 +47,21 @@ def logit_bound(x64, wg64, bias64=None):
     return gamma * s
 
 
+def logit_bound_tensor_cores(x64, wg64, bias64=None):
+    """Bound for the tensor-core router (T > 256): W_g is carried as three
+    bf16 planes (residual below 2^-24 |W| per term, counted as one more
+    rounding) and the 3d products are accumulated in fp32 by the tensor cores,
+    whose internal rounding we allow twice the fp32 unit roundoff:
+    2 gamma_{3d+4} * (sum|x W| + |b|)."""
+    d = x64.shape[1]
+    n = 3 * d + 4
+    gamma = n * U32 / (1 - n * U32)
+    s = np.abs(x64) @ np.abs(wg64)
+    if bias64 is not None:
+        s = s + np.abs(bias64)[None, :]
+    return 2 * gamma * s
+
+
 def selection_is_valid(L64_row, delta_row, sel):
     """True when some logits within [L - delta, L + delta] make `sel` (an
     ordered list of k experts) the top-k in that slot order."""

@@ -79,10 +79,12 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     bad_shape = ctypes.byref(B.MoEShape.of(**dict(VALID, k=0)))
     INV = B.MOE_ERR_INVALID_ARG
     # moe_router: null / misaligned x, null logits, invalid shape
-    assert _raw(lib, "moe_router", None, _P(A16), None, s, _P(A16), None) == INV
-    assert _raw(lib, "moe_router", _P(MIS), _P(A16), None, s, _P(A16), None) == INV
-    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, s, None, None) == INV
-    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, bad_shape, _P(A16), None) == INV
+    assert _raw(lib, "moe_router", None, _P(A16), None, s, _P(A16), _P(A16), None) == INV
+    assert _raw(lib, "moe_router", _P(MIS), _P(A16), None, s, _P(A16), _P(A16), None) == INV
+    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, s, None, _P(A16), None) == INV
+    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, s, _P(A16), None, None) == INV
+    assert _raw(lib, "moe_router", _P(A16), _P(A16), None, bad_shape, _P(A16), _P(A16),
+                None) == INV
     # moe_topk
     assert _raw(lib, "moe_topk", None, s, _P(A16), _P(A16), None) == INV
     assert _raw(lib, "moe_topk", _P(A16 + 1), s, _P(A16), _P(A16), None) == INV
@@ -114,7 +116,7 @@ def test_bad_arguments_are_rejected_before_launch(lib):
 def test_empty_batch_is_a_no_op(lib):
     s0 = ctypes.byref(B.MoEShape.of(**dict(VALID, T=0)))
     # T = 0 launches nothing, so even null activation pointers are accepted.
-    assert _raw(lib, "moe_router", None, None, None, s0, None, None) == B.MOE_OK
+    assert _raw(lib, "moe_router", None, None, None, s0, None, None, None) == B.MOE_OK
     assert _raw(lib, "moe_topk", None, s0, None, None, None) == B.MOE_OK
     assert _raw(lib, "moe_combine", None, None, None, s0, None, None) == B.MOE_OK
     assert _raw(lib, "moe_forward", *[None] * 5, s0, None, None, None, None, _P(A16),
