@@ -22,6 +22,7 @@ constexpr int kMaxR = 64;
 // Batches of at most this many tokens (so at most this many rows per expert)
 // run the expert GEMMs in swap-AB form.
 constexpr int kSwapMaxT = 256;
+
 // Batches above this many tokens compute router logits on the tensor cores.
 constexpr int kRouterTcMinT = 257;
 
@@ -74,6 +75,7 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   };
   L.err = take(64);
   L.w3 = take(2 * 3 * (size_t)d * E);  // router weight split into 3 bf16 planes
+
   L.logits = take(sizeof(float) * T * E);
   L.idx = take(sizeof(int) * T * k);
   L.w = take(sizeof(float) * T * k);
@@ -104,6 +106,16 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+// Programmatic dependent launch: every kernel of the layer lets the next one
+// launch as soon as all of its own CTAs are running (trigger), and waits for
+// its predecessor grid to complete and publish its memory before touching
+// any global data (wait).  The next kernel's launch and prologue then overlap
+// this kernel's tail.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ bool elect_one_lane() {
   return (threadIdx.x & 31) == 0;
@@ -302,6 +314,34 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Launches `kern` on `st` with programmatic stream serialization (so the
+// kernel may start while its predecessor finishes; it synchronises with
+// pdl_wait) and, if cluster > 1, a 1-D thread-block cluster.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 }  // namespace moe

@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // the work lists and operands come from the previous kernels
 
   const bool dense = args.tiles == nullptr;
   const int num_mtiles = dense ? (args.dense_rows + kGemmBM - 1) / kGemmBM : args.tiles[0];
@@ -406,6 +408,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // the work lists and operands come from the previous kernels
   const int total = tiles[1] * n_tiles;
   const int nk = K / kGemmBK;
   const int* et = tiles + 4;
@@ -638,8 +642,8 @@ static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
   }
   int grid = max_work < num_sms ? max_work : num_sms;
   if (grid < 1) grid = 1;
-  k_grouped_gemm<BN, EPI><<<grid, C::kThreads, C::kSmemBytes, st>>>(ta, tb, args);
-  return cudaGetLastError();
+  return launch_kernel(k_grouped_gemm<BN, EPI>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, st,
+                       1, ta, tb, args);
 }
 
 template <int NMAX, bool SWIGLU>
@@ -658,9 +662,8 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
   }
   int grid = max_work < num_sms ? max_work : num_sms;
   if (grid < 1) grid = 1;
-  k_expert_gemm_swap<NMAX, SWIGLU><<<grid, 192, C::kSmemBytes, st>>>(
-      tw, tx, tiles, n_tiles, K, w_rows, up_off, n_out, out, ld_out, err);
-  return cudaGetLastError();
+  return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU>, dim3(grid), dim3(192), C::kSmemBytes, st,
+                       1, tw, tx, tiles, n_tiles, K, w_rows, up_off, n_out, out, ld_out, err);
 }
 
 // Small batches (every expert has at most 256 rows): both GEMMs in swap-AB form.
@@ -761,6 +764,8 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
 // tensor cores with fp32 accumulation.
 __global__ void __launch_bounds__(256) k_router_split(const float* __restrict__ w_g, int d,
                                                       int E, __nv_bfloat16* __restrict__ w3) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float tile[32][33];
   const int k0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -790,8 +795,7 @@ cudaError_t launch_router_tc(const __nv_bfloat16* x, const float* w_g, const flo
                              const moe_shape& s, float* logits, __nv_bfloat16* w3,
                              int* err, int num_sms, cudaStream_t st) {
   dim3 g((s.d + 31) / 32, (s.E + 31) / 32);
-  k_router_split<<<g, 256, 0, st>>>(w_g, s.d, s.E, w3);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(k_router_split, g, dim3(256), 0, st, 1, w_g, s.d, s.E, w3);
   if (e != cudaSuccess) return e;
   const uint32_t bn = s.E <= 128 ? 128 : 256;
   CUtensorMap tA, tB;

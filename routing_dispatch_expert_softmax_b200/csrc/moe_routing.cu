@@ -96,6 +96,8 @@ __device__ __forceinline__ void router_store(const RouterRegs& r, float (*xs)[kR
 __global__ void __launch_bounds__(256) k_router_cluster(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ w_g,
     const float* __restrict__ bias, int T, int d, int E, float* __restrict__ logits) {
+  pdl_trigger();
+  pdl_wait();
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int CS = (int)cl.num_blocks();
@@ -209,6 +211,8 @@ template <int VPL>
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, int T, int E,
                                               int k, int* __restrict__ idx,
                                               float* __restrict__ w) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
   warp_topk<VPL>(logits + (size_t)t * E, E, k, threadIdx.x & 31, idx + (size_t)t * k,
@@ -221,6 +225,8 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, 
 __global__ void __launch_bounds__(kTokensPerRouteBlock) k_hist(
     const int* __restrict__ idx, int T, int E, int k, int R, int src_chunk,
     int* __restrict__ blockhist, int* __restrict__ blocksend, int* err) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int sm[];
   int* hist = sm;            // [E]
   int* send = sm + E;        // [R*R] when R > 1
@@ -312,6 +318,8 @@ __global__ void __launch_bounds__(1024) k_scan(
     const int* __restrict__ blocksend, int* __restrict__ blockbase,
     int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ tiles,
     int* __restrict__ send, int* __restrict__ rank_off) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int scratch[32];
   __shared__ int total;
   const int e = threadIdx.x;  // E <= 1024
@@ -348,6 +356,8 @@ __global__ void __launch_bounds__(1024) k_scan(
 // Tile list from caller-provided offsets (moe_ffn); checks the offsets.
 __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
     const int* __restrict__ offsets, int E, int P, int* __restrict__ tiles, int* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int scratch[32];
   __shared__ int total;
   const int e = threadIdx.x;
@@ -367,27 +377,79 @@ __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
 // ============================================================== fused routing, T <= 1024
 // One block of 1024 threads does selection and the whole dispatch table for a
 // batch of at most 1024 tokens: top-k (warp w takes tokens w, w+32, ...),
-// histogram, scan, tile list, virtual-EP counts and the stable scatter (one
-// token per thread).  Same results as k_topk + k_hist + k_scan + k_scatter.
+// histogram, one block scan of (rows, 128-row tiles, touched) per expert,
+// work lists, virtual-EP counts and the stable scatter (one token per
+// thread).  Same results as k_topk + k_hist + k_scan + k_scatter.
+constexpr int kFusedSmemIdx = 8192;  // T*k up to this keeps the ids in shared memory
+
+// Exclusive block scan of three ints over 1024 threads (two barriers).
+__device__ __forceinline__ int3 block_exclusive_scan3_1024(int3 v, int3* warp_tot, int3* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int3 inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, inc.x, off);
+    const int b = __shfl_up_sync(0xffffffffu, inc.y, off);
+    const int c = __shfl_up_sync(0xffffffffu, inc.z, off);
+    if (lane >= off) {
+      inc.x += a;
+      inc.y += b;
+      inc.z += c;
+    }
+  }
+  if (lane == 31) warp_tot[wid] = inc;
+  __syncthreads();
+  if (wid == 0) {
+    const int3 t = warp_tot[lane];
+    int3 si = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, si.x, off);
+      const int b = __shfl_up_sync(0xffffffffu, si.y, off);
+      const int c = __shfl_up_sync(0xffffffffu, si.z, off);
+      if (lane >= off) {
+        si.x += a;
+        si.y += b;
+        si.z += c;
+      }
+    }
+    warp_tot[lane] = make_int3(si.x - t.x, si.y - t.y, si.z - t.z);
+    if (lane == 31) *total = si;
+  }
+  __syncthreads();
+  const int3 base = warp_tot[wid];
+  return make_int3(base.x + inc.x - v.x, base.y + inc.y - v.y, base.z + inc.z - v.z);
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(1024) k_route_fused(
     const float* __restrict__ logits, int T, int E, int k, int R, int src_chunk,
     int* __restrict__ idx, float* __restrict__ w, int* __restrict__ counts,
     int* __restrict__ offsets, int* __restrict__ tiles, int* __restrict__ send_out,
     int* __restrict__ rank_off, int* __restrict__ row_of, int* __restrict__ perm, int* err) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int sm[];
   int* hist = sm;                                  // [E]
   int* off_s = hist + E;                           // [E]
   int* send = off_s + E;                           // [R*R]
   const int RR = R > 1 ? R * R : 0;
   uint32_t* masks = reinterpret_cast<uint32_t*>(send + RR);  // [32][E]
-  __shared__ int scratch[32];
-  __shared__ int total;
+  int* idx_s = reinterpret_cast<int*>(masks + 32 * E);         // [T*k] when it fits
+  __shared__ int3 warp_tot[32];
+  __shared__ int3 total;
+  const bool ids_in_smem = T * k <= kFusedSmemIdx;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 2 * E + RR + 32 * E; i += 1024) sm[i] = 0;
-  for (int t = wid; t < T; t += 32)
+  for (int t = wid; t < T; t += 32) {
     warp_topk<VPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, w + (size_t)t * k);
-  __syncthreads();  // idx (global) is visible to the whole block after the barrier
+    if (ids_in_smem && lane < k) {
+      // warp_topk left slot `lane` of token t in global memory; keep a copy
+      idx_s[t * k + lane] = idx[(size_t)t * k + lane];
+    }
+  }
+  __syncthreads();
+  const int* ids = ids_in_smem ? idx_s : idx;
   const int t = threadIdx.x;
   const bool valid = t < T;
   int my_e[kMaxK];
@@ -395,7 +457,7 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     const int per = R > 1 ? E / R : 1;
     const int src = R > 1 ? t / src_chunk : 0;
     for (int j = 0; j < k; ++j) {
-      const int e = idx[(size_t)t * k + j];
+      const int e = ids[t * k + j];
       bool ok = (e >= 0 && e < E);
       for (int j2 = 0; j2 < j && ok; ++j2) ok = my_e[j2] != e;
       my_e[j] = ok ? e : -1;
@@ -409,28 +471,46 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     }
   }
   __syncthreads();
-  const int c = (threadIdx.x < E) ? hist[threadIdx.x] : 0;
-  const int off = block_exclusive_scan_1024(c, scratch, &total);
-  const int P = total;
-  if (threadIdx.x < E) {
-    counts[threadIdx.x] = c;
-    offsets[threadIdx.x] = off;
-    off_s[threadIdx.x] = off;
+  const int e = threadIdx.x;
+  const int c = (e < E) ? hist[e] : 0;
+  const int nt = (c + kGemmBM - 1) / kGemmBM;
+  const int3 pre = block_exclusive_scan3_1024(make_int3(c, nt, c > 0 ? 1 : 0), warp_tot, &total);
+  const int3 tot = total;
+  if (e < E) {
+    counts[e] = c;
+    offsets[e] = pre.x;
+    off_s[e] = pre.x;
+    int* rt = row_tile_entries(tiles, E);
+    for (int i = 0; i < nt; ++i) {
+      rt[3 * (pre.y + i) + 0] = pre.x + i * kGemmBM;
+      rt[3 * (pre.y + i) + 1] = pre.x + c;
+      rt[3 * (pre.y + i) + 2] = e;
+    }
+    if (c > 0) {
+      int* et = expert_entries(tiles);
+      et[3 * pre.z + 0] = pre.x;
+      et[3 * pre.z + 1] = pre.x + c;
+      et[3 * pre.z + 2] = e;
+    }
   }
-  if (threadIdx.x == 0) offsets[E] = P;
-  write_work_lists(threadIdx.x, E, c, off, tiles, scratch, &total);
-  if (R > 1) {
+  if (threadIdx.x == 0) {
+    offsets[E] = tot.x;
+    tiles[0] = tot.y;
+    tiles[1] = tot.z;
+  }
+  if (R > 1)
     for (int i = threadIdx.x; i < RR; i += 1024) send_out[i] = send[i];
-    if (threadIdx.x <= R) rank_off[threadIdx.x] = (threadIdx.x == R) ? P : off_s[threadIdx.x * (E / R)];
-  }
+  __syncthreads();  // off_s complete
+  if (R > 1 && threadIdx.x <= R)
+    rank_off[threadIdx.x] = (threadIdx.x == R) ? tot.x : off_s[threadIdx.x * (E / R)];
   if (valid) {
     const uint32_t lt = (1u << lane) - 1u;
     for (int j = 0; j < k; ++j) {
-      const int e = my_e[j];
-      if (e < 0) continue;
-      int r = off_s[e];
-      for (int w2 = 0; w2 < wid; ++w2) r += __popc(masks[w2 * E + e]);
-      r += __popc(masks[wid * E + e] & lt);
+      const int ej = my_e[j];
+      if (ej < 0) continue;
+      int r = off_s[ej];
+      for (int w2 = 0; w2 < wid; ++w2) r += __popc(masks[w2 * E + ej]);
+      r += __popc(masks[wid * E + ej] & lt);
       row_of[(size_t)t * k + j] = r;
       perm[r] = t;
     }
@@ -444,6 +524,8 @@ __global__ void __launch_bounds__(kTokensPerRouteBlock) k_scatter(
     const int* __restrict__ idx, int T, int E, int k,
     const int* __restrict__ blockbase, int* __restrict__ row_of,
     int* __restrict__ perm) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint32_t masks[];  // [8][E]
   constexpr int W = kTokensPerRouteBlock / 32;
   for (int i = threadIdx.x; i < W * E; i += blockDim.x) masks[i] = 0;
@@ -478,6 +560,8 @@ __global__ void __launch_bounds__(kTokensPerRouteBlock) k_scatter(
 __global__ void __launch_bounds__(256) k_gather_rows(
     const __nv_bfloat16* __restrict__ x, const int* __restrict__ perm, long long P,
     int T, int d, __nv_bfloat16* __restrict__ x_perm, int* err) {
+  pdl_trigger();
+  pdl_wait();
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= P) return;
   const int lane = threadIdx.x & 31;
@@ -499,6 +583,8 @@ __global__ void __launch_bounds__(256) k_gather_rows(
 __global__ void __launch_bounds__(256) k_combine(
     const __nv_bfloat16* __restrict__ z, const int* __restrict__ row_of,
     const float* __restrict__ w, int T, int d, int k, __nv_bfloat16* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const long long P = (long long)T * k;
   const int nchunk = (d + 255) / 256;
   const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -574,8 +660,35 @@ cudaError_t launch_selftest_bounded_wait(unsigned long long limit_ns, int* err,
 }
 
 // ============================================================== launchers
+// Largest cluster (16 if the device allows non-portable cluster sizes, else
+// 8) whose K slices are whole 64-element chunks.
+static int router_max_cluster() {
+  static int max_cs = 0;
+  if (max_cs == 0) {
+    max_cs = 8;
+    if (cudaFuncSetAttribute(k_router_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1, 1);
+      cfg.blockDim = dim3(256, 1, 1);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_router_cluster, &cfg) == cudaSuccess && n > 0)
+        max_cs = 16;
+    }
+    cudaGetLastError();
+  }
+  return max_cs;
+}
+
 static int router_cluster_size(int d) {
-  for (int cs = 8; cs > 1; cs >>= 1)
+  for (int cs = router_max_cluster(); cs > 1; cs >>= 1)
     if (d % (64 * cs) == 0) return cs;
   return 1;
 }
@@ -583,19 +696,10 @@ static int router_cluster_size(int d) {
 cudaError_t launch_router(const __nv_bfloat16* x, const float* w_g, const float* bias,
                           const moe_shape& s, float* logits, cudaStream_t st) {
   const int cs = router_cluster_size(s.d);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(cs * ((s.E + kRtE - 1) / kRtE)), (unsigned)((s.T + kRtT - 1) / kRtT), 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_router_cluster, x, w_g, bias, s.T, s.d, s.E, logits);
+  const dim3 grid((unsigned)(cs * ((s.E + kRtE - 1) / kRtE)), (unsigned)((s.T + kRtT - 1) / kRtT),
+                  1);
+  return launch_kernel(k_router_cluster, grid, dim3(256), 0, st, cs, x, w_g, bias, s.T, s.d, s.E,
+                       logits);
 }
 
 #define MOE_VPL_DISPATCH(VPL_VAR, CALL) \
@@ -612,10 +716,10 @@ cudaError_t launch_topk(const float* logits, const moe_shape& s, int* idx, float
                         cudaStream_t st) {
   const int blocks = (s.T + 7) / 8;
   const int vpl = (s.E + 31) / 32;
-#define MOE_TOPK_CALL(V) k_topk<V><<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, idx, w)
+#define MOE_TOPK_CALL(V) \
+  return launch_kernel(k_topk<V>, dim3(blocks), dim3(256), 0, st, 1, logits, s.T, s.E, s.k, idx, w)
   MOE_VPL_DISPATCH(vpl, MOE_TOPK_CALL);
 #undef MOE_TOPK_CALL
-  return cudaGetLastError();
 }
 
 template <int VPL>
@@ -627,13 +731,14 @@ static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R,
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_route_fused<VPL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(4 * (2 * kMaxE + kMaxR * kMaxR + 32 * kMaxE)));
+                                         (int)(4 * (2 * kMaxE + kMaxR * kMaxR + 32 * kMaxE +
+                                                    kFusedSmemIdx)));
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_route_fused<VPL><<<1, 1024, smem, st>>>(logits, s.T, s.E, s.k, R, chunk, idx, w, counts,
-                                            offsets, tiles, send, rank_off, row_of, perm, err);
-  return cudaGetLastError();
+  return launch_kernel(k_route_fused<VPL>, dim3(1), dim3(1024), smem, st, 1, logits, s.T, s.E,
+                       s.k, R, chunk, idx, w, counts, offsets, tiles, send, rank_off, row_of,
+                       perm, err);
 }
 
 cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
@@ -642,7 +747,9 @@ cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx
                                cudaStream_t st) {
   const int R = s.R > 1 ? s.R : 0;
   const int chunk = R ? (s.T + R - 1) / R : 1;
-  const size_t smem = sizeof(int) * (2 * s.E + (R ? R * R : 0) + 32 * s.E);
+  const long long tk = (long long)s.T * s.k;
+  const size_t smem = sizeof(int) * (2 * s.E + (R ? R * R : 0) + 32 * s.E +
+                                     (tk <= kFusedSmemIdx ? tk : 0));
   const int vpl = (s.E + 31) / 32;
 #define MOE_FUSED_CALL(V)                                                                 \
   return route_fused_t<V>(logits, s, R, chunk, smem, idx, w, counts, offsets, tiles, send, \
@@ -662,41 +769,37 @@ cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayo
   const int R = s.R > 1 ? s.R : 0;
   const int chunk = R ? (s.T + R - 1) / R : 1;
   const size_t hist_smem = sizeof(int) * (s.E + (R ? R * R : 0));
-  k_hist<<<L.nblocks, kTokensPerRouteBlock, hist_smem, st>>>(
-      idx, s.T, s.E, s.k, R, chunk, blockhist, blocksend, err);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(k_hist, dim3(L.nblocks), dim3(kTokensPerRouteBlock), hist_smem,
+                                st, 1, idx, s.T, s.E, s.k, R, chunk, blockhist, blocksend, err);
   if (e != cudaSuccess) return e;
-  k_scan<<<1, 1024, 0, st>>>(blockhist, L.nblocks, s.E, R, blocksend, blockbase,
-                             counts, offsets, tiles, send, rank_off);
-  e = cudaGetLastError();
+  e = launch_kernel(k_scan, dim3(1), dim3(1024), 0, st, 1, blockhist, L.nblocks, s.E, R,
+                    blocksend, blockbase, counts, offsets, tiles, send, rank_off);
   if (e != cudaSuccess) return e;
   const size_t scat_smem = sizeof(uint32_t) * (kTokensPerRouteBlock / 32) * s.E;
-  k_scatter<<<L.nblocks, kTokensPerRouteBlock, scat_smem, st>>>(
-      idx, s.T, s.E, s.k, blockbase, row_of, perm);
-  return cudaGetLastError();
+  return launch_kernel(k_scatter, dim3(L.nblocks), dim3(kTokensPerRouteBlock), scat_smem, st, 1,
+                       idx, s.T, s.E, s.k, blockbase, row_of, perm);
 }
 
 cudaError_t launch_tiles_from_offsets(const int* offsets, const moe_shape& s,
                                       int* tiles, int* err, cudaStream_t st) {
-  k_tiles_from_offsets<<<1, 1024, 0, st>>>(offsets, s.E, (int)((long long)s.T * s.k),
-                                           tiles, err);
-  return cudaGetLastError();
+  return launch_kernel(k_tiles_from_offsets, dim3(1), dim3(1024), 0, st, 1, offsets, s.E,
+                       (int)((long long)s.T * s.k), tiles, err);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, int T,
                           int d, __nv_bfloat16* x_perm, int* err, cudaStream_t st) {
   if (P == 0) return cudaSuccess;
   const long long blocks = (P + 7) / 8;
-  k_gather_rows<<<(unsigned)blocks, 256, 0, st>>>(x, perm, P, T, d, x_perm, err);
-  return cudaGetLastError();
+  return launch_kernel(k_gather_rows, dim3((unsigned)blocks), dim3(256), 0, st, 1, x, perm, P, T,
+                       d, x_perm, err);
 }
 
 cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const float* w,
                            const moe_shape& s, __nv_bfloat16* y, cudaStream_t st) {
   const long long warps = (long long)s.T * ((s.d + 255) / 256);
   const unsigned blocks = (unsigned)((warps + 7) / 8);
-  k_combine<<<blocks, 256, 0, st>>>(z, row_of, w, s.T, s.d, s.k, y);
-  return cudaGetLastError();
+  return launch_kernel(k_combine, dim3(blocks), dim3(256), 0, st, 1, z, row_of, w, s.T, s.d,
+                       s.k, y);
 }
 
 }  // namespace moe
