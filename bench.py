@@ -43,11 +43,21 @@ KERNEL_SOURCES = ["routing_dispatch_expert_softmax_b200/csrc/moe_gemm_sm100.cu",
                   "routing_dispatch_expert_softmax_b200/csrc/moe_common.cuh",
                   "routing_dispatch_expert_softmax_b200/csrc/moe_routing.cu"]
 
-def launches_per_forward(T):
-    """Kernels one moe_forward launches: router, routing (one fused kernel
-    for T <= 1024, else top-k + histogram + scan + scatter), gather, GEMM1,
-    GEMM2, combine."""
-    return 6 if T <= 1024 else 9
+def launches_per_forward(cfg):
+    """Kernels one moe_forward launches: router (one cluster kernel up to 256
+    tokens; above, the W_g split and the tensor-core GEMM, plus a partial-sum
+    kernel when the GEMM is split into partial planes, i.e. fewer than ~49
+    output tiles), routing (one fused kernel for T <= 1024, else top-k +
+    histogram + scan + scatter), gather, the two expert GEMMs, combine."""
+    T = cfg.T
+    if T <= 256:
+        router = 1
+    else:
+        bn = 128 if cfg.E <= 128 else 256
+        tiles = -(-T // 128) * -(-cfg.E // bn)
+        router = 2 if tiles * 3 >= 148 else 3
+    routing = 1 if T <= 1024 else 4
+    return router + routing + 1 + 2 + 1
 
 
 def parse_args(argv=None):
@@ -496,7 +506,7 @@ def run_ours(args):
                          "(each adds a few us); the headline uses plain graph replays",
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * cfg.d * 2,
                 "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-        "gpu_launches": 2 * launches_per_forward(cfg.T) * args.steps,
+        "gpu_launches": 2 * launches_per_forward(cfg) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -70,7 +70,7 @@ cudaError_t run_router(const __nv_bfloat16* x, const float* w_g, const float* bi
                        int sms, cudaStream_t st) {
   if (s.T >= kRouterTcMinT)
     return launch_router_tc(x, w_g, bias, s, logits, at<__nv_bfloat16>(ws, L.w3),
-                            at<int>(ws, L.err), sms, st);
+                            at<float>(ws, L.logit_part), at<int>(ws, L.err), sms, st);
   return launch_router(x, w_g, bias, s, logits, st);
 }
 

@@ -26,6 +26,28 @@ constexpr int kSwapMaxT = 256;
 // Batches above this many tokens compute router logits on the tensor cores.
 constexpr int kRouterTcMinT = 257;
 
+// Tensor-core router: K = 3d (three bf16 planes of W_g) is split into P
+// partitions of whole 64-wide blocks, each a separate work item writing an
+// fp32 partial plane, so small batches still give about kRouterTargetItems
+// work items.  P = 3*S with S dividing d/64 and at least 4 blocks per part;
+// P = 1 (one item per tile, no partial planes) once the tiles alone give at
+// least a third of the target.
+constexpr int kRouterTargetItems = 148;
+inline int router_tc_parts(const moe_shape& s) {
+  if (s.T < kRouterTcMinT) return 0;
+  const int bn = s.E <= 128 ? 128 : 256;
+  const long long tiles = (long long)((s.T + 127) / 128) * ((s.E + bn - 1) / bn);
+  if (tiles * 3 >= kRouterTargetItems) return 1;  // enough tiles: no partial planes
+  const int kb = s.d / 64;  // 64-wide blocks per plane
+  int best = 1;
+  for (int S = 1; S <= kb; ++S) {
+    if (kb % S != 0 || kb / S < 4) continue;
+    best = S;
+    if (tiles * 3 * S >= kRouterTargetItems) break;
+  }
+  return 3 * best;
+}
+
 // Device error word: ws[0] = first error code, ws[1] = detail (kernel id).
 enum : int { kErrSlot = 0, kErrDetail = 1 };
 
@@ -38,7 +60,7 @@ __device__ __forceinline__ void record_error(int* err, int code, int detail) {
 
 // ----------------------------------------------------------------- workspace
 struct WsLayout {
-  size_t err, w3, logits, idx, w, counts, offsets, blockhist, blockbase,
+  size_t err, w3, logit_part, logits, idx, w, counts, offsets, blockhist, blockbase,
       blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, total;
   int nblocks;      // token blocks of kTokensPerRouteBlock
   int max_mtiles;   // upper bound of 128-row expert tiles
@@ -75,6 +97,7 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   };
   L.err = take(64);
   L.w3 = take(2 * 3 * (size_t)d * E);  // router weight split into 3 bf16 planes
+  L.logit_part = take(sizeof(float) * (size_t)router_tc_parts(s) * T * E);
 
   L.logits = take(sizeof(float) * T * E);
   L.idx = take(sizeof(int) * T * k);

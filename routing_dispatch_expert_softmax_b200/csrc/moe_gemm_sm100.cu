@@ -47,6 +47,8 @@ struct GemmArgs {
   const float* bias;      // kEpiLogits only (may be null)
   int* err;
   int weights_once;       // 1: each B tile is read by one work item (hint evict_first)
+  int kparts;             // K partitions per output tile (kEpiLogits; 1 otherwise)
+  long long part_stride;  // elements between the partial outputs of two partitions
 };
 
 template <int BN, int EPI>
@@ -137,9 +139,11 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
 
   const bool dense = args.tiles == nullptr;
   const int num_mtiles = dense ? (args.dense_rows + kGemmBM - 1) / kGemmBM : args.tiles[0];
-  const int n_tiles = args.n_tiles;
+  const int n_tiles = args.n_tiles * args.kparts;  // output tiles x K partitions
+  const int ntn = args.n_tiles;
   const int total = num_mtiles * n_tiles;
   const int nk = args.K / kGemmBK;
+  const int kpp = nk / args.kparts;  // K blocks per partition
   const int* tl = dense ? nullptr : args.tiles + 4 + 3 * args.E;  // row tiles follow the expert entries
 
   if (warp == 0) {
@@ -158,11 +162,13 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         int mt, nt;
         raster(w, n_tiles, num_mtiles, mt, nt);
+        const int part = nt / ntn, ntile = nt - part * ntn;
         const int row0 = dense ? mt * kGemmBM : tl[3 * mt + 0];
         const int e = dense ? 0 : tl[3 * mt + 2];
-        const int brow = e * args.b_rows_per_expert + nt * (SWIGLU ? BN / 2 : BN);
-        int ka = 0;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int brow = e * args.b_rows_per_expert + ntile * (SWIGLU ? BN / 2 : BN);
+        const int kb0 = part * kpp;
+        int ka = kb0 % args.a_kblocks;
+        for (int kb = kb0; kb < kb0 + kpp; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -207,7 +213,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
         if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(ab * BN);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < kpp; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -240,8 +246,9 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
     const int r_in_tile = q * 32 + lane;
     int it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      int mt, nt;
-      raster(w, n_tiles, num_mtiles, mt, nt);
+      int mt, nt_all;
+      raster(w, n_tiles, num_mtiles, mt, nt_all);
+      const int part = nt_all / ntn, nt = nt_all - part * ntn;
       const int row0 = dense ? mt * kGemmBM : tl[3 * mt + 0];
       const int rowend = dense ? args.dense_rows : tl[3 * mt + 1];
       const int ab = it & 1;
@@ -296,7 +303,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
           }
         }
       } else {
-        float* out = static_cast<float*>(args.out);
+        float* out = static_cast<float*>(args.out) + (size_t)part * args.part_stride;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t a[32];
@@ -738,8 +745,8 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
     return MOE_ERR_CUDA;
   const int nt1 = (int)((s.f + bn / 2 - 1) / (bn / 2));
   const int nt2 = (int)((s.d + bn - 1) / bn);
-  GemmArgs g1{tiles, s.E, 0, nt1, s.d, s.d / kGemmBK, 2 * s.f, s.f, s.f, h, s.f, nullptr, err, 0};
-  GemmArgs g2{tiles, s.E, 0, nt2, s.f, s.f / kGemmBK, s.d, 0, s.d, z, s.d, nullptr, err, 0};
+  GemmArgs g1{tiles, s.E, 0, nt1, s.d, s.d / kGemmBK, 2 * s.f, s.f, s.f, h, s.f, nullptr, err, 0, 1, 0};
+  GemmArgs g2{tiles, s.E, 0, nt2, s.f, s.f / kGemmBK, s.d, 0, s.d, z, s.d, nullptr, err, 0, 1, 0};
   cudaError_t e;
   if (wide) {
     e = launch_gemm_t<256, kEpiSwiGLU>(tA1, tB1, g1, L.max_mtiles * nt1, num_sms, st);
@@ -791,9 +798,23 @@ __global__ void __launch_bounds__(256) k_router_split(const float* __restrict__ 
   }
 }
 
+__global__ void __launch_bounds__(256) k_router_finish(const float* __restrict__ part, int P,
+                                                       long long n, int E,
+                                                       const float* __restrict__ bias,
+                                                       float* __restrict__ logits) {
+  pdl_trigger();
+  pdl_wait();
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    float v = part[i];
+    for (int p = 1; p < P; ++p) v += part[(size_t)p * n + i];
+    logits[i] = bias ? v + bias[i % E] : v;
+  }
+}
+
 cudaError_t launch_router_tc(const __nv_bfloat16* x, const float* w_g, const float* bias,
                              const moe_shape& s, float* logits, __nv_bfloat16* w3,
-                             int* err, int num_sms, cudaStream_t st) {
+                             float* part, int* err, int num_sms, cudaStream_t st) {
   dim3 g((s.d + 31) / 32, (s.E + 31) / 32);
   cudaError_t e = launch_kernel(k_router_split, g, dim3(256), 0, st, 1, w_g, s.d, s.E, w3);
   if (e != cudaSuccess) return e;
@@ -803,10 +824,20 @@ cudaError_t launch_router_tc(const __nv_bfloat16* x, const float* w_g, const flo
       !make_tmap(&tB, w3, (uint64_t)s.E, (uint64_t)3 * s.d, bn))
     return cudaErrorInvalidValue;
   const int nt = (s.E + bn - 1) / bn;
-  GemmArgs a{nullptr, 0, s.T, nt, 3 * s.d, s.d / kGemmBK, 0, 0, s.E, logits, s.E, bias, err, 0};
-  const int work = ((s.T + kGemmBM - 1) / kGemmBM) * nt;
-  if (bn == 128) return launch_gemm_t<128, kEpiLogits>(tA, tB, a, work, num_sms, st);
-  return launch_gemm_t<256, kEpiLogits>(tA, tB, a, work, num_sms, st);
+  const int P = router_tc_parts(s);
+  const long long n = (long long)s.T * s.E;
+  // Each partition writes its own fp32 plane; k_router_finish adds them in
+  // partition order and adds the bias.
+  // P == 1: the GEMM writes the logits (with the bias) directly.
+  GemmArgs a{nullptr, 0, s.T, nt, 3 * s.d, s.d / kGemmBK, 0, 0, s.E, P == 1 ? logits : part,
+             s.E, P == 1 ? bias : nullptr, err, 0, P, n};
+  const int work = ((s.T + kGemmBM - 1) / kGemmBM) * nt * P;
+  e = (bn == 128) ? launch_gemm_t<128, kEpiLogits>(tA, tB, a, work, num_sms, st)
+                  : launch_gemm_t<256, kEpiLogits>(tA, tB, a, work, num_sms, st);
+  if (e != cudaSuccess || P == 1) return e;
+  const int blocks = (int)std::min<long long>((n + 255) / 256, 4L * num_sms);
+  return launch_kernel(k_router_finish, dim3(blocks), dim3(256), 0, st, 1, part, P, n, s.E,
+                       bias, logits);
 }
 
 }  // namespace moe

@@ -12,7 +12,7 @@ cudaError_t launch_router(const __nv_bfloat16* x, const float* w_g, const float*
                           const moe_shape& s, float* logits, cudaStream_t st);
 cudaError_t launch_router_tc(const __nv_bfloat16* x, const float* w_g, const float* bias,
                              const moe_shape& s, float* logits, __nv_bfloat16* w3,
-                             int* err, int num_sms, cudaStream_t st);
+                             float* part, int* err, int num_sms, cudaStream_t st);
 cudaError_t launch_topk(const float* logits, const moe_shape& s, int* idx, float* w,
                         cudaStream_t st);
 // Selection + dispatch tables in one block; valid for T <= kFusedRouteMaxT.

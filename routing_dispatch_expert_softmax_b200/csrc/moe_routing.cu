@@ -158,7 +158,7 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 }
 
 template <int VPL>
-__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k,
+__device__ __forceinline__ void warp_topk_scan(const float* __restrict__ row, int E, int k,
                                           int lane, int* __restrict__ idx_row,
                                           float* __restrict__ w_row) {
   uint32_t key[VPL];
@@ -190,6 +190,94 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, 
     const uint32_t cand = (bi >= 0 && bk == wk) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
     const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
     if ((int)(we & 31) == lane) taken |= 1u << (we >> 5);
+    if (lane == j) {
+      my_key = wk;
+      my_e = (int)we;
+    }
+  }
+  const float my_v = key_value(my_key);
+  const float top = __shfl_sync(0xffffffffu, my_v, 0);
+  const float ex = (lane < k) ? expf(my_v - top) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < k) {
+    idx_row[lane] = my_e;
+    w_row[lane] = ex / sum;
+  }
+}
+
+// Compare-exchange of two (key, slot) candidates so that position a ends up
+// with the one that ranks first: larger key, or equal key and lower slot
+// (the slot order within a lane is the expert-index order).
+__device__ __forceinline__ void cmpx(uint32_t& ka, int& ia, uint32_t& kb, int& ib) {
+  const bool keep = ka > kb || (ka == kb && ia < ib);
+  if (!keep) {
+    const uint32_t tk = ka;
+    ka = kb;
+    kb = tk;
+    const int ti = ia;
+    ia = ib;
+    ib = ti;
+  }
+}
+
+template <int VPL>
+__device__ __forceinline__ void sort_candidates(uint32_t* k, int* i) {
+  if (VPL == 2) {
+    cmpx(k[0], i[0], k[1], i[1]);
+  } else if (VPL == 4) {
+    cmpx(k[0], i[0], k[1], i[1]);
+    cmpx(k[2], i[2], k[3], i[3]);
+    cmpx(k[0], i[0], k[2], i[2]);
+    cmpx(k[1], i[1], k[3], i[3]);
+    cmpx(k[1], i[1], k[2], i[2]);
+  } else if (VPL == 8) {
+    // odd-even merge sorting network, 19 comparators
+    const int net[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6},
+                            {5, 7}, {1, 2}, {5, 6}, {0, 4}, {3, 7}, {1, 5}, {2, 6},
+                            {1, 4}, {3, 6}, {2, 4}, {3, 5}, {3, 4}};
+#pragma unroll
+    for (int c = 0; c < 19; ++c) cmpx(k[net[c][0]], i[net[c][0]], k[net[c][1]], i[net[c][1]]);
+  }
+}
+
+// Up to 256 experts (at most 8 per lane): each lane sorts its candidates
+// once, then every round compares only the lanes' heads -- one redux.sync for
+// the largest key, one for the lowest index holding it -- and the winning lane
+// drops its head.  A lane's head is its best candidate and, among equal keys,
+// its lowest index, so the round picks the same expert as the rank order.
+template <int VPL>
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k, int lane,
+                                          int* __restrict__ idx_row, float* __restrict__ w_row) {
+  if (VPL > 8) {
+    warp_topk_scan<VPL>(row, E, k, lane, idx_row, w_row);
+    return;
+  }
+  constexpr int V = VPL > 8 ? 8 : VPL;
+  uint32_t key[V];
+  int slot[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = (e < E) ? order_key(row[e]) : 0u;  // 0: below every finite key
+    slot[i] = i;
+  }
+  sort_candidates<V>(key, slot);
+  uint32_t my_key = 0;
+  int my_e = 0;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t cand = (key[0] == wk) ? (uint32_t)(lane + 32 * slot[0]) : 0xffffffffu;
+    const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
+    if ((int)(we & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i + 1 < V; ++i) {
+        key[i] = key[i + 1];
+        slot[i] = slot[i + 1];
+      }
+      key[V - 1] = 0u;
+    }
     if (lane == j) {
       my_key = wk;
       my_e = (int)we;
