@@ -23,6 +23,15 @@ constexpr int kMaxR = 64;
 // run the expert GEMMs in swap-AB form.
 constexpr int kSwapMaxT = 256;
 
+// Large batches whose experts average at least one full 128-row tile run the
+// expert GEMMs on CTA pairs (256-row tiles); their work lists then give every
+// expert an even number of 128-row tiles so that a pair never straddles two
+// experts.  Between kSwapMaxT and this density the single-CTA kernel keeps
+// 128-row tiles (sparse experts would pay twice the padding in pairs).
+inline bool pair_tiles(const moe_shape& s) {
+  return s.T > kSwapMaxT && (long long)s.T * s.k >= (long long)128 * s.E;
+}
+
 // Batches above this many tokens compute router logits on the tensor cores.
 constexpr int kRouterTcMinT = 257;
 
@@ -63,7 +72,7 @@ struct WsLayout {
   size_t err, w3, logit_part, logits, idx, w, counts, offsets, blockhist, blockbase,
       blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, total;
   int nblocks;      // token blocks of kTokensPerRouteBlock
-  int max_mtiles;   // upper bound of 128-row expert tiles
+  int max_mtiles;   // upper bound of 128-row expert tiles (each expert padded to an even count)
   long long P;      // T * k
   long long Ppad;   // rows of x_perm / h including the TMA padding
 };
@@ -87,7 +96,7 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   L.P = T * k;
   L.Ppad = L.P + kGemmBM;
   L.nblocks = (int)((T + kTokensPerRouteBlock - 1) / kTokensPerRouteBlock);
-  L.max_mtiles = (int)((L.P + kGemmBM - 1) / kGemmBM + E);
+  L.max_mtiles = (int)((L.P + kGemmBM - 1) / kGemmBM + 2 * E);  // + padding to tile pairs
   (void)num_sms;
   size_t o = 0;
   auto take = [&](size_t bytes) {

@@ -334,6 +334,307 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ============================================================== large-batch kernel, CTA pairs
+// Expert GEMMs for large batches on pairs of SMs (tcgen05 cta_group::2).  A
+// 2-CTA cluster owns a 256-row x 256-column output tile; each CTA loads its
+// own 128 activation rows and 128 of the 256 weight rows (GEMM1: the leader
+// the gate rows, the peer the up rows), so a K-stage costs each CTA 32 KB of
+// operand traffic instead of 48 KB for the same MMA work per SM.  The leader's
+// single MMA thread issues M=256 x N=256 MMAs that read both CTAs' shared
+// memory and write 128 rows x 256 columns into each CTA's TMEM.
+//   full[s]   (leader only) armed by the leader with both CTAs' bytes; the
+//             peer's TMA loads complete on it through the cluster address
+//   empty[s]  (both) freed by the leader's multicast commit
+//   tfull[a]  (both) accumulator ready, multicast commit
+//   tempty[a] (leader only) 128 + 128 epilogue arrivals, the peer's remote
+// Work lists give every expert an even number of 128-row tiles, so tile pair
+// p = (2p, 2p+1) stays inside one expert.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* tm,
+                                                 uint32_t leader_bar, int c0, int c1,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(leader_bar), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_ss_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives once on the barrier at this offset in every CTA of `mask` when all
+// tcgen05.mma issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar, uint32_t cta) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(cta)
+      : "memory");
+}
+
+template <int EPI>
+struct PairCfg {
+  static constexpr int kStages = 6;
+  static constexpr int kABytes = 128 * kGemmBK * 2;  // this CTA's 128 activation rows
+  static constexpr int kBBytes = 128 * kGemmBK * 2;  // this CTA's 128 weight rows
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 512;  // two 128 x 256 fp32 accumulators
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    const GemmArgs args) {
+  using C = PairCfg<EPI>;
+  constexpr int S = C::kStages;
+  constexpr int BN = 256;
+  constexpr bool SWIGLU = (EPI == kEpiSwiGLU);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(&full[s2], 1);
+      mbar_init(&empty[s2], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 256);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer signals the leader's barriers only after both are set up
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // the work lists and operands come from the previous kernels
+
+  const int num_pairs = args.tiles[0] / 2;
+  const int n_tiles = args.n_tiles;
+  const int total = num_pairs * n_tiles;
+  const int nk = args.K / kGemmBK;
+  const int* tl = args.tiles + 4 + 3 * args.E;  // row tiles follow the expert entries
+  const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer (both CTAs)
+      const uint64_t pol = policy_evict_normal();
+      int fills[S];
+#pragma unroll
+      for (int s2 = 0; s2 < S; ++s2) fills[s2] = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int w = cluster_id; w < total && ok; w += num_clusters) {
+        int mp, nt;
+        raster(w, n_tiles, num_pairs, mp, nt);
+        const int row0 = tl[3 * (2 * mp) + 0];
+        const int e = tl[3 * (2 * mp) + 2];
+        const int a_row = row0 + (int)rank * 128;
+        const int b_row = SWIGLU ? e * args.b_rows_per_expert + nt * 128 + (int)rank * args.up_offset
+                                 : e * args.b_rows_per_expert + nt * BN + (int)rank * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = smem + stage * C::kStageBytes;
+          uint8_t* b_dst = a_dst + C::kABytes;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+          const uint32_t lbar = smem_u32(&full[stage]) & 0xFEFFFFFFu;  // the leader's barrier
+          tma_load_2d_pair(a_dst, &tmA, lbar, kb * kGemmBK, a_row, pol);
+          tma_load_2d_pair(b_dst, &tmB, lbar, kb * kGemmBK, b_row, pol);
+          ++fills[stage];
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag && leader) {
+#pragma unroll
+        for (int s2 = 0; s2 < S; ++s2)
+          if (fills[s2] > 0) mbar_wait_limit(&full[s2], (uint32_t)((fills[s2] - 1) & 1), 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------ MMA issuer (leader)
+      constexpr uint32_t idesc = idesc_bf16_f32(256, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = cluster_id; w < total && ok; w += num_clusters, ++it) {
+        const int ab = it & 1;
+        const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(ab * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk)
+            umma_bf16_ss_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                              sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(&empty[stage], 0x3);  // frees this stage in both CTAs
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit_pair_mc(&tfull[ab], 0x3);
+      }
+      if (*abort_flag) {
+        umma_commit_pair(drain);
+        mbar_wait_limit(drain, 0, 100000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    int it = 0;
+    for (int w = cluster_id; w < total; w += num_clusters, ++it) {
+      int mp, nt;
+      raster(w, n_tiles, num_pairs, mp, nt);
+      const int row0 = tl[3 * (2 * mp) + 0];
+      const int rowend = tl[3 * (2 * mp) + 1];
+      const int ab = it & 1;
+      const uint32_t aph = (uint32_t)((it >> 1) & 1);
+      const bool got = mbar_wait_bounded(&tfull[ab], aph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t t_addr = tmem_base + (uint32_t)(ab * BN) + ((uint32_t)(q * 32) << 16);
+      const int row = row0 + (int)rank * 128 + q * 32 + lane;
+      const bool row_ok = row < rowend;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+      if (SWIGLU) {
+        constexpr int H = BN / 2;
+#pragma unroll 1
+        for (int c = 0; c < H; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(t_addr + c, g);
+          tmem_ld_32x32b_x32(t_addr + H + c, u);
+          tmem_ld_wait();
+          const int col = nt * H + c;
+          if (row_ok && col < args.n_out) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              p[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * args.ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(t_addr + c, a);
+          tmem_ld_wait();
+          const int col = nt * BN + c;
+          if (row_ok && col < args.n_out) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              p[i] = pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * args.ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      if (leader) mbar_arrive(&tempty[ab]);
+      else mbar_arrive_cta(&tempty[ab], 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the leader's MMAs read this CTA's shared memory until here
+  tc_fence_after();
+  if (threadIdx.x == 0 && *abort_flag) record_error(args.err, MOE_ERR_TIMEOUT, 13);
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::kTmemCols)
+                 : "memory");
+}
+
 // ============================================================== small-batch kernel
 // Swap-AB form for batches of at most NMAX tokens per expert (decode): the
 // expert's weights are the M = 128 operand (128 weight rows per work item:
@@ -716,6 +1017,25 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+template <int EPI>
+static cudaError_t launch_gemm_2sm(const CUtensorMap& ta, const CUtensorMap& tb,
+                                   const GemmArgs& args, int max_pairs_work, int num_sms,
+                                   cudaStream_t st) {
+  using C = PairCfg<EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_2sm<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int clusters = max_pairs_work < num_sms / 2 ? max_pairs_work : num_sms / 2;
+  if (clusters < 1) clusters = 1;
+  return launch_kernel(k_grouped_gemm_2sm<EPI>, dim3(2 * clusters), dim3(192), C::kSmemBytes, st,
+                       2, ta, tb, args);
+}
+
 // Both expert GEMMs over the rows described by the device tile list.
 //   x_rows: rows of x_perm visible to TMA (P for a caller buffer, Ppad inside
 //   the workspace); h has Ppad rows (workspace).
@@ -735,20 +1055,29 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
-  const bool wide = (L.P >= 64LL * s.E);  // many rows per expert: 256-wide tiles
+  const bool pairs = pair_tiles(s);  // the work lists hold tile pairs
+  const bool wide = pairs || (L.P >= 64LL * s.E);  // many rows per expert: 256-wide tiles
   CUtensorMap tA1, tB1, tA2, tB2;
   const uint32_t bn = wide ? 256 : 128;
+  // Each CTA of a pair loads 128 of the 256 weight rows of a tile.
+  const uint32_t b1_box = pairs ? 128 : bn / 2, b2_box = pairs ? 128 : bn;
   if (!make_tmap(&tA1, x_perm, (uint64_t)x_rows, (uint64_t)s.d, kGemmBM) ||
-      !make_tmap(&tB1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, bn / 2) ||
+      !make_tmap(&tB1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, b1_box) ||
       !make_tmap(&tA2, h, (uint64_t)L.Ppad, (uint64_t)s.f, kGemmBM) ||
-      !make_tmap(&tB2, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, bn))
+      !make_tmap(&tB2, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, b2_box))
     return MOE_ERR_CUDA;
   const int nt1 = (int)((s.f + bn / 2 - 1) / (bn / 2));
   const int nt2 = (int)((s.d + bn - 1) / bn);
   GemmArgs g1{tiles, s.E, 0, nt1, s.d, s.d / kGemmBK, 2 * s.f, s.f, s.f, h, s.f, nullptr, err, 0, 1, 0};
   GemmArgs g2{tiles, s.E, 0, nt2, s.f, s.f / kGemmBK, s.d, 0, s.d, z, s.d, nullptr, err, 0, 1, 0};
   cudaError_t e;
-  if (wide) {
+  if (pairs) {
+    const int max_pairs = (L.max_mtiles + 1) / 2;
+    e = launch_gemm_2sm<kEpiSwiGLU>(tA1, tB1, g1, max_pairs * nt1, num_sms, st);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess)
+      e = launch_gemm_2sm<kEpiStore>(tA2, tB2, g2, max_pairs * nt2, num_sms, st);
+  } else if (wide) {
     e = launch_gemm_t<256, kEpiSwiGLU>(tA1, tB1, g1, L.max_mtiles * nt1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)

@@ -377,8 +377,9 @@ __device__ int block_exclusive_scan_1024(int v, int* scratch /*[32]*/, int* tota
 // 1024-thread block calls this; thread e < E passes expert e's row count c
 // and first row off.
 __device__ void write_work_lists(int e, int E, int c, int off, int* tiles, int* scratch,
-                                 int* total) {
-  const int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
+                                 int* total, bool pair) {
+  int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
+  if (pair) nt = (nt + 1) & ~1;  // 256-row tiles of CTA pairs never straddle experts
   const int tb = block_exclusive_scan_1024(nt, scratch, total);
   if (threadIdx.x == 0) tiles[0] = *total;
   int* rt = row_tile_entries(tiles, E);
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(1024) k_scan(
     const int* __restrict__ blockhist, int nblocks, int E, int R,
     const int* __restrict__ blocksend, int* __restrict__ blockbase,
     int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ tiles,
-    int* __restrict__ send, int* __restrict__ rank_off) {
+    int* __restrict__ send, int* __restrict__ rank_off, int pair) {
   pdl_trigger();
   pdl_wait();
   __shared__ int scratch[32];
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(1024) k_scan(
     for (int b = 0; b < nblocks; ++b) blockbase[(size_t)b * E + e] += off;
   }
   if (e == 0) offsets[E] = P;
-  write_work_lists(e, E, c, off, tiles, scratch, &total);
+  write_work_lists(e, E, c, off, tiles, scratch, &total, pair != 0);
   if (R > 1) {
     for (int i = threadIdx.x; i < R * R; i += blockDim.x) {
       int s = 0;
@@ -443,7 +444,8 @@ __global__ void __launch_bounds__(1024) k_scan(
 
 // Tile list from caller-provided offsets (moe_ffn); checks the offsets.
 __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
-    const int* __restrict__ offsets, int E, int P, int* __restrict__ tiles, int* err) {
+    const int* __restrict__ offsets, int E, int P, int* __restrict__ tiles, int* err,
+    int pair) {
   pdl_trigger();
   pdl_wait();
   __shared__ int scratch[32];
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
       c = 0;
     }
   }
-  write_work_lists(e, E, c, a, tiles, scratch, &total);
+  write_work_lists(e, E, c, a, tiles, scratch, &total, pair != 0);
 }
 
 // ============================================================== fused routing, T <= 1024
@@ -514,7 +516,8 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     const float* __restrict__ logits, int T, int E, int k, int R, int src_chunk,
     int* __restrict__ idx, float* __restrict__ w, int* __restrict__ counts,
     int* __restrict__ offsets, int* __restrict__ tiles, int* __restrict__ send_out,
-    int* __restrict__ rank_off, int* __restrict__ row_of, int* __restrict__ perm, int* err) {
+    int* __restrict__ rank_off, int* __restrict__ row_of, int* __restrict__ perm, int* err,
+    int pair) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int sm[];
@@ -561,7 +564,8 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   __syncthreads();
   const int e = threadIdx.x;
   const int c = (e < E) ? hist[e] : 0;
-  const int nt = (c + kGemmBM - 1) / kGemmBM;
+  int nt = (c + kGemmBM - 1) / kGemmBM;
+  if (pair) nt = (nt + 1) & ~1;  // pairs of 128-row tiles for the 2-SM GEMM
   const int3 pre = block_exclusive_scan3_1024(make_int3(c, nt, c > 0 ? 1 : 0), warp_tot, &total);
   const int3 tot = total;
   if (e < E) {
@@ -826,7 +830,7 @@ static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R,
   }
   return launch_kernel(k_route_fused<VPL>, dim3(1), dim3(1024), smem, st, 1, logits, s.T, s.E,
                        s.k, R, chunk, idx, w, counts, offsets, tiles, send, rank_off, row_of,
-                       perm, err);
+                       perm, err, pair_tiles(s) ? 1 : 0);
 }
 
 cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
@@ -861,7 +865,8 @@ cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayo
                                 st, 1, idx, s.T, s.E, s.k, R, chunk, blockhist, blocksend, err);
   if (e != cudaSuccess) return e;
   e = launch_kernel(k_scan, dim3(1), dim3(1024), 0, st, 1, blockhist, L.nblocks, s.E, R,
-                    blocksend, blockbase, counts, offsets, tiles, send, rank_off);
+                    blocksend, blockbase, counts, offsets, tiles, send, rank_off,
+                    pair_tiles(s) ? 1 : 0);
   if (e != cudaSuccess) return e;
   const size_t scat_smem = sizeof(uint32_t) * (kTokensPerRouteBlock / 32) * s.E;
   return launch_kernel(k_scatter, dim3(L.nblocks), dim3(kTokensPerRouteBlock), scat_smem, st, 1,
@@ -871,7 +876,7 @@ cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayo
 cudaError_t launch_tiles_from_offsets(const int* offsets, const moe_shape& s,
                                       int* tiles, int* err, cudaStream_t st) {
   return launch_kernel(k_tiles_from_offsets, dim3(1), dim3(1024), 0, st, 1, offsets, s.E,
-                       (int)((long long)s.T * s.k), tiles, err);
+                       (int)((long long)s.T * s.k), tiles, err, pair_tiles(s) ? 1 : 0);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, int T,

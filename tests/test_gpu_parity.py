@@ -389,6 +389,20 @@ def test_forward_deepseek(T):
     _check_forward(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=None if T == 1 else _token_sample(6))
 
 
+@pytest.mark.parametrize("cfg", [
+    # 2-SM tile pairs, routing in one block (T <= 1024)
+    wl.MoEConfig("pairs-fused", T=1000, d=256, E=8, k=2, f=512),
+    # 2-SM tile pairs, multi-block routing; d and f not multiples of 256 / 128
+    wl.MoEConfig("pairs-tables", T=1100, d=192, E=4, k=1, f=320),
+    # sparse experts: single-CTA 128 x 128 tiles
+    wl.MoEConfig("narrow", T=600, d=256, E=64, k=2, f=256),
+    # single-CTA 128 x 256 tiles
+    wl.MoEConfig("wide", T=700, d=256, E=16, k=2, f=256),
+], ids=lambda c: c.name)
+def test_forward_large_batch_gemm_regimes(cfg):
+    _check_forward(cfg)
+
+
 def test_forward_k_equals_E_and_single_expert():
     _check_forward(wl.MoEConfig("dense-k=E", T=70, d=128, E=4, k=4, f=128))
     _check_forward(wl.MoEConfig("E=1", T=33, d=256, E=1, k=1, f=192))
