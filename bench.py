@@ -46,8 +46,9 @@ KERNEL_SOURCES = ["routing_dispatch_expert_softmax_b200/csrc/moe_gemm_sm100.cu",
 def launches_per_forward(cfg):
     """Kernels one moe_forward launches: router (one cluster kernel up to 256
     tokens; above, the W_g split and the tensor-core GEMM, plus a partial-sum
-    kernel when the GEMM is split into partial planes, i.e. fewer than ~49
-    output tiles), routing (one fused kernel for T <= 1024, else top-k +
+    kernel when the GEMM's K is split into P > 1 partial planes: P is the
+    largest divisor of the 3d/64 K blocks, at most a quarter of them, with
+    tiles * P <= 148), routing (one fused kernel for T <= 1024, else top-k +
     histogram + scan + scatter), gather, the two expert GEMMs, combine."""
     T = cfg.T
     if T <= 256:
@@ -55,7 +56,15 @@ def launches_per_forward(cfg):
     else:
         bn = 128 if cfg.E <= 128 else 256
         tiles = -(-T // 128) * -(-cfg.E // bn)
-        router = 2 if tiles * 3 >= 148 else 3
+        nk = 3 * cfg.d // 64
+        parts = 1
+        for p in range(2, nk // 4 + 1):
+            if nk % p:
+                continue
+            if tiles * p > 148:
+                break
+            parts = p
+        router = 2 if parts == 1 else 3
     routing = 1 if T <= 1024 else 4
     return router + routing + 1 + 2 + 1
 

@@ -36,25 +36,25 @@ inline bool pair_tiles(const moe_shape& s) {
 constexpr int kRouterTcMinT = 257;
 
 // Tensor-core router: K = 3d (three bf16 planes of W_g) is split into P
-// partitions of whole 64-wide blocks, each a separate work item writing an
-// fp32 partial plane, so small batches still give about kRouterTargetItems
-// work items.  P = 3*S with S dividing d/64 and at least 4 blocks per part;
-// P = 1 (one item per tile, no partial planes) once the tiles alone give at
-// least a third of the target.
+// partitions of whole 64-wide blocks (at least 4 per part), each a separate
+// work item writing an fp32 partial plane that a finish kernel adds in
+// partition order.  P is the largest divisor of the block count that keeps
+// tiles * P within one wave of kRouterTargetItems work items: a 128 x E
+// logit tile streams 32 KB of operands per 64-deep K block, so one SM alone
+// cannot feed its tensor cores and the tiles must be spread over all SMs.
 constexpr int kRouterTargetItems = 148;
 inline int router_tc_parts(const moe_shape& s) {
   if (s.T < kRouterTcMinT) return 0;
   const int bn = s.E <= 128 ? 128 : 256;
   const long long tiles = (long long)((s.T + 127) / 128) * ((s.E + bn - 1) / bn);
-  if (tiles * 3 >= kRouterTargetItems) return 1;  // enough tiles: no partial planes
-  const int kb = s.d / 64;  // 64-wide blocks per plane
+  const int nk = 3 * s.d / 64;  // 64-wide K blocks over the three planes
   int best = 1;
-  for (int S = 1; S <= kb; ++S) {
-    if (kb % S != 0 || kb / S < 4) continue;
-    best = S;
-    if (tiles * 3 * S >= kRouterTargetItems) break;
+  for (int P = 2; P <= nk / 4; ++P) {
+    if (nk % P != 0) continue;
+    if (tiles * P > kRouterTargetItems) break;
+    best = P;
   }
-  return 3 * best;
+  return best;
 }
 
 // Device error word: ws[0] = first error code, ws[1] = detail (kernel id).

@@ -413,7 +413,10 @@ struct PairCfg {
   static constexpr int kBBytes = 128 * kGemmBK * 2;  // this CTA's 128 weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;  // two 128 x 256 fp32 accumulators
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+  // Per epilogue warp: 32 rows x 128 bytes of output staged for full-line
+  // stores (the plain-store epilogue only).
+  static constexpr int kOutStageBytes = EPI == kEpiStore ? 4 * 32 * 128 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kOutStageBytes + 1024 + 256;
 };
 
 template <int EPI>
@@ -427,7 +430,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint4* out_stage = reinterpret_cast<uint4*>(smem + S * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kOutStageBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -560,7 +564,14 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
     }
   } else {
     // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    // Each warp owns TMEM lanes q*32.. (32 output rows).  GEMM2: a 64-column
+    // slice is packed to bf16, written row by row into the warp's staging
+    // tile (16-byte chunks XOR-swizzled by row: no bank conflicts either way)
+    // and read back so that every store instruction writes 4 full 128-byte
+    // rows instead of half sectors of 32 rows.
     const int q = warp & 3;
+    uint4* st_tile = out_stage + (size_t)(warp - 2) * 32 * 8;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int it = 0;
     for (int w = cluster_id; w < total; w += num_clusters, ++it) {
       int mp, nt;
@@ -573,11 +584,29 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t t_addr = tmem_base + (uint32_t)(ab * BN) + ((uint32_t)(q * 32) << 16);
-      const int row = row0 + (int)rank * 128 + q * 32 + lane;
-      const bool row_ok = row < rowend;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+      const int row_base = row0 + (int)rank * 128 + q * 32;
+      // Stores the staged 32 x 64 slice at output column col0 (a multiple of
+      // 64; n_out is one too, so a slice is wholly inside or outside).
+      auto drain_slice = [&](int col0) {
+        __syncwarp();
+        if (col0 < args.n_out) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = i * 4 + (lane >> 3), v = lane & 7;
+            const uint4 val = st_tile[r * 8 + (v ^ (r & 7))];
+            if (row_base + r < rowend)
+              *reinterpret_cast<uint4*>(out + (size_t)(row_base + r) * args.ld_out + col0 + v * 8) =
+                  val;
+          }
+        }
+        __syncwarp();
+      };
       if (SWIGLU) {
+        // h is half as wide as the accumulator; direct 16-byte stores measured
+        // faster here than the staged path.
         constexpr int H = BN / 2;
+        const int row = row_base + lane;
+        const bool row_ok = row < rowend;
 #pragma unroll 1
         for (int c = 0; c < H; c += 32) {
           uint32_t g[32], u[32];
@@ -601,21 +630,24 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t a[32];
-          tmem_ld_32x32b_x32(t_addr + c, a);
-          tmem_ld_wait();
-          const int col = nt * BN + c;
-          if (row_ok && col < args.n_out) {
+        for (int c = 0; c < BN; c += 64) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t a[32];
+            tmem_ld_32x32b_x32(t_addr + c + 32 * half, a);
+            tmem_ld_wait();
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               p[i] = pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * args.ld_out + col);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) {
+              const int chunk = 4 * half + v;
+              st_tile[lane * 8 + (chunk ^ (lane & 7))] =
+                  make_uint4(p[4 * v], p[4 * v + 1], p[4 * v + 2], p[4 * v + 3]);
+            }
           }
+          drain_slice(nt * BN + c);
         }
       }
       tc_fence_before();

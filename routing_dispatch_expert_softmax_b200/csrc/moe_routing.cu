@@ -119,10 +119,19 @@ __global__ void __launch_bounds__(256) k_router_cluster(
     __syncthreads();
     if (kc + kRtKC < kend)
       router_load(regs, x, w_g, T, d, E, t0, e0, kc + kRtKC, min(kRtKC, kend - kc - kRtKC));
-    for (int kk = 0; kk < chunk; ++kk) {
-      const float wv = ws[kk][tx];
+    for (int kk = 0; kk < chunk; kk += 4) {  // same FMA order as one kk at a time
+      float4 xv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fmaf(xs[ty + 8 * i][kk], wv, acc[i]);
+      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(&xs[ty + 8 * i][kk]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float wv = ws[kk + j][tx];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float xe = j == 0 ? xv[i].x : j == 1 ? xv[i].y : j == 2 ? xv[i].z : xv[i].w;
+          acc[i] = fmaf(xe, wv, acc[i]);
+        }
+      }
     }
     __syncthreads();
   }
@@ -131,8 +140,14 @@ __global__ void __launch_bounds__(256) k_router_cluster(
   cl.sync();
   const int per = (kRtT * kRtE) / CS;
   for (int o = rank * per + threadIdx.x; o < (rank + 1) * per; o += 256) {
+    // all CS remote loads in flight at once, then the sum in rank order
+    float pv[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) pv[r] = r < CS ? *cl.map_shared_rank(&part[o], r) : 0.f;
     float v = 0.f;
-    for (int r = 0; r < CS; ++r) v += *cl.map_shared_rank(&part[o], r);
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      if (r < CS) v += pv[r];
     const int t = t0 + o / kRtE, e = e0 + (o % kRtE);
     if (t < T && e < E) logits[(size_t)t * E + e] = bias ? v + bias[e] : v;
   }
