@@ -39,9 +39,10 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+# The sources of the expert GEMM kernels whose DRAM traffic profiles/traffic.json
+# records (the kernels and the header they are built from).
 KERNEL_SOURCES = ["routing_dispatch_expert_softmax_b200/csrc/moe_gemm_sm100.cu",
-                  "routing_dispatch_expert_softmax_b200/csrc/moe_common.cuh",
-                  "routing_dispatch_expert_softmax_b200/csrc/moe_routing.cu"]
+                  "routing_dispatch_expert_softmax_b200/csrc/moe_common.cuh"]
 
 def launches_per_forward(cfg):
     """Kernels one moe_forward launches: router (one cluster kernel up to 256
