@@ -384,8 +384,11 @@ def test_forward_mixtral_sampled():
     _check_forward(wl.MIXTRAL_8X7B, sample=_token_sample(24))
 
 
-@pytest.mark.parametrize("T", [1, 64])
+@pytest.mark.parametrize("T", [1, 64, 512, 16384])
 def test_forward_deepseek(T):
+    # T = 512: single-CTA tiles over sparse experts; T = 16384: multi-block
+    # routing tables and CTA-pair tiles with E = 256.  The sampled tokens
+    # include ones routed to the hottest and the coldest expert.
     _check_forward(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=None if T == 1 else _token_sample(6))
 
 
