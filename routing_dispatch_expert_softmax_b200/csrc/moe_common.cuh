@@ -24,10 +24,9 @@ constexpr int kMaxR = 64;
 constexpr int kSwapMaxT = 256;
 
 // Large batches whose experts average at least one full 128-row tile run the
-// expert GEMMs on CTA pairs (256-row tiles); their work lists then give every
-// expert an even number of 128-row tiles so that a pair never straddles two
-// experts.  Between kSwapMaxT and this density the single-CTA kernel keeps
-// 128-row tiles (sparse experts would pay twice the padding in pairs).
+// expert GEMMs on CTA pairs (256-row tiles); their work lists then split each
+// expert's tiles into pairs and at most one leftover tile.  Between kSwapMaxT
+// and this density the single-CTA kernel runs all 128-row tiles.
 inline bool pair_tiles(const moe_shape& s) {
   return s.T > kSwapMaxT && (long long)s.T * s.k >= (long long)128 * s.E;
 }
@@ -72,7 +71,7 @@ struct WsLayout {
   size_t err, w3, logit_part, logits, idx, w, counts, offsets, blockhist, blockbase,
       blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, total;
   int nblocks;      // token blocks of kTokensPerRouteBlock
-  int max_mtiles;   // upper bound of 128-row expert tiles (each expert padded to an even count)
+  int max_mtiles;   // upper bound of 128-row expert tiles
   long long P;      // T * k
   long long Ppad;   // rows of x_perm / h including the TMA padding
 };
@@ -80,14 +79,27 @@ struct WsLayout {
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Work lists the routing kernels build for the expert GEMMs, in one int
-// buffer: [0] = number of 128-row tiles, [1] = number of touched experts,
-// then E entries (row0, row_end, expert) for the touched experts in expert
-// order, then the row tiles (row0, row_end, expert), 128 rows each.
+// buffer: [0] = number of 128-row tiles in the row-tile list, [1] = number of
+// touched experts, [2] = number of leftover tiles; then E entries (row0,
+// row_end, expert) for the touched experts in expert order, then E leftover
+// entries, then the row tiles (row0, row_end, expert), 128 rows each.  When
+// the expert GEMMs run on CTA pairs (pair_row_tiles), an expert's tile count
+// is rounded up to an even number so pairs never span experts, except that an
+// expert with a single tile goes to the leftover list, which a single-CTA
+// kernel runs; otherwise every tile is a row tile and the leftover list is
+// empty.
+// Row tiles of an expert with nt 128-row tiles in the CTA-pair layout.  An
+// odd count is padded to the next pair: the pair's empty half costs MMA work
+// but the expert's weights stream through L2 once.  A lone tile (nt = 1)
+// would be half empty, so it runs as a single-CTA leftover tile instead.
+__host__ __device__ inline int pair_row_tiles(int nt) { return nt == 1 ? 0 : (nt + 1) & ~1; }
+
 __host__ __device__ inline size_t tile_list_ints(int max_mtiles, int E) {
-  return 4 + 3 * ((size_t)max_mtiles + (size_t)E);
+  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E);
 }
 __host__ __device__ inline int* expert_entries(int* tiles) { return tiles + 4; }
-__host__ __device__ inline int* row_tile_entries(int* tiles, int E) { return tiles + 4 + 3 * E; }
+__host__ __device__ inline int* leftover_entries(int* tiles, int E) { return tiles + 4 + 3 * E; }
+__host__ __device__ inline int* row_tile_entries(int* tiles, int E) { return tiles + 4 + 6 * E; }
 
 inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   WsLayout L{};
@@ -96,7 +108,8 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
   L.P = T * k;
   L.Ppad = L.P + kGemmBM;
   L.nblocks = (int)((T + kTokensPerRouteBlock - 1) / kTokensPerRouteBlock);
-  L.max_mtiles = (int)((L.P + kGemmBM - 1) / kGemmBM + 2 * E);  // + padding to tile pairs
+  // each expert: one partial tile and, in the CTA-pair layout, one padding tile
+  L.max_mtiles = (int)((L.P + kGemmBM - 1) / kGemmBM + 2 * E);
   (void)num_sms;
   size_t o = 0;
   auto take = [&](size_t bytes) {

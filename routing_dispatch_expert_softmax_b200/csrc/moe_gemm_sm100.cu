@@ -32,9 +32,24 @@ enum : int {
   kEpiLogits = 2   // fp32 accumulator + bias[col] (router logits)
 };
 
+// Where a GEMM kernel synchronises with the kernels before and after it
+// (programmatic dependent launch):
+//   kPdlStart:     lets the next kernel launch, then waits for the previous one
+//                  before touching its outputs (the usual chain).
+//   kPdlAfterWait: waits first, then lets the next kernel launch, so the next
+//                  kernel may read everything complete before this one began.
+//   kPdlTail:      reads only data complete before the previous kernel began
+//                  (which must be kPdlAfterWait), so it starts without waiting
+//                  and fills the SMs the previous kernel's tail leaves idle; it
+//                  lets the next kernel launch at once (so that kernel's set-up
+//                  is not exposed) and waits for the previous kernel at its
+//                  end, so its own completion implies both.
+enum : int { kPdlStart = 0, kPdlAfterWait = 1, kPdlTail = 2 };
+
 struct GemmArgs {
-  const int* tiles;       // device work lists; nullptr = dense rows [0, dense_rows)
-  int E;                  // experts (the row tiles follow E expert entries)
+  const int* tile_count;  // device number of row tiles; nullptr = dense rows [0, dense_rows)
+  const int* tile_rows;   // (row0, row_end, expert) per 128-row tile
+  int E;                  // experts
   int dense_rows;         // rows of A in dense mode
   int n_tiles;            // output tiles of width BN (BN/2 for SwiGLU) per row tile
   int K;                  // reduction length of B (multiple of 64)
@@ -49,7 +64,28 @@ struct GemmArgs {
   int weights_once;       // 1: each B tile is read by one work item (hint evict_first)
   int kparts;             // K partitions per output tile (kEpiLogits; 1 otherwise)
   long long part_stride;  // elements between the partial outputs of two partitions
+  int pdl;                // kPdlStart / kPdlAfterWait / kPdlTail
 };
+
+__device__ __forceinline__ void pdl_enter(int mode) {
+  if (mode == kPdlStart) {
+    pdl_trigger();
+    pdl_wait();
+  } else if (mode == kPdlAfterWait) {
+    pdl_wait();
+    pdl_trigger();
+  } else {
+    pdl_trigger();
+  }
+}
+
+__device__ __forceinline__ void pdl_leave(int mode) {
+  if (mode == kPdlTail) pdl_wait();
+}
+
+// Work-list entries another kernel wrote; read through L2 (not L1) so a
+// kernel that starts without waiting never sees a stale line.
+__device__ __forceinline__ int tile_ld(const int* p) { return __ldcg(p); }
 
 template <int BN, int EPI>
 struct GemmCfg {
@@ -134,17 +170,17 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();  // the work lists and operands come from the previous kernels
+  pdl_enter(args.pdl);  // the work lists and operands come from earlier kernels
 
-  const bool dense = args.tiles == nullptr;
-  const int num_mtiles = dense ? (args.dense_rows + kGemmBM - 1) / kGemmBM : args.tiles[0];
+  const bool dense = args.tile_count == nullptr;
+  const int num_mtiles =
+      dense ? (args.dense_rows + kGemmBM - 1) / kGemmBM : tile_ld(args.tile_count);
   const int n_tiles = args.n_tiles * args.kparts;  // output tiles x K partitions
   const int ntn = args.n_tiles;
   const int total = num_mtiles * n_tiles;
   const int nk = args.K / kGemmBK;
   const int kpp = nk / args.kparts;  // K blocks per partition
-  const int* tl = dense ? nullptr : args.tiles + 4 + 3 * args.E;  // row tiles follow the expert entries
+  const int* tl = args.tile_rows;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -163,8 +199,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
         int mt, nt;
         raster(w, n_tiles, num_mtiles, mt, nt);
         const int part = nt / ntn, ntile = nt - part * ntn;
-        const int row0 = dense ? mt * kGemmBM : tl[3 * mt + 0];
-        const int e = dense ? 0 : tl[3 * mt + 2];
+        const int row0 = dense ? mt * kGemmBM : tile_ld(tl + 3 * mt + 0);
+        const int e = dense ? 0 : tile_ld(tl + 3 * mt + 2);
         const int brow = e * args.b_rows_per_expert + ntile * (SWIGLU ? BN / 2 : BN);
         const int kb0 = part * kpp;
         int ka = kb0 % args.a_kblocks;
@@ -249,8 +285,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
       int mt, nt_all;
       raster(w, n_tiles, num_mtiles, mt, nt_all);
       const int part = nt_all / ntn, nt = nt_all - part * ntn;
-      const int row0 = dense ? mt * kGemmBM : tl[3 * mt + 0];
-      const int rowend = dense ? args.dense_rows : tl[3 * mt + 1];
+      const int row0 = dense ? mt * kGemmBM : tile_ld(tl + 3 * mt + 0);
+      const int rowend = dense ? args.dense_rows : tile_ld(tl + 3 * mt + 1);
       const int ab = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       const bool got = mbar_wait_bounded(&tfull[ab], aph, abort_flag);
@@ -332,6 +368,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   tc_fence_after();
   if (threadIdx.x == 0 && *abort_flag) record_error(args.err, MOE_ERR_TIMEOUT, 10);
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  pdl_leave(args.pdl);
 }
 
 // ============================================================== large-batch kernel, CTA pairs
@@ -471,14 +508,13 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
   cluster_sync_all();  // the peer signals the leader's barriers only after both are set up
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();  // the work lists and operands come from the previous kernels
+  pdl_enter(args.pdl);  // the work lists and operands come from earlier kernels
 
-  const int num_pairs = args.tiles[0] / 2;
+  const int num_pairs = tile_ld(args.tile_count) / 2;
   const int n_tiles = args.n_tiles;
   const int total = num_pairs * n_tiles;
   const int nk = args.K / kGemmBK;
-  const int* tl = args.tiles + 4 + 3 * args.E;  // row tiles follow the expert entries
+  const int* tl = args.tile_rows;
   const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
 
   if (warp == 0) {
@@ -494,8 +530,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
       for (int w = cluster_id; w < total && ok; w += num_clusters) {
         int mp, nt;
         raster(w, n_tiles, num_pairs, mp, nt);
-        const int row0 = tl[3 * (2 * mp) + 0];
-        const int e = tl[3 * (2 * mp) + 2];
+        const int row0 = tile_ld(tl + 3 * (2 * mp) + 0);
+        const int e = tile_ld(tl + 3 * (2 * mp) + 2);
         const int a_row = row0 + (int)rank * 128;
         const int b_row = SWIGLU ? e * args.b_rows_per_expert + nt * 128 + (int)rank * args.up_offset
                                  : e * args.b_rows_per_expert + nt * BN + (int)rank * 128;
@@ -576,8 +612,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
     for (int w = cluster_id; w < total; w += num_clusters, ++it) {
       int mp, nt;
       raster(w, n_tiles, num_pairs, mp, nt);
-      const int row0 = tl[3 * (2 * mp) + 0];
-      const int rowend = tl[3 * (2 * mp) + 1];
+      const int row0 = tile_ld(tl + 3 * (2 * mp) + 0);
+      const int rowend = tile_ld(tl + 3 * (2 * mp) + 1);
       const int ab = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       const bool got = mbar_wait_bounded(&tfull[ab], aph, abort_flag);
@@ -1100,15 +1136,32 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
     return MOE_ERR_CUDA;
   const int nt1 = (int)((s.f + bn / 2 - 1) / (bn / 2));
   const int nt2 = (int)((s.d + bn - 1) / bn);
-  GemmArgs g1{tiles, s.E, 0, nt1, s.d, s.d / kGemmBK, 2 * s.f, s.f, s.f, h, s.f, nullptr, err, 0, 1, 0};
-  GemmArgs g2{tiles, s.E, 0, nt2, s.f, s.f / kGemmBK, s.d, 0, s.d, z, s.d, nullptr, err, 0, 1, 0};
+  const int* count = tiles;                          // row tiles
+  const int* rows = row_tile_entries(const_cast<int*>(tiles), s.E);
+  GemmArgs g1{count, rows, s.E, 0, nt1, s.d, s.d / kGemmBK, 2 * s.f, s.f, s.f, h, s.f, nullptr,
+              err, 0, 1, 0, kPdlStart};
+  GemmArgs g2{count, rows, s.E, 0, nt2, s.f, s.f / kGemmBK, s.d, 0, s.d, z, s.d, nullptr,
+              err, 0, 1, 0, kPdlStart};
   cudaError_t e;
   if (pairs) {
+    // Pairs first; each expert's odd last tile runs in a single-CTA kernel
+    // that starts on the SMs the pair kernel's tail frees (kPdlTail).
+    CUtensorMap tB2w;  // 256-row boxes for the single-CTA GEMM2
+    if (!make_tmap(&tB2w, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, 256)) return MOE_ERR_CUDA;
+    const int* lcount = tiles + 2;
+    const int* lrows = leftover_entries(const_cast<int*>(tiles), s.E);
+    GemmArgs l1 = g1, l2 = g2;
+    l1.tile_count = l2.tile_count = lcount;
+    l1.tile_rows = l2.tile_rows = lrows;
+    l1.pdl = l2.pdl = kPdlTail;
+    g1.pdl = g2.pdl = kPdlAfterWait;
     const int max_pairs = (L.max_mtiles + 1) / 2;
     e = launch_gemm_2sm<kEpiSwiGLU>(tA1, tB1, g1, max_pairs * nt1, num_sms, st);
+    if (e == cudaSuccess) e = launch_gemm_t<256, kEpiSwiGLU>(tA1, tB1, l1, s.E * nt1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_gemm_2sm<kEpiStore>(tA2, tB2, g2, max_pairs * nt2, num_sms, st);
+    if (e == cudaSuccess) e = launch_gemm_t<256, kEpiStore>(tA2, tB2w, l2, s.E * nt2, num_sms, st);
   } else if (wide) {
     e = launch_gemm_t<256, kEpiSwiGLU>(tA1, tB1, g1, L.max_mtiles * nt1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
@@ -1190,8 +1243,8 @@ cudaError_t launch_router_tc(const __nv_bfloat16* x, const float* w_g, const flo
   // Each partition writes its own fp32 plane; k_router_finish adds them in
   // partition order and adds the bias.
   // P == 1: the GEMM writes the logits (with the bias) directly.
-  GemmArgs a{nullptr, 0, s.T, nt, 3 * s.d, s.d / kGemmBK, 0, 0, s.E, P == 1 ? logits : part,
-             s.E, P == 1 ? bias : nullptr, err, 0, P, n};
+  GemmArgs a{nullptr, nullptr, 0, s.T, nt, 3 * s.d, s.d / kGemmBK, 0, 0, s.E,
+             P == 1 ? logits : part, s.E, P == 1 ? bias : nullptr, err, 0, P, n, kPdlStart};
   const int work = ((s.T + kGemmBM - 1) / kGemmBM) * nt * P;
   e = (bn == 128) ? launch_gemm_t<128, kEpiLogits>(tA, tB, a, work, num_sms, st)
                   : launch_gemm_t<256, kEpiLogits>(tA, tB, a, work, num_sms, st);

@@ -262,51 +262,76 @@ __device__ __forceinline__ void sort_candidates(uint32_t* k, int* i) {
 // the largest key, one for the lowest index holding it -- and the winning lane
 // drops its head.  A lane's head is its best candidate and, among equal keys,
 // its lowest index, so the round picks the same expert as the rank order.
-template <int VPL>
-__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k, int lane,
-                                          int* __restrict__ idx_row, float* __restrict__ w_row) {
-  if (VPL > 8) {
-    warp_topk_scan<VPL>(row, E, k, lane, idx_row, w_row);
-    return;
-  }
-  constexpr int V = VPL > 8 ? 8 : VPL;
-  uint32_t key[V];
-  int slot[V];
+template <int V>
+__device__ __forceinline__ void topk_load(const float* __restrict__ row, int E, int lane,
+                                          uint32_t* key, int* slot) {
 #pragma unroll
   for (int i = 0; i < V; ++i) {
     const int e = lane + 32 * i;
     key[i] = (e < E) ? order_key(row[e]) : 0u;  // 0: below every finite key
     slot[i] = i;
   }
-  sort_candidates<V>(key, slot);
-  uint32_t my_key = 0;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    const uint32_t wk = __reduce_max_sync(0xffffffffu, key[0]);
-    const uint32_t cand = (key[0] == wk) ? (uint32_t)(lane + 32 * slot[0]) : 0xffffffffu;
-    const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
-    if ((int)(we & 31) == lane) {
+}
+
+// One selection round: the winner's key and expert, and the winning lane
+// drops its head.
+template <int V>
+__device__ __forceinline__ void topk_round(uint32_t* key, int* slot, int lane, uint32_t& wk,
+                                           uint32_t& we) {
+  wk = __reduce_max_sync(0xffffffffu, key[0]);
+  const uint32_t cand = (key[0] == wk) ? (uint32_t)(lane + 32 * slot[0]) : 0xffffffffu;
+  we = __reduce_min_sync(0xffffffffu, cand);
+  if ((int)(we & 31) == lane) {
 #pragma unroll
-      for (int i = 0; i + 1 < V; ++i) {
-        key[i] = key[i + 1];
-        slot[i] = slot[i + 1];
-      }
-      key[V - 1] = 0u;
+    for (int i = 0; i + 1 < V; ++i) {
+      key[i] = key[i + 1];
+      slot[i] = slot[i + 1];
     }
-    if (lane == j) {
-      my_key = wk;
-      my_e = (int)we;
-    }
+    key[V - 1] = 0u;
   }
+}
+
+// Gate of slot `lane` (< k): softmax over the k selected logits.
+__device__ __forceinline__ float topk_gate(uint32_t my_key, int k, int lane) {
   const float my_v = key_value(my_key);
   const float top = __shfl_sync(0xffffffffu, my_v, 0);
   const float ex = (lane < k) ? expf(my_v - top) : 0.f;
   float sum = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  return ex / sum;
+}
+
+// idx_s_row (optional): a shared-memory copy of the selected ids.
+template <int VPL>
+__device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k, int lane,
+                                          int* __restrict__ idx_row, float* __restrict__ w_row,
+                                          int* idx_s_row = nullptr) {
+  if (VPL > 8) {
+    warp_topk_scan<VPL>(row, E, k, lane, idx_row, w_row);
+    if (idx_s_row && lane < k) idx_s_row[lane] = idx_row[lane];  // this lane's own store
+    return;
+  }
+  constexpr int V = VPL > 8 ? 8 : VPL;
+  uint32_t key[V];
+  int slot[V];
+  topk_load<V>(row, E, lane, key, slot);
+  sort_candidates<V>(key, slot);
+  uint32_t my_key = 0;
+  int my_e = 0;
+  for (int j = 0; j < k; ++j) {
+    uint32_t wk, we;
+    topk_round<V>(key, slot, lane, wk, we);
+    if (lane == j) {
+      my_key = wk;
+      my_e = (int)we;
+    }
+  }
+  const float g = topk_gate(my_key, k, lane);
   if (lane < k) {
     idx_row[lane] = my_e;
-    w_row[lane] = ex / sum;
+    w_row[lane] = g;
+    if (idx_s_row) idx_s_row[lane] = my_e;
   }
 }
 
@@ -390,15 +415,17 @@ __device__ int block_exclusive_scan_1024(int v, int* scratch /*[32]*/, int* tota
 
 // The expert GEMMs' work lists (layout in tile_list_ints): every thread of a
 // 1024-thread block calls this; thread e < E passes expert e's row count c
-// and first row off.
+// and first row off.  pair: tile pairs for CTA-pair GEMMs (see
+// pair_row_tiles).
 __device__ void write_work_lists(int e, int E, int c, int off, int* tiles, int* scratch,
                                  int* total, bool pair) {
-  int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
-  if (pair) nt = (nt + 1) & ~1;  // 256-row tiles of CTA pairs never straddle experts
-  const int tb = block_exclusive_scan_1024(nt, scratch, total);
+  const int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
+  const int nrow = pair ? pair_row_tiles(nt) : nt;  // tiles in the row-tile list
+  const int left = (pair && nt == 1) ? 1 : 0;       // a lone tile: leftover list
+  const int tb = block_exclusive_scan_1024(nrow, scratch, total);
   if (threadIdx.x == 0) tiles[0] = *total;
   int* rt = row_tile_entries(tiles, E);
-  for (int i = 0; i < nt; ++i) {
+  for (int i = 0; i < nrow; ++i) {
     rt[3 * (tb + i) + 0] = off + i * kGemmBM;
     rt[3 * (tb + i) + 1] = off + c;
     rt[3 * (tb + i) + 2] = e;
@@ -411,6 +438,14 @@ __device__ void write_work_lists(int e, int E, int c, int off, int* tiles, int* 
     et[3 * eb + 0] = off;
     et[3 * eb + 1] = off + c;
     et[3 * eb + 2] = e;
+  }
+  const int lb = block_exclusive_scan_1024(left, scratch, total);
+  if (threadIdx.x == 0) tiles[2] = *total;
+  if (left) {
+    int* lt = leftover_entries(tiles, E);
+    lt[3 * lb + 0] = off;
+    lt[3 * lb + 1] = off + c;
+    lt[3 * lb + 2] = e;
   }
 }
 
@@ -487,43 +522,48 @@ __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
 // thread).  Same results as k_topk + k_hist + k_scan + k_scatter.
 constexpr int kFusedSmemIdx = 8192;  // T*k up to this keeps the ids in shared memory
 
-// Exclusive block scan of three ints over 1024 threads (two barriers).
-__device__ __forceinline__ int3 block_exclusive_scan3_1024(int3 v, int3* warp_tot, int3* total) {
+// Exclusive block scan of four ints over 1024 threads (two barriers).
+__device__ __forceinline__ int4 block_exclusive_scan4_1024(int4 v, int4* warp_tot, int4* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int3 inc = v;
+  int4 inc = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int a = __shfl_up_sync(0xffffffffu, inc.x, off);
     const int b = __shfl_up_sync(0xffffffffu, inc.y, off);
     const int c = __shfl_up_sync(0xffffffffu, inc.z, off);
+    const int d = __shfl_up_sync(0xffffffffu, inc.w, off);
     if (lane >= off) {
       inc.x += a;
       inc.y += b;
       inc.z += c;
+      inc.w += d;
     }
   }
   if (lane == 31) warp_tot[wid] = inc;
   __syncthreads();
   if (wid == 0) {
-    const int3 t = warp_tot[lane];
-    int3 si = t;
+    const int4 t = warp_tot[lane];
+    int4 si = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int a = __shfl_up_sync(0xffffffffu, si.x, off);
       const int b = __shfl_up_sync(0xffffffffu, si.y, off);
       const int c = __shfl_up_sync(0xffffffffu, si.z, off);
+      const int d = __shfl_up_sync(0xffffffffu, si.w, off);
       if (lane >= off) {
         si.x += a;
         si.y += b;
         si.z += c;
+        si.w += d;
       }
     }
-    warp_tot[lane] = make_int3(si.x - t.x, si.y - t.y, si.z - t.z);
+    warp_tot[lane] = make_int4(si.x - t.x, si.y - t.y, si.z - t.z, si.w - t.w);
     if (lane == 31) *total = si;
   }
   __syncthreads();
-  const int3 base = warp_tot[wid];
-  return make_int3(base.x + inc.x - v.x, base.y + inc.y - v.y, base.z + inc.z - v.z);
+  const int4 base = warp_tot[wid];
+  return make_int4(base.x + inc.x - v.x, base.y + inc.y - v.y, base.z + inc.z - v.z,
+                   base.w + inc.w - v.w);
 }
 
 template <int VPL>
@@ -542,18 +582,14 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   const int RR = R > 1 ? R * R : 0;
   uint32_t* masks = reinterpret_cast<uint32_t*>(send + RR);  // [32][E]
   int* idx_s = reinterpret_cast<int*>(masks + 32 * E);         // [T*k] when it fits
-  __shared__ int3 warp_tot[32];
-  __shared__ int3 total;
+  __shared__ int4 warp_tot[32];
+  __shared__ int4 total;
   const bool ids_in_smem = T * k <= kFusedSmemIdx;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 2 * E + RR + 32 * E; i += 1024) sm[i] = 0;
-  for (int t = wid; t < T; t += 32) {
-    warp_topk<VPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, w + (size_t)t * k);
-    if (ids_in_smem && lane < k) {
-      // warp_topk left slot `lane` of token t in global memory; keep a copy
-      idx_s[t * k + lane] = idx[(size_t)t * k + lane];
-    }
-  }
+  for (int t = wid; t < T; t += 32)
+    warp_topk<VPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, w + (size_t)t * k,
+                   ids_in_smem ? idx_s + t * k : nullptr);
   __syncthreads();
   const int* ids = ids_in_smem ? idx_s : idx;
   const int t = threadIdx.x;
@@ -579,16 +615,19 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   __syncthreads();
   const int e = threadIdx.x;
   const int c = (e < E) ? hist[e] : 0;
-  int nt = (c + kGemmBM - 1) / kGemmBM;
-  if (pair) nt = (nt + 1) & ~1;  // pairs of 128-row tiles for the 2-SM GEMM
-  const int3 pre = block_exclusive_scan3_1024(make_int3(c, nt, c > 0 ? 1 : 0), warp_tot, &total);
-  const int3 tot = total;
+  const int nt = (c + kGemmBM - 1) / kGemmBM;
+  // CTA-pair GEMMs: pairs of row tiles; a lone tile goes to the leftover list
+  const int nrow = pair ? pair_row_tiles(nt) : nt;
+  const int left = (pair && nt == 1) ? 1 : 0;
+  const int4 pre =
+      block_exclusive_scan4_1024(make_int4(c, nrow, c > 0 ? 1 : 0, left), warp_tot, &total);
+  const int4 tot = total;
   if (e < E) {
     counts[e] = c;
     offsets[e] = pre.x;
     off_s[e] = pre.x;
     int* rt = row_tile_entries(tiles, E);
-    for (int i = 0; i < nt; ++i) {
+    for (int i = 0; i < nrow; ++i) {
       rt[3 * (pre.y + i) + 0] = pre.x + i * kGemmBM;
       rt[3 * (pre.y + i) + 1] = pre.x + c;
       rt[3 * (pre.y + i) + 2] = e;
@@ -599,11 +638,18 @@ __global__ void __launch_bounds__(1024) k_route_fused(
       et[3 * pre.z + 1] = pre.x + c;
       et[3 * pre.z + 2] = e;
     }
+    if (left) {
+      int* lt = leftover_entries(tiles, E);
+      lt[3 * pre.w + 0] = pre.x;
+      lt[3 * pre.w + 1] = pre.x + c;
+      lt[3 * pre.w + 2] = e;
+    }
   }
   if (threadIdx.x == 0) {
     offsets[E] = tot.x;
     tiles[0] = tot.y;
     tiles[1] = tot.z;
+    tiles[2] = tot.w;
   }
   if (R > 1)
     for (int i = threadIdx.x; i < RR; i += 1024) send_out[i] = send[i];
@@ -685,62 +731,80 @@ __global__ void __launch_bounds__(256) k_gather_rows(
 
 // ============================================================== combine
 // y[t] = sum_j w[t,j] * z[row_of[t,j]] in fp32, slot order.  One warp per
-// (token, 256-column chunk): each lane owns 8 columns (one 16-byte vector).
-// A row index outside [0, T*k) contributes nothing (never dereferenced).
+// (token, 256*V-column chunk): each lane owns V 16-byte vectors (8 columns
+// each, 256 columns apart), so a warp reads V*512 contiguous bytes of each of
+// the token's k rows with all k*V loads in flight.  A row index outside
+// [0, T*k) contributes nothing (never dereferenced).
+template <int V>
 __global__ void __launch_bounds__(256) k_combine(
     const __nv_bfloat16* __restrict__ z, const int* __restrict__ row_of,
     const float* __restrict__ w, int T, int d, int k, __nv_bfloat16* __restrict__ y) {
   pdl_trigger();
   pdl_wait();
   const long long P = (long long)T * k;
-  const int nchunk = (d + 255) / 256;
+  const int span = 256 * V;
+  const int nchunk = (d + span - 1) / span;
   const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (gw >= (long long)T * nchunk) return;
   const int lane = threadIdx.x & 31;
   const int t = (int)(gw / nchunk);
-  const int col = (int)(gw - (long long)t * nchunk) * 256 + lane * 8;
+  const int col0 = (int)(gw - (long long)t * nchunk) * span + lane * 8;
   // lane j < k holds slot j's row and gate; broadcast them with shuffles so
-  // the k row loads below are all independent.
+  // the row loads below are all independent.
   int my_r = -1;
   float my_w = 0.f;
   if (lane < k) {
     my_r = __ldg(row_of + (size_t)t * k + lane);
     my_w = __ldg(w + (size_t)t * k + lane);
   }
-  float acc[8];
+  float acc[V][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int v = 0; v < V; ++v)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[v][i] = 0.f;
   for (int j0 = 0; j0 < k; j0 += 8) {
-    uint4 v[8];
+    uint4 val[8][V];
     float wj[8];
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       const int r = __shfl_sync(0xffffffffu, my_r, (j0 + jj) & 31);
       wj[jj] = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
-      const bool ok = (j0 + jj < k) && r >= 0 && r < P && col < d;
-      v[jj] = ok ? __ldg(reinterpret_cast<const uint4*>(z + (size_t)r * d + col))
-                 : make_uint4(0, 0, 0, 0);
+      const bool ok = (j0 + jj < k) && r >= 0 && r < P;
       if (!ok) wj[jj] = 0.f;
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int col = col0 + 256 * v;
+        val[jj][v] = (ok && col < d)
+                         ? __ldcs(reinterpret_cast<const uint4*>(z + (size_t)r * d + col))
+                         : make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       if (j0 + jj >= k) break;
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[jj]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f2 = __bfloat1622float2(p[i]);
-        acc[2 * i] = fmaf(wj[jj], f2.x, acc[2 * i]);
-        acc[2 * i + 1] = fmaf(wj[jj], f2.y, acc[2 * i + 1]);
+      for (int v = 0; v < V; ++v) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&val[jj][v]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f2 = __bfloat1622float2(p[i]);
+          acc[v][2 * i] = fmaf(wj[jj], f2.x, acc[v][2 * i]);
+          acc[v][2 * i + 1] = fmaf(wj[jj], f2.y, acc[v][2 * i + 1]);
+        }
       }
     }
   }
-  if (col >= d) return;
-  uint4 o;
-  o.x = pack_bf16x2(acc[0], acc[1]);
-  o.y = pack_bf16x2(acc[2], acc[3]);
-  o.z = pack_bf16x2(acc[4], acc[5]);
-  o.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(y + (size_t)t * d + col) = o;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const int col = col0 + 256 * v;
+    if (col >= d) continue;
+    uint4 o;
+    o.x = pack_bf16x2(acc[v][0], acc[v][1]);
+    o.y = pack_bf16x2(acc[v][2], acc[v][3]);
+    o.z = pack_bf16x2(acc[v][4], acc[v][5]);
+    o.w = pack_bf16x2(acc[v][6], acc[v][7]);
+    *reinterpret_cast<uint4*>(y + (size_t)t * d + col) = o;
+  }
 }
 
 // ============================================================== self-test
@@ -904,9 +968,16 @@ cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, 
 
 cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const float* w,
                            const moe_shape& s, __nv_bfloat16* y, cudaStream_t st) {
-  const long long warps = (long long)s.T * ((s.d + 255) / 256);
+  // Large batches: 512 columns per warp (1 KB of each row per request
+  // stream); small ones keep 256 so more warps share the latency.
+  const bool wide = (long long)s.T * s.d >= (1LL << 22) && s.d % 512 == 0;
+  const int span = wide ? 512 : 256;
+  const long long warps = (long long)s.T * ((s.d + span - 1) / span);
   const unsigned blocks = (unsigned)((warps + 7) / 8);
-  return launch_kernel(k_combine, dim3(blocks), dim3(256), 0, st, 1, z, row_of, w, s.T, s.d,
+  if (wide)
+    return launch_kernel(k_combine<2>, dim3(blocks), dim3(256), 0, st, 1, z, row_of, w, s.T,
+                         s.d, s.k, y);
+  return launch_kernel(k_combine<1>, dim3(blocks), dim3(256), 0, st, 1, z, row_of, w, s.T, s.d,
                        s.k, y);
 }
 

@@ -198,7 +198,9 @@ def test_empty_batch_dispatch_zeroes_tables():
 
 
 # ---------------------------------------------------------------- combine
-@pytest.mark.parametrize("T,d,E,k", [(64, 256, 8, 2), (333, 2048, 128, 8), (1, 7168, 256, 8)])
+@pytest.mark.parametrize("T,d,E,k", [(64, 256, 8, 2), (333, 2048, 128, 8), (1, 7168, 256, 8),
+                                     # large batches: 512 columns per warp, and d off that grid
+                                     (2049, 2048, 64, 4), (2000, 2304, 32, 3)])
 def test_combine_matches_oracle(T, d, E, k):
     L = wl.make_logits(T, E, device="cpu", seed=5 + T)
     idx = oracle.topk_select_sorted(L.numpy(), k)
