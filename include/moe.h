@@ -82,8 +82,11 @@ MOE_API int moe_version(void);
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
  * need for shape *s (enough for all three).  Returns 0 if *s is invalid.
  * The workspace must be 256-byte aligned.  Its first 64 bytes hold the
- * device error word: zero them once before the first call (moe_check clears
- * them after reporting an error); the rest needs no initialisation. */
+ * device error word and a block counter of moe_forward's routing kernel:
+ * zero them once before the first call (every call leaves the counter at
+ * zero again; moe_check clears the error word after reporting an error); the
+ * rest needs no initialisation.  Calls sharing one workspace must not run
+ * concurrently. */
 MOE_API size_t moe_workspace_size(const moe_shape* s);
 
 /* Router gate ("What is an MoE layer?": the gate scores each token).

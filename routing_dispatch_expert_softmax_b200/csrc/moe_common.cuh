@@ -56,8 +56,10 @@ inline int router_tc_parts(const moe_shape& s) {
   return best;
 }
 
-// Device error word: ws[0] = first error code, ws[1] = detail (kernel id).
-enum : int { kErrSlot = 0, kErrDetail = 1 };
+// Workspace header (the 64 bytes the caller zeroes once): ws[0] = first error
+// code, ws[1] = detail (kernel id), ws[2] = the fused routing kernel's block
+// ticket (back to 0 at the end of every call).
+enum : int { kErrSlot = 0, kErrDetail = 1, kRouteTicket = 2 };
 
 // Every bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

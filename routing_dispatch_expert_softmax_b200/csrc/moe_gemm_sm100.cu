@@ -1218,8 +1218,36 @@ __global__ void __launch_bounds__(256) k_router_finish(const float* __restrict__
                                                        float* __restrict__ logits) {
   pdl_trigger();
   pdl_wait();
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long i0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const bool vec = (E & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0 &&
+                   (!bias || (reinterpret_cast<uintptr_t>(bias) & 15) == 0);
+  if (vec) {
+    // 4 logits per thread step; every partial plane's load in flight at once
+    // (P <= 84: the partitions hold at least 4 of the 3d/64 <= 768 K blocks).
+    const long long n4 = n / 4;
+    const float4* p4 = reinterpret_cast<const float4*>(part);
+    for (long long i = i0; i < n4; i += stride) {
+      float4 v = __ldcs(p4 + i);
+      for (int p = 1; p < P; ++p) {
+        const float4 u = __ldcs(p4 + (size_t)p * n4 + i);
+        v.x += u.x;
+        v.y += u.y;
+        v.z += u.z;
+        v.w += u.w;
+      }
+      if (bias) {
+        const float4 b = __ldg(reinterpret_cast<const float4*>(bias) + (i % (E / 4)));
+        v.x += b.x;
+        v.y += b.y;
+        v.z += b.z;
+        v.w += b.w;
+      }
+      reinterpret_cast<float4*>(logits)[i] = v;
+    }
+    return;
+  }
+  for (long long i = i0; i < n; i += stride) {
     float v = part[i];
     for (int p = 1; p < P; ++p) v += part[(size_t)p * n + i];
     logits[i] = bias ? v + bias[i % E] : v;

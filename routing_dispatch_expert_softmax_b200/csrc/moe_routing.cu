@@ -515,12 +515,17 @@ __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
 }
 
 // ============================================================== fused routing, T <= 1024
-// One block of 1024 threads does selection and the whole dispatch table for a
-// batch of at most 1024 tokens: top-k (warp w takes tokens w, w+32, ...),
-// histogram, one block scan of (rows, 128-row tiles, touched) per expert,
-// work lists, virtual-EP counts and the stable scatter (one token per
-// thread).  Same results as k_topk + k_hist + k_scan + k_scatter.
+// Selection and the whole dispatch table for a batch of at most 1024 tokens
+// in one launch.  Blocks of 1024 threads each select kFusedSelTokens tokens
+// (one warp per token: selection throughput is bounded per SM, so the tokens
+// are spread over ceil(T / kFusedSelTokens) SMs); the last block to take a
+// ticket (a counter in the workspace's zeroed header, reset by that block)
+// then builds the tables: histogram, one block scan of (rows, row tiles,
+// touched, leftover) per expert, work lists, virtual-EP counts and the
+// stable scatter (one token per thread).  Same results as k_topk + k_hist +
+// k_scan + k_scatter.
 constexpr int kFusedSmemIdx = 8192;  // T*k up to this keeps the ids in shared memory
+constexpr int kFusedSelTokens = 8;   // tokens selected per block
 
 // Exclusive block scan of four ints over 1024 threads (two barriers).
 __device__ __forceinline__ int4 block_exclusive_scan4_1024(int4 v, int4* warp_tot, int4* total) {
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     int* __restrict__ idx, float* __restrict__ w, int* __restrict__ counts,
     int* __restrict__ offsets, int* __restrict__ tiles, int* __restrict__ send_out,
     int* __restrict__ rank_off, int* __restrict__ row_of, int* __restrict__ perm, int* err,
-    int pair) {
+    int* ticket, int pair) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int sm[];
@@ -584,13 +589,35 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   int* idx_s = reinterpret_cast<int*>(masks + 32 * E);         // [T*k] when it fits
   __shared__ int4 warp_tot[32];
   __shared__ int4 total;
+  __shared__ int is_last;
   const bool ids_in_smem = T * k <= kFusedSmemIdx;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const bool single = gridDim.x == 1;  // one block: no ticket, ids straight to smem
   for (int i = threadIdx.x; i < 2 * E + RR + 32 * E; i += 1024) sm[i] = 0;
-  for (int t = wid; t < T; t += 32)
-    warp_topk<VPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k, w + (size_t)t * k,
-                   ids_in_smem ? idx_s + t * k : nullptr);
+  // Selection: block b, warp w < kFusedSelTokens takes token b*kFusedSelTokens + w.
+  {
+    const int t = blockIdx.x * kFusedSelTokens + wid;
+    if (wid < kFusedSelTokens && t < T) {
+      warp_topk<VPL>(logits + (size_t)t * E, E, k, lane, idx + (size_t)t * k,
+                     w + (size_t)t * k, single && ids_in_smem ? idx_s + t * k : nullptr);
+      if (!single) __threadfence();  // this lane's ids and gates before the block's ticket
+    }
+  }
   __syncthreads();
+  if (!single) {
+    if (threadIdx.x == 0) {
+      __threadfence();
+      is_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!is_last) return;
+    // The last block to finish selection builds the tables for the whole batch.
+    __threadfence();
+    if (threadIdx.x == 0) *ticket = 0;  // ready for the next call
+    if (ids_in_smem)
+      for (int i = threadIdx.x; i < T * k; i += 1024) idx_s[i] = __ldcg(idx + i);
+    __syncthreads();
+  }
   const int* ids = ids_in_smem ? idx_s : idx;
   const int t = threadIdx.x;
   const bool valid = t < T;
@@ -599,7 +626,7 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     const int per = R > 1 ? E / R : 1;
     const int src = R > 1 ? t / src_chunk : 0;
     for (int j = 0; j < k; ++j) {
-      const int e = ids[t * k + j];
+      const int e = ids_in_smem ? ids[t * k + j] : __ldcg(ids + t * k + j);
       bool ok = (e >= 0 && e < E);
       for (int j2 = 0; j2 < j && ok; ++j2) ok = my_e[j2] != e;
       my_e[j] = ok ? e : -1;
@@ -726,7 +753,21 @@ __global__ void __launch_bounds__(256) k_gather_rows(
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
   uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
   const int nv = d / 8;
-  for (int c = lane; c < nv; c += 32) dst[c] = __ldg(src + c);
+  // Up to 8 vectors per lane in flight; x_perm is written with streaming
+  // stores so it does not push x (read k times) out of L2.
+  for (int c0 = 0; c0 < nv; c0 += 256) {
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = c0 + lane + 32 * i;
+      if (c < nv) v[i] = __ldg(src + c);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = c0 + lane + 32 * i;
+      if (c < nv) __stcs(dst + c, v[i]);
+    }
+  }
 }
 
 // ============================================================== combine
@@ -907,9 +948,10 @@ static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R,
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_kernel(k_route_fused<VPL>, dim3(1), dim3(1024), smem, st, 1, logits, s.T, s.E,
-                       s.k, R, chunk, idx, w, counts, offsets, tiles, send, rank_off, row_of,
-                       perm, err, pair_tiles(s) ? 1 : 0);
+  const unsigned blocks = (unsigned)((s.T + kFusedSelTokens - 1) / kFusedSelTokens);
+  return launch_kernel(k_route_fused<VPL>, dim3(blocks), dim3(1024), smem, st, 1, logits, s.T,
+                       s.E, s.k, R, chunk, idx, w, counts, offsets, tiles, send, rank_off, row_of,
+                       perm, err, err + kRouteTicket, pair_tiles(s) ? 1 : 0);
 }
 
 cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
