@@ -715,7 +715,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
 // epilogue pairs gate lane j with up lane 64 + j through shared memory.
 template <int NMAX, bool SWIGLU>
 struct SwapCfg {
-  static constexpr int kStages = NMAX <= 64 ? 8 : 4;
+  static constexpr int kStages = NMAX <= 64 ? 8 : NMAX <= 128 ? 6 : 4;
   static constexpr int kABytes = 128 * kGemmBK * 2;   // weights, 16 KB
   static constexpr int kBBytes = NMAX * kGemmBK * 2;  // tokens
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -738,10 +738,16 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Work items come from a list of (row0, row_end, expert) entries: the
+// touched-expert list (every item holds all of an expert's rows, at most
+// NMAX), or with row_tiles the 128-row tile list, whose entry i covers rows
+// [row0, min(row_end, row0 + 128)) so an expert with more than NMAX = 128
+// rows becomes several items.
 template <int NMAX, bool SWIGLU>
 __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-    const int* __restrict__ tiles, int n_tiles, int K, int w_rows_per_expert,
+    const int* __restrict__ list_count, const int* __restrict__ list, int row_tiles,
+    int n_tiles, int K, int w_rows_per_expert,
     int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
     int* __restrict__ err) {
   using C = SwapCfg<NMAX, SWIGLU>;
@@ -786,9 +792,14 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   const uint32_t tmem_base = *tmem_slot;
   pdl_trigger();
   pdl_wait();  // the work lists and operands come from the previous kernels
-  const int total = tiles[1] * n_tiles;
+  const int total = list_count[0] * n_tiles;
   const int nk = K / kGemmBK;
-  const int* et = tiles + 4;
+  const int* et = list;
+  // rows of item i (row_end is the expert's end; a row tile holds at most 128)
+  auto item_rows = [&](int i) {
+    const int r = et[3 * i + 1] - et[3 * i + 0];
+    return row_tiles ? min(r, kGemmBM) : r;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -804,7 +815,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
         const int row0 = et[3 * i + 0];
-        const int n = et[3 * i + 1] - row0;
+        const int n = item_rows(i);
         const int e = et[3 * i + 2];
         if (n < 1 || n > NMAX) continue;  // not a small-batch item (recorded by the epilogue)
         const int nb = (n + 15) >> 4;
@@ -851,7 +862,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
         const int i = w / n_tiles;
-        const int n = et[3 * i + 1] - et[3 * i + 0];
+        const int n = item_rows(i);
         if (n < 1 || n > NMAX) {
           --it;  // skipped items use no accumulator buffer (same in the epilogue)
           continue;
@@ -895,7 +906,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
       const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
       const int row0 = et[3 * i + 0];
-      const int n = et[3 * i + 1] - row0;
+      const int n = item_rows(i);
       if (n < 1 || n > NMAX) {
         if (threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
         --it;  // the MMA warp skipped it too: no accumulator was used
@@ -1024,7 +1035,8 @@ static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
 
 template <int NMAX, bool SWIGLU>
 static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
-                                 const int* tiles, int max_work, int n_tiles, int K,
+                                 const int* list_count, const int* list, int row_tiles,
+                                 int max_work, int n_tiles, int K,
                                  int w_rows, int up_off, int n_out, __nv_bfloat16* out,
                                  int ld_out, int* err, int num_sms, cudaStream_t st) {
   using C = SwapCfg<NMAX, SWIGLU>;
@@ -1039,7 +1051,8 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
   int grid = max_work < num_sms ? max_work : num_sms;
   if (grid < 1) grid = 1;
   return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU>, dim3(grid), dim3(192), C::kSmemBytes, st,
-                       1, tw, tx, tiles, n_tiles, K, w_rows, up_off, n_out, out, ld_out, err);
+                       1, tw, tx, list_count, list, row_tiles, n_tiles, K, w_rows, up_off,
+                       n_out, out, ld_out, err);
 }
 
 // Small batches (every expert has at most 256 rows): both GEMMs in swap-AB form.
@@ -1067,19 +1080,26 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
   const int E = s.E;
   cudaError_t e;
   if (s.T <= 64) {
-    e = launch_swap_t<64, true>(tW1, tX1, tiles, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h, s.f,
-                                err, num_sms, st);
+    // one item per touched expert (at most 64 rows)
+    const int* cnt = tiles + 1;
+    const int* ents = expert_entries(const_cast<int*>(tiles));
+    e = launch_swap_t<64, true>(tW1, tX1, cnt, ents, 0, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h,
+                                s.f, err, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
-      e = launch_swap_t<64, false>(tW2, tX2, tiles, E * nt2, nt2, s.f, s.d, 0, s.d, z, s.d,
-                                   err, num_sms, st);
+      e = launch_swap_t<64, false>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d, z,
+                                   s.d, err, num_sms, st);
   } else {
-    e = launch_swap_t<256, true>(tW1, tX1, tiles, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h,
-                                 s.f, err, num_sms, st);
+    // one item per 128-row tile: 6 K-stages of weights in flight instead of
+    // the 4 that 256-row items leave room for
+    const int* cnt = tiles;
+    const int* ents = row_tile_entries(const_cast<int*>(tiles), E);
+    e = launch_swap_t<128, true>(tW1, tX1, cnt, ents, 1, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
+                                 s.f, s.f, h, s.f, err, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
-      e = launch_swap_t<256, false>(tW2, tX2, tiles, E * nt2, nt2, s.f, s.d, 0, s.d, z, s.d,
-                                    err, num_sms, st);
+      e = launch_swap_t<128, false>(tW2, tX2, cnt, ents, 1, L.max_mtiles * nt2, nt2, s.f, s.d,
+                                    0, s.d, z, s.d, err, num_sms, st);
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
