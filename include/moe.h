@@ -148,8 +148,11 @@ MOE_API int moe_dispatch(const int32_t* idx, const moe_bf16* x, const moe_shape*
  *   w2     [E, d, f] bf16 in    Wd_e^T
  *   z      [T*k, d] bf16 out
  *   ws     workspace of moe_workspace_size(s) bytes
- * Runs on the tcgen05 tensor cores with TMA-fed operands.  Bad offsets are
- * recorded as MOE_ERR_DEVICE_CHECK.                                        */
+ * Runs on the tcgen05 tensor cores with TMA-fed operands: up to 256 tokens
+ * with the weights as the 128-row MMA operand and the expert's tokens as N;
+ * larger batches with 128-row token tiles, on 2-CTA clusters (256 x 256
+ * tiles) once experts average at least 128 rows.  Bad offsets are recorded
+ * as MOE_ERR_DEVICE_CHECK.                                                 */
 MOE_API int moe_ffn(const moe_bf16* x_perm, const int32_t* offsets,
             const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
             moe_bf16* z, void* ws, void* stream);

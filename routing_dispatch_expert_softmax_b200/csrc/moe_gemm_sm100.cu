@@ -89,12 +89,16 @@ __device__ __forceinline__ int tile_ld(const int* p) { return __ldcg(p); }
 
 template <int BN, int EPI>
 struct GemmCfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  // The router (logits) epilogue's staging tile costs a K-stage: kernels of
+  // a programmatic-launch chain measured slower above ~200 KB of shared memory.
+  static constexpr int kStages = EPI == kEpiLogits ? ((BN == 256) ? 3 : 5) : ((BN == 256) ? 4 : 6);
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
   static constexpr int kBBytes = BN * kGemmBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;  // double-buffered accumulator
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256;
+  // Logits epilogue: per epilogue warp 32 rows x 32 fp32 staged for full-line stores.
+  static constexpr int kOutStageBytes = EPI == kEpiLogits ? 4 * 32 * 128 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kOutStageBytes + 1024 /*align*/ + 256;
   static constexpr int kThreads = 192;
 };
 
@@ -136,7 +140,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint4* out_stage = reinterpret_cast<uint4*>(smem + S * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kOutStageBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -340,13 +345,47 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm(
         }
       } else {
         float* out = static_cast<float*>(args.out) + (size_t)part * args.part_stride;
+        // Rows of 16-byte-aligned fp32 vectors: stage each 32 x 32 slice in
+        // the warp's tile (16-byte chunks XOR-swizzled by row) and store 4
+        // whole 128-byte rows per instruction; otherwise one float at a time.
+        const bool vec = (args.ld_out & 3) == 0 && (args.part_stride & 3) == 0 &&
+                         (reinterpret_cast<uintptr_t>(args.out) & 15) == 0 &&
+                         (!args.bias || (reinterpret_cast<uintptr_t>(args.bias) & 15) == 0);
+        uint4* st_tile = out_stage + (size_t)(warp - 2) * 32 * 8;
+        const int row_base = row0 + q * 32;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t a[32];
           tmem_ld_32x32b_x32(t_addr + c, a);
           tmem_ld_wait();
           const int col = nt * BN + c;
-          if (row_ok && col < args.n_out) {
+          if (vec) {
+            if (col < args.n_out) {  // warp-uniform
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                st_tile[lane * 8 + (v ^ (lane & 7))] =
+                    make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
+              __syncwarp();
+              const int v = lane & 7, cv = col + 4 * v;
+              float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (args.bias && cv < args.n_out)
+                bv = __ldg(reinterpret_cast<const float4*>(args.bias + cv));
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int r = i * 4 + (lane >> 3);
+                const uint4 u = st_tile[r * 8 + (v ^ (r & 7))];
+                if (row_base + r < rowend && cv < args.n_out) {
+                  const float4 o = make_float4(__uint_as_float(u.x) + bv.x,
+                                               __uint_as_float(u.y) + bv.y,
+                                               __uint_as_float(u.z) + bv.z,
+                                               __uint_as_float(u.w) + bv.w);
+                  *reinterpret_cast<float4*>(out + (size_t)(row_base + r) * args.ld_out + cv) =
+                      o;
+                }
+              }
+              __syncwarp();
+            }
+          } else if (row_ok && col < args.n_out) {
             float* dst = out + (size_t)row * args.ld_out + col;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -445,7 +484,9 @@ __device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar, uint32_t cta) {
 
 template <int EPI>
 struct PairCfg {
-  static constexpr int kStages = 6;
+  // GEMM2's staging tile costs it a K-stage: at 214 KB of shared memory the
+  // pair GEMM2 measured 13 us slower than at 182 KB (same-box A/B, prefill).
+  static constexpr int kStages = EPI == kEpiStore ? 5 : 6;
   static constexpr int kABytes = 128 * kGemmBK * 2;  // this CTA's 128 activation rows
   static constexpr int kBBytes = 128 * kGemmBK * 2;  // this CTA's 128 weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;

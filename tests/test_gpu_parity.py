@@ -108,7 +108,11 @@ def test_topk_on_router_logits_of_model_shapes(cfg):
                                  wl.QWEN3_30B_A3B_DECODE.with_T(257),
                                  wl.QWEN3_30B_A3B_PREFILL.with_T(4096),
                                  wl.DEEPSEEK_V3_ROUTED.with_T(1000),
-                                 wl.MIXTRAL_8X7B.with_T(700)], ids=lambda c: c.name)
+                                 wl.MIXTRAL_8X7B.with_T(700),
+                                 # E not a multiple of 4: the tensor-core epilogue's scalar stores
+                                 wl.MoEConfig("router-odd-E", T=300, d=256, E=6, k=2, f=64,
+                                              zipf_s=1.0)],
+                         ids=lambda c: c.name)
 def test_router_within_fp32_error_bound(cfg):
     x = wl.make_hidden(cfg, "cpu", 0)
     w_g, bias = wl.make_router(cfg, "cpu", 0)
