@@ -621,19 +621,21 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   const int* ids = ids_in_smem ? idx_s : idx;
   const int t = threadIdx.x;
   const bool valid = t < T;
-  int my_e[kMaxK];
+  // The ids come from this kernel's own selection: distinct per token by
+  // construction, and in range unless a logit is a NaN whose bits sort below
+  // every candidate (an out-of-range pick is recorded and skipped).  Bit j of
+  // okmask marks slot j as usable.
+  uint32_t okmask = 0;
   if (valid) {
     const int per = R > 1 ? E / R : 1;
     const int src = R > 1 ? t / src_chunk : 0;
     for (int j = 0; j < k; ++j) {
       const int e = ids_in_smem ? ids[t * k + j] : __ldcg(ids + t * k + j);
-      bool ok = (e >= 0 && e < E);
-      for (int j2 = 0; j2 < j && ok; ++j2) ok = my_e[j2] != e;
-      my_e[j] = ok ? e : -1;
-      if (!ok) {
+      if (e < 0 || e >= E) {
         record_error(err, MOE_ERR_DEVICE_CHECK, 4);
         continue;
       }
+      okmask |= 1u << j;
       atomicAdd(&hist[e], 1);
       atomicOr(&masks[wid * E + e], 1u << lane);
       if (R > 1) atomicAdd(&send[src * R + e / per], 1);
@@ -686,8 +688,8 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   if (valid) {
     const uint32_t lt = (1u << lane) - 1u;
     for (int j = 0; j < k; ++j) {
-      const int ej = my_e[j];
-      if (ej < 0) continue;
+      if (!((okmask >> j) & 1u)) continue;
+      const int ej = ids_in_smem ? ids[t * k + j] : __ldcg(ids + t * k + j);
       int r = off_s[ej];
       for (int w2 = 0; w2 < wid; ++w2) r += __popc(masks[w2 * E + ej]);
       r += __popc(masks[wid * E + ej] & lt);

@@ -294,6 +294,38 @@ def test_ffn_ragged_rows_and_single_expert():
     _ffn_case(wl.MoEConfig("one-expert", T=129, d=128, E=1, k=1, f=128))
 
 
+@pytest.mark.parametrize("counts", [
+    # CTA-pair regime (T*k >= 128*E): lone-tile experts (<= 128 rows) go to the
+    # single-CTA list, odd tile counts (300 -> 3, 600 -> 5 tiles) to padded pairs,
+    # empty experts to nothing
+    [600, 100, 300, 50, 0, 50, 0, 1],
+    # every expert a lone tile but one, the first empty
+    [0, 128, 1, 127, 64, 8, 9, 1024 + 129],
+], ids=["mixed", "lone"])
+def test_ffn_pair_regime_tile_kinds(counts):
+    """moe_ffn on caller offsets chosen to hit each kind of work item of the
+    large-batch GEMMs, checked row by row against the oracle."""
+    counts = np.array(counts, dtype=np.int64)
+    E, P = counts.size, int(counts.sum())
+    cfg = wl.MoEConfig("tile-kinds", T=P, d=256, E=E, k=1, f=384)
+    x_perm = wl.make_hidden(cfg, DEV, 7)
+    w13, w2 = wl.make_experts(cfg, DEV, 7)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    shape = MoEShape.from_config(cfg)
+    ws = moe.workspace(shape)
+    z = torch.empty(P, cfg.d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn(x_perm, torch.from_numpy(offsets).to(DEV), w13, w2, z, shape, ws)
+    _check_clean(ws)
+    xp = np64(x_perm)
+    ref = np.zeros((P, cfg.d))
+    lazy13, lazy2 = LazyExperts(w13), LazyExperts(w2)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if b > a:
+            ref[a:b] = oracle.swiglu_ffn(xp[a:b], lazy13[e], lazy2[e])
+    assert_layer_close(z, ref, "moe_ffn tile kinds")
+
+
 def test_ffn_qwen_prefill_sampled():
     _ffn_case(wl.QWEN3_30B_A3B_PREFILL, sample_rows=_sample_rows())
 
