@@ -6,4 +6,8 @@ library and never receives a value computed by it.
 """
 
 from .moe_oracle import *  # noqa: F401,F403
-from .moe_oracle import __all__  # noqa: F401
+from .eplb_oracle import *  # noqa: F401,F403
+from . import eplb_oracle as _eplb
+from . import moe_oracle as _moe
+
+__all__ = list(_moe.__all__) + list(_eplb.__all__)

@@ -7,6 +7,8 @@ plausible bugs into the oracle (on the CPU) and confirm a pin catches each.
 """
 
 import itertools
+import json
+import os
 import math
 from fractions import Fraction
 
@@ -337,3 +339,77 @@ def test_planted_wrong_silu_sign_is_caught(monkeypatch, golden):
         z = np.asarray(z, np.float64)
         return z / (1.0 + np.exp(z))
     assert _pins_fail(monkeypatch, "silu", bad, golden) > 0
+
+
+# ---------------------------------------------------------------- EPLB-style balancing
+def _eplb_cases():
+    path = os.path.join(os.path.dirname(__file__), "golden", "eplb_worked_examples.json")
+    with open(path) as fh:
+        return json.load(fh)["cases"]
+
+
+@pytest.mark.parametrize("case", _eplb_cases(), ids=lambda c: str(c["load"]))
+def test_eplb_plan_matches_hand_worked_examples(case):
+    n = oracle.eplb_replicate(case["load"], case["n_redundant"])
+    assert n.tolist() == case["copies"]
+    p2l, off, phys = oracle.eplb_plan(case["load"], case["n_redundant"], case["R"])
+    assert p2l.tolist() == case["phys_to_logical"]
+    assert off.tolist() == case["rep_offsets"]
+    assert phys.tolist() == case["rep_phys"]
+    shares = {(e, i): s for e, i, s in oracle.eplb_shares(case["load"], n)}
+    S = len(p2l) // case["R"]
+    loads = [0] * case["R"]
+    for e in range(len(case["load"])):
+        for i in range(off[e + 1] - off[e]):
+            loads[phys[off[e] + i] // S] += shares[(e, i)]
+    assert loads == case["rank_loads"]
+
+
+def test_eplb_replication_minimises_the_largest_load_per_copy():
+    # brute force over every way to hand out the redundant copies
+    rng = np.random.default_rng(3)
+    for _ in range(40):
+        E = int(rng.integers(2, 5))
+        rd = int(rng.integers(0, 5))
+        load = rng.integers(0, 30, E).tolist()
+        n = oracle.eplb_replicate(load, rd)
+        best = min(max(l / c for l, c in zip(load, comp))
+                   for comp in itertools.product(range(1, rd + 2), repeat=E)
+                   if sum(comp) == E + rd)
+        assert max(l / c for l, c in zip(load, n)) == pytest.approx(best)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_eplb_plan_invariants(seed):
+    rng = np.random.default_rng(seed)
+    R = int(rng.choice([1, 2, 4, 8]))
+    E = R * int(rng.integers(1, 9))
+    rd = R * int(rng.integers(0, 3))
+    load = (1000 * rng.zipf(1.3, E).clip(max=50)).tolist()
+    p2l, off, phys = oracle.eplb_plan(load, rd, R)
+    n = np.diff(off)
+    assert n.sum() == E + rd and (n >= 1).all()
+    assert sorted(phys.tolist()) == list(range(E + rd))        # every slot used once
+    for e in range(E):
+        assert (p2l[phys[off[e]:off[e + 1]]] == e).all()      # replicas map back
+    assert sum(s for _, _, s in oracle.eplb_shares(load, n)) == sum(load)
+
+
+def test_eplb_remap_conserves_counts_and_uses_t_mod_copies():
+    rng = np.random.default_rng(7)
+    E, k, T, R, rd = 16, 4, 300, 4, 4
+    logits = rng.normal(size=(T, E)) - np.log(np.arange(1, E + 1))  # skewed popularity
+    idx = oracle.topk_select_sorted(logits.astype(np.float32), k)
+    counts = oracle.expert_counts(idx, E)
+    p2l, off, phys = oracle.eplb_plan(counts, rd, R)
+    idx_p = oracle.eplb_remap(idx, off, phys)
+    counts_p = oracle.expert_counts(idx_p, E + rd)
+    for e in range(E):
+        assert counts_p[phys[off[e]:off[e + 1]]].sum() == counts[e]
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            assert idx_p[t, j] == phys[off[e] + t % (off[e + 1] - off[e])]
+    # the balanced placement evens the per-rank rows out on this skewed batch
+    assert (oracle.rank_loads(counts_p, R).max() <
+            oracle.rank_loads(counts, R).max())
