@@ -44,13 +44,16 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ["routing_dispatch_expert_softmax_b200/csrc/moe_gemm_sm100.cu",
                   "routing_dispatch_expert_softmax_b200/csrc/moe_common.cuh"]
 
-def launches_per_forward(cfg):
-    """Kernels one moe_forward launches: router (one cluster kernel up to 256
-    tokens; above, the W_g split and the tensor-core GEMM, plus a partial-sum
-    kernel when the GEMM's K is split into P > 1 partial planes: P is the
-    largest divisor of the 3d/64 K blocks, at most a quarter of them, with
-    tiles * P <= 148), routing (one fused kernel for T <= 1024, else top-k +
-    histogram + scan + scatter), gather, the two expert GEMMs, combine."""
+def launches_per_forward(cfg, eplb_redundant=0):
+    """Kernels one moe_forward (moe_forward_eplb with eplb_redundant > 0)
+    launches: router (one cluster kernel up to 256 tokens; above, the W_g
+    split and the tensor-core GEMM, plus a partial-sum kernel when the GEMM's
+    K is split into P > 1 partial planes: P is the largest divisor of the
+    3d/64 K blocks, at most a quarter of them, with tiles * P <= 148),
+    routing (one fused kernel for T <= 1024, else top-k + histogram + scan +
+    scatter; with replicas top-k + remap + histogram + scan + scatter),
+    gather, the two expert GEMMs (each followed by the lone-tile kernel when
+    they run on CTA pairs), combine."""
     T = cfg.T
     if T <= 256:
         router = 1
@@ -67,7 +70,12 @@ def launches_per_forward(cfg):
             parts = p
         router = 2 if parts == 1 else 3
     routing = 1 if T <= 1024 else 4
-    return router + routing + 1 + 2 + 1
+    if eplb_redundant:
+        routing = 5
+    gemms = 2
+    if T > 256 and T * cfg.k >= 128 * (cfg.E + eplb_redundant):
+        gemms = 4
+    return router + routing + 1 + gemms + 1
 
 
 def parse_args(argv=None):
@@ -79,6 +87,9 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="qwen3-30b-a3b-decode")
     p.add_argument("--T", type=int, default=None, help="override the token count")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--eplb-redundant", type=int, default=0,
+                   help="time the layer with this many redundant expert copies placed by "
+                        "the EPLB-style plan (built from the counts of one warm-up call)")
     return p.parse_args(argv)
 
 
@@ -382,10 +393,31 @@ def run_ours(args):
     moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws)
     torch.cuda.synchronize(dev)
 
+    eplb_info = None
+    if args.eplb_redundant:
+        # Replicated experts: the plan comes from one call's counts (the load
+        # window), the layer then runs moe_forward_eplb.  The staged pass
+        # below still times the plain layer's stages.
+        counts0 = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+        moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, counts_out=counts0)
+        layer.rebalance(counts0.cpu().long(), args.eplb_redundant)
+        counts_p = torch.empty(layer.physical_experts, dtype=torch.int32, device=dev)
+        layer(x, out=y, counts_out=counts_p)
+        ws_e = layer.workspace(cfg.T)
+        R_e = max(cfg.R, 1)
+        cl = counts0.cpu().long().view(R_e, -1).sum(1)
+        cp = counts_p.cpu().long().view(R_e, -1).sum(1)
+        eplb_info = {"redundant": args.eplb_redundant, "physical_experts": layer.physical_experts,
+                     "ranks": R_e, "rank_rows_plain": cl.tolist(), "rank_rows_eplb": cp.tolist(),
+                     "imbalance_plain": float(cl.max() / cl.float().mean()),
+                     "imbalance_eplb": float(cp.max() / cp.float().mean())}
+
     def capture(events=None):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            if events is None:
+            if events is None and eplb_info is not None:
+                layer(x, out=y)
+            elif events is None:
                 moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws)
             else:
                 moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, events)
@@ -397,6 +429,8 @@ def run_ours(args):
         plain.replay()
     torch.cuda.synchronize(dev)
     st = moe.moe_check(ws)
+    if st == moe.MOE_OK and eplb_info is not None:
+        st = moe.moe_check(ws_e)
     if st != moe.MOE_OK:
         raise RuntimeError(moe.moe_error_string(st))
 
@@ -463,8 +497,10 @@ def run_ours(args):
     y_dev = torch.empty_like(y)
 
     # ---------------- roofline of the dominant kernel
+    # touched logical experts: the algorithmic bytes count each expert's
+    # weights once even when replicas stream copies of them
     counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
-    layer(x, out=y_dev, counts_out=counts)
+    moe.moe_forward(x, w_g, bias, w13, w2, y_dev, shape, ws, counts_out=counts)
     touched = int((counts > 0).sum().item())
     alg = algorithmic(cfg, touched)
     mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
@@ -519,6 +555,12 @@ def run_ours(args):
         "gpu_launches": 2 * launches_per_forward(cfg) * args.steps,
         "clocks": clk,
     }
+    if eplb_info is not None:
+        line["eplb"] = eplb_info
+        line["config"]["eplb_redundant"] = args.eplb_redundant
+        line["stage_ms_note"] += "; with --eplb-redundant the stages are the plain layer's"
+        line["gpu_launches"] = (launches_per_forward(cfg, args.eplb_redundant) +
+                                launches_per_forward(cfg)) * args.steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, {"x": x, "w_g": w_g, "bias": bias,
                                                   "w13": w13, "w2": w2})

@@ -76,7 +76,7 @@ typedef enum moe_status {
 /* Human-readable name of a moe_status. Never NULL. */
 MOE_API const char* moe_error_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 101 adds the EPLB calls. */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -221,6 +221,72 @@ MOE_API int moe_dispatch_noalloc(const int32_t* idx, const moe_bf16* x, const mo
                                  int32_t* counts, int32_t* offsets, int32_t* perm,
                                  int32_t* row_of, moe_bf16* x_perm, int32_t* send_counts,
                                  int32_t* rank_offsets, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Expert load balancing with replicated experts ("Serving MoE models with
+ * expert parallelism on 8xH200", section "Routing imbalance": measure
+ * per-expert load, place redundant copies of popular experts on less-loaded
+ * GPUs, co-locate hot and cold experts; "vLLM Expert Parallel deployment",
+ * EPLB section: load collected over a window, a number of redundant experts).
+ * The pages give no algorithm; these calls implement the plainest integer
+ * reading (the oracle's tests/golden/eplb_worked_examples.json cases are
+ * worked by hand from it):
+ *   1. each expert starts with one copy; n_redundant times the expert with
+ *      the largest load per copy gets another (ties: lower id);
+ *   2. replica i of expert e is credited load[e] / n_e, plus one if
+ *      i < load[e] mod n_e;
+ *   3. by decreasing credit (ties: lower expert, then lower replica) each
+ *      replica goes to the least-loaded rank with a free slot (ties: lower
+ *      rank); rank r owns physical experts r*S .. r*S+S-1, S = P / R, in the
+ *      order they were filled;
+ *   4. slot j of token t with logical expert e uses replica t mod n_e.
+ * ------------------------------------------------------------------------- */
+
+/* The replica plan, on the host (no device work, no allocation).
+ *   load            [E] int64 host in   per-expert load, 0 .. 2^50 (e.g. the
+ *                                       counts of moe_forward over a window)
+ *   E, R            logical experts, ranks (1 .. 64)
+ *   n_redundant     extra copies; P = E + n_redundant <= 1024, P % R == 0
+ *   phys_to_logical [P] int32 host out  logical expert of each physical slot
+ *   rep_offsets     [E+1] int32 host out  replicas of e are
+ *   rep_phys        [P] int32 host out    rep_phys[rep_offsets[e] .. rep_offsets[e+1])
+ * Returns MOE_ERR_INVALID_ARG for null pointers or out-of-range arguments. */
+MOE_API int moe_eplb_plan(const int64_t* load, int32_t E, int32_t R, int32_t n_redundant,
+                          int32_t* phys_to_logical, int32_t* rep_offsets,
+                          int32_t* rep_phys);
+
+/* Logical -> physical expert ids (rule 4), on the device:
+ *   idx [T, k] int32 in (logical ids < s->E); rep_offsets [s->E + 1],
+ *   rep_phys [E_phys] int32 in, device-resident (moe_eplb_plan's output);
+ *   idx_phys [T, k] int32 out.  ws: only its error word is used.
+ * An id or plan entry out of range gives -1 and MOE_ERR_DEVICE_CHECK. */
+MOE_API int moe_eplb_remap(const int32_t* idx, const moe_shape* s, const int32_t* rep_offsets,
+                           const int32_t* rep_phys, int32_t E_phys, int32_t* idx_phys,
+                           void* ws, void* stream);
+
+/* Workspace bytes for moe_forward_eplb (0 if the arguments are invalid). */
+MOE_API size_t moe_workspace_size_eplb(const moe_shape* s, int32_t E_phys);
+
+/* The layer with replicated experts: router and top-k over the s->E logical
+ * experts (as moe_forward), every selection mapped to its replica (rule 4),
+ * then dispatch, expert FFNs and combine over the E_phys physical experts.
+ *   w13_phys [E_phys, 2f, d], w2_phys [E_phys, d, f]: the weights of
+ *     physical expert p are those of logical expert phys_to_logical[p]
+ *     (the caller lays them out when it adopts a plan).
+ *   idx_out / w_out: logical ids and gates; counts_out [E_phys]: rows per
+ *     physical expert.  With s->R > 1, rank r owns physical experts
+ *     [r*E_phys/R, (r+1)*E_phys/R) in the virtual-EP layout.
+ * Replicas hold the same weights and every output row depends only on its own
+ * token, so y equals moe_forward's y; bit for bit whenever both pick the same
+ * expert-GEMM kernels (always up to 256 tokens; above, the CTA-pair choice
+ * depends on rows per expert, which replicas lower).
+ * ws: moe_workspace_size_eplb(s, E_phys) bytes, first 64 bytes zeroed once. */
+MOE_API int moe_forward_eplb(const moe_bf16* x, const float* w_g, const float* bias,
+                             const moe_bf16* w13_phys, const moe_bf16* w2_phys,
+                             const moe_shape* s, const int32_t* rep_offsets,
+                             const int32_t* rep_phys, int32_t E_phys, moe_bf16* y,
+                             int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
+                             void* stream);
 
 /* Self-test of the failure path every device-side wait uses: launches one
  * kernel that waits on a barrier nothing will ever complete, through the same

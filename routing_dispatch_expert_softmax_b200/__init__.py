@@ -12,5 +12,6 @@ from .binding import (EXPORTS, MOE_STAGE_EVENTS, STAGE_NAMES, MOE_ERR_CUDA, MOE_
                       moe_combine, moe_dispatch, moe_dispatch_noalloc, moe_error_string, moe_ffn,
                       moe_forward, moe_forward_staged, moe_router, moe_selftest_bounded_wait,
                       moe_topk, moe_version,
-                      moe_workspace_size, workspace)
+                      moe_workspace_size, workspace, moe_eplb_plan, moe_eplb_remap,
+                      moe_workspace_size_eplb, workspace_eplb, moe_forward_eplb)
 from .layer import MoELayer  # noqa: F401

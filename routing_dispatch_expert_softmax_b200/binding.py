@@ -29,7 +29,8 @@ MOE_ERR_DEVICE_CHECK = 5
 EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router",
            "moe_topk", "moe_dispatch", "moe_ffn", "moe_combine", "moe_forward",
            "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check",
-           "moe_dispatch_noalloc")
+           "moe_dispatch_noalloc", "moe_eplb_plan", "moe_eplb_remap",
+           "moe_workspace_size_eplb", "moe_forward_eplb")
 
 
 class MoEError(RuntimeError):
@@ -92,6 +93,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_check.argtypes = [_P, _P]
     lib.moe_selftest_bounded_wait.restype = ctypes.c_int
     lib.moe_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _P, _P]
+    _i32 = ctypes.c_int32
+    lib.moe_eplb_plan.restype = ctypes.c_int
+    lib.moe_eplb_plan.argtypes = [_P, _i32, _i32, _i32, _P, _P, _P]
+    lib.moe_eplb_remap.restype = ctypes.c_int
+    lib.moe_eplb_remap.argtypes = [_P, _S, _P, _P, _i32, _P, _P, _P]
+    lib.moe_workspace_size_eplb.restype = ctypes.c_size_t
+    lib.moe_workspace_size_eplb.argtypes = [_S, _i32]
+    lib.moe_forward_eplb.restype = ctypes.c_int
+    lib.moe_forward_eplb.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _i32, _P, _P, _P, _P,
+                                     _P, _P]
     _lib = lib
     return lib
 
@@ -208,6 +219,54 @@ def moe_forward(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, idx_out=None, w_o
         _ptr(idx_out, torch.int32, "idx_out"), _ptr(w_out, torch.float32, "w_out"),
         _ptr(counts_out, torch.int32, "counts_out"), _ptr(ws, torch.uint8, "ws"),
         _stream(stream)), "moe_forward")
+
+
+def moe_eplb_plan(load, E: int, R: int, n_redundant: int):
+    """Replica plan on the host: returns (phys_to_logical, rep_offsets,
+    rep_phys) as int32 CPU tensors.  ``load``: E per-expert loads."""
+    load = torch.as_tensor(load, dtype=torch.int64).contiguous()
+    if load.device.type != "cpu" or load.numel() != E:
+        raise ValueError("load: E int64 values on the host")
+    P = E + n_redundant
+    p2l = torch.empty(max(P, 1), dtype=torch.int32)
+    off = torch.empty(E + 1, dtype=torch.int32)
+    phys = torch.empty(max(P, 1), dtype=torch.int32)
+    _check(load_library().moe_eplb_plan(load.data_ptr(), E, R, n_redundant, p2l.data_ptr(),
+                                        off.data_ptr(), phys.data_ptr()), "moe_eplb_plan")
+    return p2l[:P], off, phys[:P]
+
+
+def moe_eplb_remap(idx, rep_offsets, rep_phys, E_phys: int, idx_phys, shape: MoEShape, ws,
+                   stream=None):
+    _check(load_library().moe_eplb_remap(
+        _ptr(idx, torch.int32, "idx"), ctypes.byref(shape),
+        _ptr(rep_offsets, torch.int32, "rep_offsets"), _ptr(rep_phys, torch.int32, "rep_phys"),
+        E_phys, _ptr(idx_phys, torch.int32, "idx_phys"), _ptr(ws, torch.uint8, "ws"),
+        _stream(stream)), "moe_eplb_remap")
+
+
+def moe_workspace_size_eplb(shape: MoEShape, E_phys: int) -> int:
+    return int(load_library().moe_workspace_size_eplb(ctypes.byref(shape), E_phys))
+
+
+def workspace_eplb(shape: MoEShape, E_phys: int, device="cuda") -> torch.Tensor:
+    n = moe_workspace_size_eplb(shape, E_phys)
+    if n == 0:
+        raise ValueError("invalid shape or E_phys for moe_forward_eplb")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_forward_eplb(x, w_g, bias, w13_phys, w2_phys, y, shape: MoEShape, rep_offsets,
+                     rep_phys, E_phys: int, ws, idx_out=None, w_out=None, counts_out=None,
+                     stream=None):
+    _check(load_library().moe_forward_eplb(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13_phys, torch.bfloat16, "w13_phys"),
+        _ptr(w2_phys, torch.bfloat16, "w2_phys"), ctypes.byref(shape),
+        _ptr(rep_offsets, torch.int32, "rep_offsets"), _ptr(rep_phys, torch.int32, "rep_phys"),
+        E_phys, _ptr(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
+        _ptr(w_out, torch.float32, "w_out"), _ptr(counts_out, torch.int32, "counts_out"),
+        _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_forward_eplb")
 
 
 MOE_STAGE_EVENTS = 6

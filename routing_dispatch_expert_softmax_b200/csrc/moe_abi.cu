@@ -9,7 +9,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kVersion = 100;
+constexpr int kVersion = 101;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
@@ -264,6 +264,80 @@ int moe_forward_staged(const moe_bf16* x, const float* w_g, const float* bias,
                        moe_bf16* y, void* ws, void* const* events, void* stream) {
   return forward_impl(x, w_g, bias, w13, w2, s, y, nullptr, nullptr, nullptr, ws, stream,
                       events);
+}
+
+size_t moe_workspace_size_eplb(const moe_shape* s, int32_t E_phys) {
+  if (!shape_ok(s) || E_phys < s->E || E_phys > kMaxE || (s->R > 1 && E_phys % s->R))
+    return 0;
+  return ws_layout(*s, 0, E_phys).total;
+}
+
+int moe_eplb_remap(const int32_t* idx, const moe_shape* s, const int32_t* rep_offsets,
+                   const int32_t* rep_phys, int32_t E_phys, int32_t* idx_phys, void* ws,
+                   void* stream) {
+  if (!shape_ok(s) || E_phys < s->E || E_phys > kMaxE) return MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok4(idx) || !ok4(rep_offsets) || !ok4(rep_phys) || !ok4(idx_phys))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_eplb_remap(idx, s->T, s->k, s->E, rep_offsets, rep_phys, E_phys,
+                                       idx_phys, static_cast<int*>(ws),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_forward_eplb(const moe_bf16* x, const float* w_g, const float* bias,
+                     const moe_bf16* w13_phys, const moe_bf16* w2_phys, const moe_shape* s,
+                     const int32_t* rep_offsets, const int32_t* rep_phys, int32_t E_phys,
+                     moe_bf16* y, int32_t* idx_out, float* w_out, int32_t* counts_out,
+                     void* ws, void* stream) {
+  if (!shape_ok(s) || E_phys < s->E || E_phys > kMaxE || (s->R > 1 && E_phys % s->R))
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(x) || !ok4(w_g) || (bias && !aligned(bias, 4)) || !ok16(w13_phys) ||
+      !ok16(w2_phys) || !ok16(y) || !ok4(rep_offsets) || !ok4(rep_phys) ||
+      (idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4)) ||
+      (counts_out && !aligned(counts_out, 4)))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  moe_shape sp = *s;  // the physical experts: dispatch tables and expert GEMMs
+  sp.E = E_phys;
+  const WsLayout L = ws_layout(*s, sms, E_phys);
+  char* wsb = static_cast<char*>(ws);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  float* logits = at<float>(ws, L.logits);
+  int* idx = idx_out ? idx_out : at<int>(ws, L.idx);
+  int* idx_p = at<int>(ws, L.idx_phys);
+  float* gw = w_out ? w_out : at<float>(ws, L.w);
+  int* counts = counts_out ? counts_out : at<int>(ws, L.counts);
+  int* perm = at<int>(ws, L.perm);
+  int* row_of = at<int>(ws, L.row_of);
+  __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+  __nv_bfloat16* z = at<__nv_bfloat16>(ws, L.z);
+  int* err = at<int>(ws, L.err);
+  // router and selection over the logical experts, then each selection to
+  // its replica, then the layer over the physical experts
+  cudaError_t e = run_router(xb, w_g, bias, *s, logits, L, ws, sms, cs);
+  if (e == cudaSuccess) e = launch_topk(logits, *s, idx, gw, cs);
+  if (e == cudaSuccess)
+    e = launch_eplb_remap(idx, s->T, s->k, s->E, rep_offsets, rep_phys, E_phys, idx_p, err, cs);
+  if (e == cudaSuccess)
+    e = launch_route_tables(idx_p, sp, L, wsb, counts, at<int>(ws, L.offsets), row_of, perm,
+                            at<int>(ws, L.send), at<int>(ws, L.rank_off), cs);
+  if (e == cudaSuccess) e = launch_gather(xb, perm, L.P, s->T, s->d, x_perm, err, cs);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  int r = launch_expert_ffn(x_perm, L.Ppad, reinterpret_cast<const __nv_bfloat16*>(w13_phys),
+                            reinterpret_cast<const __nv_bfloat16*>(w2_phys), sp, L, wsb, z, sms,
+                            cs, nullptr);
+  if (r != MOE_OK) return r;
+  return cuda_status(
+      launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs));
 }
 
 int moe_selftest_bounded_wait(long long limit_ns, void* ws, void* stream) {

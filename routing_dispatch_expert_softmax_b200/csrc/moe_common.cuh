@@ -70,7 +70,7 @@ __device__ __forceinline__ void record_error(int* err, int code, int detail) {
 
 // ----------------------------------------------------------------- workspace
 struct WsLayout {
-  size_t err, w3, logit_part, logits, idx, w, counts, offsets, blockhist, blockbase,
+  size_t err, w3, logit_part, logits, idx, idx_phys, w, counts, offsets, blockhist, blockbase,
       blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, total;
   int nblocks;      // token blocks of kTokensPerRouteBlock
   int max_mtiles;   // upper bound of 128-row expert tiles
@@ -103,9 +103,14 @@ __host__ __device__ inline int* expert_entries(int* tiles) { return tiles + 4; }
 __host__ __device__ inline int* leftover_entries(int* tiles, int E) { return tiles + 4 + 3 * E; }
 __host__ __device__ inline int* row_tile_entries(int* tiles, int E) { return tiles + 4 + 6 * E; }
 
-inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
+// E_tab: experts of the dispatch tables and expert GEMMs (the physical
+// experts when replicas are used, moe_forward_eplb); the router regions use
+// the s.E logical experts.  -1: E_tab = s.E.
+inline WsLayout ws_layout(const moe_shape& s, int num_sms, int E_tab = -1) {
   WsLayout L{};
-  const long long T = s.T, E = s.E, k = s.k, d = s.d, f = s.f;
+  const long long T = s.T, k = s.k, d = s.d, f = s.f;
+  const long long E_log = s.E;
+  const long long E = E_tab > 0 ? E_tab : s.E;
   const long long R = s.R > 1 ? s.R : 1;
   L.P = T * k;
   L.Ppad = L.P + kGemmBM;
@@ -120,11 +125,12 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms) {
     return at;
   };
   L.err = take(64);
-  L.w3 = take(2 * 3 * (size_t)d * E);  // router weight split into 3 bf16 planes
-  L.logit_part = take(sizeof(float) * (size_t)router_tc_parts(s) * T * E);
+  L.w3 = take(2 * 3 * (size_t)d * E_log);  // router weight split into 3 bf16 planes
+  L.logit_part = take(sizeof(float) * (size_t)router_tc_parts(s) * T * E_log);
 
-  L.logits = take(sizeof(float) * T * E);
+  L.logits = take(sizeof(float) * T * E_log);
   L.idx = take(sizeof(int) * T * k);
+  L.idx_phys = take(sizeof(int) * T * k);
   L.w = take(sizeof(float) * T * k);
   L.counts = take(sizeof(int) * E);
   L.offsets = take(sizeof(int) * (E + 1));

@@ -38,4 +38,9 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       __nv_bfloat16* z, int num_sms, cudaStream_t st,
                       void* const* events = nullptr);
 
+// Logical -> physical expert ids of a replica plan (moe_eplb.cu).
+cudaError_t launch_eplb_remap(const int* idx, int T, int k, int E, const int* rep_offsets,
+                              const int* rep_phys, int P, int* idx_phys, int* err,
+                              cudaStream_t st);
+
 }  // namespace moe

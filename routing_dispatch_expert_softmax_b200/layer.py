@@ -1,7 +1,8 @@
 """``MoELayer``: the user-facing call of the routed MoE layer forward.
 
 Holds the layer's weights (device tensors) and per-batch-size workspaces, and
-runs the whole layer through the C ABI's ``moe_forward``.  All arithmetic
+runs the whole layer through the C ABI's ``moe_forward`` (``moe_forward_eplb``
+once ``rebalance`` has adopted a replica plan).  All arithmetic
 happens in the library's CUDA kernels.  ``forward_graphed`` /
 ``forward_host`` replay a CUDA graph of the layer captured once per batch size
 (static input/output buffers), which removes the per-call launch cost that
@@ -24,17 +25,14 @@ class _Graphed:
         dev = layer.w13.device
         self.x = torch.zeros(T, layer.d, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(T, layer.d, dtype=torch.bfloat16, device=dev)
-        self.ws = B.workspace(layer.shape(T), dev)
-        shape = layer.shape(T)
+        self.ws = layer._new_workspace(T)
         # One eager call first: first-use set-up (kernel attributes, driver
         # entry points) must not happen under capture.
-        B.moe_forward(self.x, layer.w_g, layer.bias, layer.w13, layer.w2, self.y, shape,
-                      self.ws)
+        layer._call(self.x, self.y, self.ws)
         torch.cuda.current_stream(dev).synchronize()
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
-            B.moe_forward(self.x, layer.w_g, layer.bias, layer.w13, layer.w2, self.y, shape,
-                          self.ws)
+            layer._call(self.x, self.y, self.ws)
 
 
 class MoELayer:
@@ -52,14 +50,54 @@ class MoELayer:
         self._ws: Dict[int, torch.Tensor] = {}
         self._graphs: Dict[int, _Graphed] = {}
         self._last_ws: Optional[torch.Tensor] = None
+        self._eplb: Optional[dict] = None
 
     def shape(self, T: int) -> B.MoEShape:
         return B.MoEShape.of(T, self.d, self.E, self.k, self.f, self.R)
 
+    def _new_workspace(self, T: int) -> torch.Tensor:
+        if self._eplb is None:
+            return B.workspace(self.shape(T), self.w13.device)
+        return B.workspace_eplb(self.shape(T), self._eplb["E_phys"], self.w13.device)
+
     def workspace(self, T: int) -> torch.Tensor:
         if T not in self._ws:
-            self._ws[T] = B.workspace(self.shape(T), self.w13.device)
+            self._ws[T] = self._new_workspace(T)
         return self._ws[T]
+
+    def _call(self, x, y, ws, idx_out=None, w_out=None, counts_out=None, stream=None):
+        shape = self.shape(int(x.shape[0]))
+        if self._eplb is None:
+            B.moe_forward(x, self.w_g, self.bias, self.w13, self.w2, y, shape, ws,
+                          idx_out=idx_out, w_out=w_out, counts_out=counts_out, stream=stream)
+        else:
+            p = self._eplb
+            B.moe_forward_eplb(x, self.w_g, self.bias, p["w13"], p["w2"], y, shape, p["off"],
+                               p["phys"], p["E_phys"], ws, idx_out=idx_out, w_out=w_out,
+                               counts_out=counts_out, stream=stream)
+
+    def rebalance(self, load, n_redundant: int):
+        """Adopt an EPLB-style replica plan built from per-expert ``load``
+        (e.g. counts gathered over a window of calls): n_redundant extra
+        copies of the busiest experts, placed on max(R, 1) virtual ranks.
+        The physical weights are laid out once here; later calls run
+        moe_forward_eplb, whose ``counts_out`` then has E + n_redundant
+        entries (rows per physical expert).  Returns the plan
+        (phys_to_logical, rep_offsets, rep_phys) as CPU int32 tensors."""
+        dev = self.w13.device
+        p2l, off, phys = B.moe_eplb_plan(load, self.E, max(self.R, 1), n_redundant)
+        sel = p2l.long().to(dev)
+        self._eplb = dict(E_phys=self.E + int(n_redundant),
+                          w13=self.w13.index_select(0, sel).contiguous(),
+                          w2=self.w2.index_select(0, sel).contiguous(),
+                          off=off.to(dev), phys=phys.to(dev))
+        self._ws.clear()
+        self._graphs.clear()
+        return p2l, off, phys
+
+    @property
+    def physical_experts(self) -> int:
+        return self.E if self._eplb is None else self._eplb["E_phys"]
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
                 idx_out=None, w_out=None, counts_out=None, stream=None) -> torch.Tensor:
@@ -68,8 +106,8 @@ class MoELayer:
         y = out if out is not None else torch.empty_like(x)
         ws = self.workspace(T)
         self._last_ws = ws
-        B.moe_forward(x, self.w_g, self.bias, self.w13, self.w2, y, self.shape(T), ws,
-                      idx_out=idx_out, w_out=w_out, counts_out=counts_out, stream=stream)
+        self._call(x, y, ws, idx_out=idx_out, w_out=w_out, counts_out=counts_out,
+                   stream=stream)
         return y
 
     __call__ = forward

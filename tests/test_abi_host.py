@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_error_strings(lib):
-    assert moe.moe_version() == 100
+    assert moe.moe_version() == 101
     for code in range(6):
         assert moe.moe_error_string(code).startswith("MOE_")
     assert "unknown" in moe.moe_error_string(99)
@@ -111,6 +111,15 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     assert _raw(lib, "moe_selftest_bounded_wait", ctypes.c_longlong(2 * 10 ** 9), _P(A16),
                 None) == INV
     assert _raw(lib, "moe_check", _P(A16 + 8), None) == INV
+    # EPLB: fewer physical than logical experts, misaligned plan, null workspace
+    assert _raw(lib, "moe_eplb_remap", _P(A16), s, _P(A16), _P(A16), VALID["E"] - 1, _P(A16),
+                _P(A16), None) == INV
+    assert _raw(lib, "moe_eplb_remap", _P(A16), s, _P(A16 + 2), _P(A16), VALID["E"], _P(A16),
+                _P(A16), None) == INV
+    assert _raw(lib, "moe_forward_eplb", *[_P(A16)] * 5, s, _P(A16), _P(A16), VALID["E"] + 8,
+                _P(A16), None, None, None, None, None) == INV
+    assert _raw(lib, "moe_forward_eplb", *[_P(A16)] * 5, s, _P(A16), _P(A16), 1025,
+                _P(A16), None, None, None, _P(A16), None) == INV
 
 
 def test_empty_batch_is_a_no_op(lib):
@@ -136,3 +145,50 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA tensor"):
         moe.moe_combine(x, x, x, x, B.MoEShape.of(4, 64, 8, 1, 64))
+
+
+# ---------------------------------------------------------------- EPLB plan (host code)
+def test_eplb_plan_matches_oracle_on_random_loads(lib):
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        R = int(rng.choice([1, 2, 4, 8]))
+        E = R * int(rng.integers(1, 17))
+        rd = R * int(rng.integers(0, 4))
+        load = (rng.zipf(1.2, E).clip(max=1000) * int(rng.integers(1, 50))).tolist()
+        if rng.random() < 0.2:
+            load = [int(rng.integers(0, 3))] * E  # all ties
+        want = [a.tolist() for a in oracle.eplb_plan(load, rd, R)]
+        got = [a.tolist() for a in moe.moe_eplb_plan(load, E, R, rd)]
+        assert got == want, (load, rd, R)
+
+
+def test_eplb_plan_rejects_bad_arguments(lib):
+    import numpy as np
+    load = np.ones(8, dtype=np.int64)
+    out = [np.zeros(16, dtype=np.int32) for _ in range(3)]
+    INV = B.MOE_ERR_INVALID_ARG
+
+    def call(E, R, rd, lo=load):
+        return lib.moe_eplb_plan(lo.ctypes.data, E, R, rd, out[0].ctypes.data,
+                                 out[1].ctypes.data, out[2].ctypes.data)
+    assert call(8, 4, 4) == B.MOE_OK
+    assert call(8, 3, 0) == INV          # 8 slots on 3 ranks
+    assert call(8, 4, -4) == INV
+    assert call(0, 1, 0) == INV
+    assert call(8, 65, 57) == INV        # R above 64
+    assert call(1024, 1, 8) == INV       # more than 1024 physical experts
+    neg = load.copy()
+    neg[3] = -1
+    assert call(8, 4, 4, neg) == INV
+    assert lib.moe_eplb_plan(None, 8, 4, 4, out[0].ctypes.data, out[1].ctypes.data,
+                             out[2].ctypes.data) == INV
+
+
+def test_eplb_workspace_size(lib):
+    s = B.MoEShape.of(**VALID)
+    assert moe.moe_workspace_size_eplb(s, VALID["E"] + 8) >= moe.moe_workspace_size(s)
+    assert moe.moe_workspace_size_eplb(s, VALID["E"] - 1) == 0
+    assert moe.moe_workspace_size_eplb(s, 1025) == 0
