@@ -503,3 +503,8 @@ def test_layer_graph_replay_matches_eager():
     assert layer.check() == moe.MOE_OK
     assert torch.equal(y_eager, y_graph) and torch.equal(y2_eager, y2_graph)
     assert torch.equal(y_host, y_eager.cpu())
+    # the host graph re-reads the pinned input on every replay
+    x_host.copy_(x2.cpu())
+    layer.forward_host(x_host, y_host)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, y2_eager.cpu())
