@@ -413,3 +413,61 @@ def test_eplb_remap_conserves_counts_and_uses_t_mod_copies():
     # the balanced placement evens the per-rank rows out on this skewed batch
     assert (oracle.rank_loads(counts_p, R).max() <
             oracle.rank_loads(counts, R).max())
+
+
+# ---------------------------------------------------------------- token-deduplicated dispatch
+def test_dedup_layout_matches_hand_worked_example():
+    path = os.path.join(os.path.dirname(__file__), "golden", "dedup_worked_example.json")
+    with open(path) as fh:
+        c = json.load(fh)
+    S, off, tok, mask, row_of = oracle.dedup_layout(np.array(c["idx"]), c["E"], c["R"])
+    assert S.tolist() == c["send_counts"]
+    assert off.tolist() == c["rank_offsets"]
+    assert tok.tolist() == c["token_of"]
+    assert mask.tolist() == c["slot_mask"]
+    assert row_of.tolist() == c["rank_row_of"]
+
+
+def test_dedup_layout_reduces_to_the_plain_layout_for_k1_and_r1():
+    rng = np.random.default_rng(5)
+    T, E, R = 37, 16, 4
+    idx = rng.integers(0, E, (T, 1))
+    S, off, tok, mask, _ = oracle.dedup_layout(idx, E, R)
+    S_plain, off_plain = oracle.virtual_ep_layout(idx, E, R)
+    np.testing.assert_array_equal(S, S_plain)
+    np.testing.assert_array_equal(off, off_plain)
+    assert (mask == 1).all()
+    # R = 1: every token once, all k slots local
+    idx = oracle.topk_select_sorted(rng.normal(size=(T, E)).astype(np.float32), 3)
+    S, off, tok, mask, _ = oracle.dedup_layout(idx, E, 1)
+    assert S.tolist() == [[T]] and tok.tolist() == list(range(T)) and (mask == 7).all()
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_dedup_layout_invariants(seed):
+    rng = np.random.default_rng(seed)
+    R = int(rng.choice([2, 4, 8]))
+    E = R * int(rng.integers(1, 9))
+    k = int(rng.integers(1, min(E, 8) + 1))
+    T = int(rng.integers(1, 200))
+    idx = oracle.topk_select_sorted(rng.normal(size=(T, E)).astype(np.float32), k)
+    S, off, tok, mask, row_of = oracle.dedup_layout(idx, E, R)
+    S_plain, _ = oracle.virtual_ep_layout(idx, E, R)
+    assert (S <= S_plain).all() and (S > 0).sum() == (S_plain > 0).sum()
+    per = E // R
+    for t in range(T):
+        rows = [row_of[t, r] for r in range(R) if row_of[t, r] >= 0]
+        got = 0
+        for row in rows:
+            assert tok[row] == t
+            assert (got & int(mask[row])) == 0            # slots split across ranks
+            got |= int(mask[row])
+        assert got == (1 << k) - 1                         # every slot goes somewhere
+        for r in range(R):
+            want = sum(1 << j for j in range(k) if idx[t, j] // per == r)
+            assert (row_of[t, r] >= 0) == (want != 0)
+            if want:
+                assert mask[row_of[t, r]] == want
+    for r in range(R):                                     # tokens ascending per rank
+        seg = tok[off[r]:off[r + 1]]
+        assert (np.diff(seg) > 0).all()
