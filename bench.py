@@ -496,6 +496,55 @@ def run_ours(args):
     e2e_value = tokens / (e2e_ms / 1e3)
     y_dev = torch.empty_like(y)
 
+    # ---------------- dispatch exchange volume (virtual EP, R > 1)
+    # The plain dispatch buffer (one row per (token, slot)) against the
+    # token-deduplicated one (one row per (token, destination rank)), each
+    # timed alone on the device after an L2 flush: rows are what an
+    # all-to-all would carry.
+    dedup_info = None
+    if cfg.R > 1:
+        idx_d = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+        moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, idx_out=idx_d)
+        P = cfg.T * cfg.k
+        rows_max = cfg.T * min(cfg.k, cfg.R)
+        i32 = lambda n: torch.empty(n, dtype=torch.int32, device=dev)
+        cnt, offs, perm_, row_of_, xp = (i32(cfg.E), i32(cfg.E + 1), i32(P), i32(P),
+                                         torch.empty(P, cfg.d, dtype=torch.bfloat16, device=dev))
+        snd, roff = i32(cfg.R * cfg.R), i32(cfg.R + 1)
+        snd2, roff2, tok, msk = i32(cfg.R * cfg.R), i32(cfg.R + 1), i32(rows_max), i32(rows_max)
+        xd = torch.empty(rows_max, cfg.d, dtype=torch.bfloat16, device=dev)
+
+        def plain_dispatch():
+            moe.moe_dispatch(idx_d, x, cnt, offs, perm_, row_of_, xp, shape, ws, snd, roff)
+
+        def dedup_dispatch():
+            moe.moe_dispatch_dedup(idx_d, x, snd2, roff2, tok, msk, shape, ws, x_dedup=xd)
+
+        times = {}
+        for name, fn in (("plain", plain_dispatch), ("dedup", dedup_dispatch)):
+            for _ in range(3):
+                fn()
+            acc = 0.0
+            for _ in range(10):
+                flush_l2()
+                a, b = ev(), ev()
+                a.record(stream)
+                fn()
+                b.record(stream)
+                b.synchronize()
+                acc += a.elapsed_time(b)
+            times[name] = acc / 10 * 1e3
+        st = moe.moe_check(ws)
+        if st != moe.MOE_OK:
+            raise RuntimeError(moe.moe_error_string(st))
+        rows_dedup = int(roff2[-1].item())
+        dedup_info = {"rows_plain": P, "rows_dedup": rows_dedup,
+                      "bytes_plain": P * cfg.d * 2, "bytes_dedup": rows_dedup * cfg.d * 2,
+                      "us_plain_dispatch": times["plain"], "us_dedup_dispatch": times["dedup"],
+                      "note": "moe_dispatch vs moe_dispatch_dedup on this batch's selection, "
+                              "each timed alone after an L2 flush; rows are what an "
+                              "all-to-all would carry"}
+
     # ---------------- roofline of the dominant kernel
     # touched logical experts: the algorithmic bytes count each expert's
     # weights once even when replicas stream copies of them
@@ -555,6 +604,8 @@ def run_ours(args):
         "gpu_launches": 2 * launches_per_forward(cfg) * args.steps,
         "clocks": clk,
     }
+    if dedup_info is not None:
+        line["dispatch_volume"] = dedup_info
     if eplb_info is not None:
         line["eplb"] = eplb_info
         line["config"]["eplb_redundant"] = args.eplb_redundant

@@ -76,7 +76,8 @@ typedef enum moe_status {
 /* Human-readable name of a moe_status. Never NULL. */
 MOE_API const char* moe_error_string(int status);
 
-/* Library ABI version (major * 100 + minor): 101 adds the EPLB calls. */
+/* Library ABI version (major * 100 + minor): 101 adds the EPLB calls and
+ * moe_dispatch_dedup. */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -221,6 +222,32 @@ MOE_API int moe_dispatch_noalloc(const int32_t* idx, const moe_bf16* x, const mo
                                  int32_t* counts, int32_t* offsets, int32_t* perm,
                                  int32_t* row_of, moe_bf16* x_perm, int32_t* send_counts,
                                  int32_t* rank_offsets, void* stream);
+
+/* Token-deduplicated per-rank dispatch ("Serving MoE models with expert
+ * parallelism on 8xH200", section "Tensor parallel vs expert parallel";
+ * "Expert Parallelism for MoE Models", section "Mechanics of Token Routing
+ * and All-to-All Communication": a token's representation travels to the
+ * devices holding its experts).  A token goes once to every virtual rank that
+ * owns at least one of its k experts (owner(e) = e / (E/R), source rank
+ * t / ceil(T/R)); the send buffer is rank-major with tokens ascending inside a
+ * rank (the pages give no layout; this is the plainest reading).  Needs
+ * s->R >= 2.  rows = T * min(k, R) bounds the buffer.
+ *   idx          [T, k] int32 in    expert ids
+ *   x            [T, d] bf16 in     (only read when x_dedup != NULL)
+ *   send_counts  [R, R] int32 out   tokens source rank s sends to rank r
+ *   rank_offsets [R+1] int32 out    first row of each destination rank;
+ *                                   rank_offsets[R] = rows used
+ *   token_of     [rows] int32 out   token of each row
+ *   slot_mask    [rows] uint32 out  bit j: slot j's expert is on that rank
+ *   rank_row_of  [T, R] int32 out or NULL: row of (t, r), -1 if none
+ *   x_dedup      [rows, d] bf16 out or NULL: x[token_of[row]]
+ *   ws           workspace of moe_workspace_size(s) bytes
+ * Out-of-range ids are recorded as MOE_ERR_DEVICE_CHECK and skipped.      */
+MOE_API int moe_dispatch_dedup(const int32_t* idx, const moe_bf16* x, const moe_shape* s,
+                               int32_t* send_counts, int32_t* rank_offsets,
+                               int32_t* token_of, uint32_t* slot_mask,
+                               int32_t* rank_row_of, moe_bf16* x_dedup, void* ws,
+                               void* stream);
 
 /* ---------------------------------------------------------------------------
  * Expert load balancing with replicated experts ("Serving MoE models with

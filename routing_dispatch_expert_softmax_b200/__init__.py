@@ -13,5 +13,6 @@ from .binding import (EXPORTS, MOE_STAGE_EVENTS, STAGE_NAMES, MOE_ERR_CUDA, MOE_
                       moe_forward, moe_forward_staged, moe_router, moe_selftest_bounded_wait,
                       moe_topk, moe_version,
                       moe_workspace_size, workspace, moe_eplb_plan, moe_eplb_remap,
-                      moe_workspace_size_eplb, workspace_eplb, moe_forward_eplb)
+                      moe_workspace_size_eplb, workspace_eplb, moe_forward_eplb,
+                      moe_dispatch_dedup)
 from .layer import MoELayer  # noqa: F401

@@ -30,7 +30,7 @@ EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router"
            "moe_topk", "moe_dispatch", "moe_ffn", "moe_combine", "moe_forward",
            "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check",
            "moe_dispatch_noalloc", "moe_eplb_plan", "moe_eplb_remap",
-           "moe_workspace_size_eplb", "moe_forward_eplb")
+           "moe_workspace_size_eplb", "moe_forward_eplb", "moe_dispatch_dedup")
 
 
 class MoEError(RuntimeError):
@@ -100,6 +100,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_eplb_remap.argtypes = [_P, _S, _P, _P, _i32, _P, _P, _P]
     lib.moe_workspace_size_eplb.restype = ctypes.c_size_t
     lib.moe_workspace_size_eplb.argtypes = [_S, _i32]
+    lib.moe_dispatch_dedup.restype = ctypes.c_int
+    lib.moe_dispatch_dedup.argtypes = [_P, _P, _S, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.moe_forward_eplb.restype = ctypes.c_int
     lib.moe_forward_eplb.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _i32, _P, _P, _P, _P,
                                      _P, _P]
@@ -219,6 +221,19 @@ def moe_forward(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, idx_out=None, w_o
         _ptr(idx_out, torch.int32, "idx_out"), _ptr(w_out, torch.float32, "w_out"),
         _ptr(counts_out, torch.int32, "counts_out"), _ptr(ws, torch.uint8, "ws"),
         _stream(stream)), "moe_forward")
+
+
+def moe_dispatch_dedup(idx, x, send_counts, rank_offsets, token_of, slot_mask, shape: MoEShape,
+                       ws, rank_row_of=None, x_dedup=None, stream=None):
+    """Token-deduplicated per-rank dispatch (uint32 slot masks are passed as
+    int32 tensors of the same bits)."""
+    _check(load_library().moe_dispatch_dedup(
+        _ptr(idx, torch.int32, "idx"), _ptr(x, torch.bfloat16, "x"), ctypes.byref(shape),
+        _ptr(send_counts, torch.int32, "send_counts"),
+        _ptr(rank_offsets, torch.int32, "rank_offsets"), _ptr(token_of, torch.int32, "token_of"),
+        _ptr(slot_mask, torch.int32, "slot_mask"), _ptr(rank_row_of, torch.int32, "rank_row_of"),
+        _ptr(x_dedup, torch.bfloat16, "x_dedup"), _ptr(ws, torch.uint8, "ws"),
+        _stream(stream)), "moe_dispatch_dedup")
 
 
 def moe_eplb_plan(load, E: int, R: int, n_redundant: int):

@@ -111,6 +111,14 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     assert _raw(lib, "moe_selftest_bounded_wait", ctypes.c_longlong(2 * 10 ** 9), _P(A16),
                 None) == INV
     assert _raw(lib, "moe_check", _P(A16 + 8), None) == INV
+    # dedup dispatch: needs R >= 2 and a workspace
+    s_r4 = ctypes.byref(B.MoEShape.of(**dict(VALID, R=4)))
+    assert _raw(lib, "moe_dispatch_dedup", _P(A16), None, s, _P(A16), _P(A16), _P(A16),
+                _P(A16), None, None, _P(A16), None) == INV
+    assert _raw(lib, "moe_dispatch_dedup", _P(A16), None, s_r4, _P(A16), _P(A16), _P(A16),
+                _P(A16), None, None, None, None) == INV
+    assert _raw(lib, "moe_dispatch_dedup", _P(A16), None, s_r4, _P(A16), _P(A16), _P(A16),
+                _P(A16), None, _P(A16), _P(A16), None) == INV   # x_dedup without x
     # EPLB: fewer physical than logical experts, misaligned plan, null workspace
     assert _raw(lib, "moe_eplb_remap", _P(A16), s, _P(A16), _P(A16), VALID["E"] - 1, _P(A16),
                 _P(A16), None) == INV
