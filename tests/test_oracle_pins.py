@@ -471,3 +471,99 @@ def test_dedup_layout_invariants(seed):
     for r in range(R):                                     # tokens ascending per rank
         seg = tok[off[r]:off[r + 1]]
         assert (np.diff(seg) > 0).all()
+
+
+# ---------------------------------------------------------------- planted mistakes (EPLB, dedup)
+def _eplb_pins_fail(monkeypatch, module, name, bad):
+    monkeypatch.setattr(module, name, bad)
+    monkeypatch.setattr(oracle, name, bad)
+    failures = 0
+    checks = [lambda c=c: test_eplb_plan_matches_hand_worked_examples(c) for c in _eplb_cases()]
+    checks += [test_eplb_replication_minimises_the_largest_load_per_copy,
+               test_eplb_remap_conserves_counts_and_uses_t_mod_copies]
+    for fn in checks:
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            failures += 1
+    return failures
+
+
+def test_planted_replication_tie_to_higher_id_is_caught(monkeypatch):
+    def bad(load, n_redundant):
+        load = [int(v) for v in load]
+        n = [1] * len(load)
+        for _ in range(int(n_redundant)):
+            best = 0
+            for e in range(1, len(load)):
+                if load[e] * n[best] >= load[best] * n[e]:  # ties to the higher id
+                    best = e
+            n[best] += 1
+        return np.array(n, dtype=np.int64)
+    assert _eplb_pins_fail(monkeypatch, oracle.eplb_oracle, "eplb_replicate", bad) > 0
+
+
+def test_planted_placement_on_most_loaded_rank_is_caught(monkeypatch):
+    real_shares = oracle.eplb_oracle.eplb_shares
+
+    def bad(load, n, R):
+        n = [int(c) for c in n]
+        P = sum(n)
+        S = P // R
+        reps = sorted(real_shares(load, n), key=lambda r: (-r[2], r[0], r[1]))
+        rank_load, rank_fill = [0] * R, [0] * R
+        off = np.concatenate([[0], np.cumsum(n)]).astype(np.int64)
+        phys, p2l = np.full(P, -1, np.int64), np.full(P, -1, np.int64)
+        for e, i, share in reps:
+            r = max((r for r in range(R) if rank_fill[r] < S), key=lambda r: (rank_load[r], -r))
+            slot = r * S + rank_fill[r]
+            rank_fill[r] += 1
+            rank_load[r] += share
+            phys[off[e] + i] = slot
+            p2l[slot] = e
+        return p2l, off, phys
+    assert _eplb_pins_fail(monkeypatch, oracle.eplb_oracle, "eplb_place", bad) > 0
+
+
+def test_planted_replica_choice_by_division_is_caught(monkeypatch):
+    def bad(idx, off, phys):
+        idx = np.asarray(idx, dtype=np.int64)
+        out = np.empty_like(idx)
+        for t in range(idx.shape[0]):
+            for j in range(idx.shape[1]):
+                e = idx[t, j]
+                c = off[e + 1] - off[e]
+                out[t, j] = phys[off[e] + min(t // 97, c - 1)]
+        return out
+    assert _eplb_pins_fail(monkeypatch, oracle.eplb_oracle, "eplb_remap", bad) > 0
+
+
+def test_planted_dedup_mistakes_are_caught(monkeypatch):
+    real = oracle.dedup_oracle.dedup_layout
+
+    def reversed_masks(idx, E, R):
+        S, off, tok, mask, row_of = real(idx, E, R)
+        k = np.asarray(idx).shape[1]
+        flip = np.array([int(format(int(m), f"0{k}b")[::-1], 2) for m in mask], dtype=np.uint32)
+        return S, off, tok, flip, row_of
+
+    def tokens_descending(idx, E, R):
+        S, off, tok, mask, row_of = real(idx, E, R)
+        tok, mask = tok.copy(), mask.copy()
+        for r in range(R):
+            tok[off[r]:off[r + 1]] = tok[off[r]:off[r + 1]][::-1]
+            mask[off[r]:off[r + 1]] = mask[off[r]:off[r + 1]][::-1]
+        return S, off, tok, mask, row_of
+
+    for bad in (reversed_masks, tokens_descending):
+        monkeypatch.setattr(oracle.dedup_oracle, "dedup_layout", bad)
+        monkeypatch.setattr(oracle, "dedup_layout", bad)
+        failures = 0
+        for fn in (test_dedup_layout_matches_hand_worked_example,
+                   lambda: test_dedup_layout_invariants(0),
+                   lambda: test_dedup_layout_invariants(1)):
+            try:
+                fn()
+            except (AssertionError, ValueError, IndexError):
+                failures += 1
+        assert failures > 0, bad.__name__
