@@ -8,8 +8,11 @@ library and never receives a value computed by it.
 from .moe_oracle import *  # noqa: F401,F403
 from .eplb_oracle import *  # noqa: F401,F403
 from .dedup_oracle import *  # noqa: F401,F403
+from .fp8_oracle import *  # noqa: F401,F403
 from . import dedup_oracle as _dedup
 from . import eplb_oracle as _eplb
+from . import fp8_oracle as _fp8
 from . import moe_oracle as _moe
 
-__all__ = list(_moe.__all__) + list(_eplb.__all__) + list(_dedup.__all__)
+__all__ = (list(_moe.__all__) + list(_eplb.__all__) + list(_dedup.__all__)
+           + list(_fp8.__all__))

@@ -32,6 +32,7 @@ from typing import Optional
 import torch
 
 X_ID, WG_ID, PERM_ID, W13_ID, W2_ID = 1, 2, 3, 4, 5
+W13Q_ID, W2Q_ID, W13S_ID, W2S_ID = 6, 7, 8, 9
 
 
 @dataclasses.dataclass(frozen=True)
@@ -128,6 +129,39 @@ def make_experts(cfg: MoEConfig, device="cpu", seed: int = 0):
         w2[e] = (torch.randn(cfg.d, cfg.f, generator=g2, device=device,
                              dtype=torch.float32) * s2).to(torch.bfloat16)
     return w13, w2
+
+
+# FP8 codes are drawn as N(0, FP8_CODE_STD^2), clamped to the largest E4M3
+# magnitude and cast to the nearest code, so they use most of E4M3's range.
+FP8_CODE_STD = 64.0
+FP8_MAX = 448.0
+
+
+def make_experts_fp8(cfg: MoEConfig, device="cpu", seed: int = 0):
+    """FP8 expert weights: (w13 codes (E, 2f, d) uint8, w13 row scales (E, 2f)
+    fp32, w2 codes (E, d, f) uint8, w2 row scales (E, d) fp32).
+
+    Codes are E4M3 bit patterns; each row scale is sigma / FP8_CODE_STD times
+    a U(0.5, 1.5) draw, sigma the bf16 weights' std (1/sqrt(d) for w13,
+    1/sqrt(f) for w2), so the weights have the bf16 weights' size and every
+    row a different scale.
+    """
+    def codes(rows, cols, g):
+        v = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32)
+        v = (v * FP8_CODE_STD).clamp_(-FP8_MAX, FP8_MAX)
+        return v.to(torch.float8_e4m3fn).view(torch.uint8)
+
+    w13 = torch.empty(cfg.E, 2 * cfg.f, cfg.d, device=device, dtype=torch.uint8)
+    w2 = torch.empty(cfg.E, cfg.d, cfg.f, device=device, dtype=torch.uint8)
+    g13, g2 = _gen(device, seed, W13Q_ID), _gen(device, seed, W2Q_ID)
+    for e in range(cfg.E):
+        w13[e] = codes(2 * cfg.f, cfg.d, g13)
+        w2[e] = codes(cfg.d, cfg.f, g2)
+    u13 = torch.rand(cfg.E, 2 * cfg.f, generator=_gen(device, seed, W13S_ID), device=device)
+    u2 = torch.rand(cfg.E, cfg.d, generator=_gen(device, seed, W2S_ID), device=device)
+    s13 = (u13 + 0.5) * (1.0 / (math.sqrt(cfg.d) * FP8_CODE_STD))
+    s2 = (u2 + 0.5) * (1.0 / (math.sqrt(cfg.f) * FP8_CODE_STD))
+    return w13, s13.float().contiguous(), w2, s2.float().contiguous()
 
 
 def make_layer(cfg: MoEConfig, device="cpu", seed: int = 0) -> dict:

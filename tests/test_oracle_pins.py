@@ -567,3 +567,123 @@ def test_planted_dedup_mistakes_are_caught(monkeypatch):
             except (AssertionError, ValueError, IndexError):
                 failures += 1
         assert failures > 0, bad.__name__
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) weights
+# (code, value) worked out by hand from the E4M3 bit layout: sign | 4 exponent
+# bits, bias 7 | 3 mantissa bits; exponent 0 holds the subnormals m/8 * 2^-6.
+E4M3_HAND = [(0x00, 0.0), (0x80, -0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9),
+             (0x08, 2.0 ** -6), (0x38, 1.0), (0x3C, 1.5), (0x40, 2.0), (0xB8, -1.0),
+             (0x77, 240.0), (0x78, 256.0), (0x7E, 448.0), (0xFE, -448.0)]
+
+
+def test_e4m3_decode_hand_values_and_library_cast():
+    got = oracle.e4m3_decode(np.array([c for c, _ in E4M3_HAND], dtype=np.uint8))
+    for (c, want), v in zip(E4M3_HAND, got):
+        assert v == want and math.copysign(1.0, v) == math.copysign(1.0, want), hex(c)
+    assert np.isnan(oracle.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_decode(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+
+
+def _fp8_case(seed=0, T=24, d=64, E=4, k=2, f=64):
+    """Tiny layer with E4M3 weights and power-of-two row scales (so the
+    dequantised weights are exact bf16 values)."""
+    rng = np.random.default_rng(seed)
+    cfg = wl.MoEConfig("fp8-tiny", T=T, d=d, E=E, k=k, f=f)
+    x = _np(wl.make_hidden(cfg, "cpu", seed))
+    w_g, bias = wl.make_router(cfg, "cpu", seed)
+    c13, _, c2, _ = wl.make_experts_fp8(cfg, "cpu", seed)
+    c13, c2 = c13.numpy(), c2.numpy()
+    s13 = np.ldexp(1.0, rng.integers(-10, -5, (E, 2 * f))).astype(np.float32)
+    s2 = np.ldexp(1.0, rng.integers(-10, -5, (E, d))).astype(np.float32)
+    return cfg, x, _np(w_g), _np(bias), c13, s13, c2, s2
+
+
+def _y_fp8(case, s13=None, s2=None):
+    cfg, x, w_g, b, c13, S13, c2, S2 = case
+    return oracle.moe_forward_fp8(x, w_g, b, c13, S13 if s13 is None else s13, c2,
+                                  S2 if s2 is None else s2, cfg.k, select_dtype=None)["y"]
+
+
+def test_fp8_layer_is_the_bf16_layer_on_library_dequantised_weights():
+    cfg, x, w_g, b, c13, s13, c2, s2 = case = _fp8_case()
+
+    def deq(c, s):  # torch's E4M3 cast, row scale broadcast over K, then bf16
+        w = torch.from_numpy(c).view(torch.float8_e4m3fn).float() * torch.from_numpy(s)[..., None]
+        w16 = w.to(torch.bfloat16)
+        assert torch.equal(w16.float(), w)  # power-of-two scales keep it exact
+        return _np(w16)
+
+    ref = oracle.moe_forward(x, w_g, b, deq(c13, s13), deq(c2, s2), cfg.k,
+                             select_dtype=None)["y"]
+    np.testing.assert_array_equal(_y_fp8(case), ref)
+
+
+def test_fp8_row_scales_act_on_output_rows():
+    cfg, x, w_g, b, c13, s13, c2, s2 = case = _fp8_case(seed=1)
+    y = _y_fp8(case)
+    # W_down row r produces output column r: doubling its scale in every
+    # expert doubles y[:, r] exactly and leaves the other columns alone.
+    r = 5
+    s2b = s2.copy()
+    s2b[:, r] *= 2
+    y2 = _y_fp8(case, s2=s2b)
+    np.testing.assert_array_equal(y2[:, r], 2 * y[:, r])
+    np.testing.assert_array_equal(np.delete(y2, r, 1), np.delete(y, r, 1))
+    # Up row j scales h_j linearly: y is affine in that scale.
+    j = 3
+    ys = []
+    for m in (1.0, 2.0, 3.0):
+        s = s13.copy()
+        s[:, cfg.f + j] *= m
+        ys.append(_y_fp8(case, s13=s))
+    np.testing.assert_allclose(ys[2] - ys[0], 2 * (ys[1] - ys[0]), rtol=0, atol=1e-12)
+    assert np.abs(ys[1] - ys[0]).max() > 1e-6
+    # Zeroing gate row j or up row j removes the same term h_j = silu(g_j) u_j.
+    zg, zu = s13.copy(), s13.copy()
+    zg[:, j] = 0
+    zu[:, cfg.f + j] = 0
+    np.testing.assert_allclose(_y_fp8(case, s13=zg), _y_fp8(case, s13=zu), rtol=0, atol=1e-12)
+
+
+def _fp8_pins_fail(monkeypatch, name, bad):
+    monkeypatch.setattr(oracle.fp8_oracle, name, bad)
+    monkeypatch.setattr(oracle, name, bad)
+    failures = 0
+    for fn in (test_e4m3_decode_hand_values_and_library_cast,
+               test_fp8_layer_is_the_bf16_layer_on_library_dequantised_weights,
+               test_fp8_row_scales_act_on_output_rows):
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            failures += 1
+    return failures
+
+
+def test_planted_fp8_mistakes_are_caught(monkeypatch):
+    good_decode = oracle.fp8_oracle.e4m3_decode
+
+    def bias8(codes):  # exponent bias 8 instead of 7
+        return good_decode(codes) / 2
+
+    def no_subnormals(codes):  # exponent field 0 read with an implicit leading 1
+        c = np.asarray(codes, dtype=np.uint8)
+        v = good_decode(c)
+        e0 = ((c >> 3) & 0xF) == 0
+        return np.where(e0, np.where(c >> 7, -1.0, 1.0) * np.ldexp(1 + (c & 7) / 8.0, -7), v)
+
+    def per_column(codes, scale):  # the scale applied along K instead of the rows
+        w = good_decode(codes)
+        s = np.asarray(scale, dtype=np.float64)
+        return w * np.resize(s, w.shape[-1])[None, :]
+
+    assert _fp8_pins_fail(monkeypatch, "e4m3_decode", bias8) > 0
+    monkeypatch.undo()
+    assert _fp8_pins_fail(monkeypatch, "e4m3_decode", no_subnormals) > 0
+    monkeypatch.undo()
+    assert _fp8_pins_fail(monkeypatch, "dequantise_rows", per_column) > 0
