@@ -8,7 +8,7 @@ tokens, d=2048, E=128 experts, top-8, f=768, Zipf(1.0) expert skew), the
 configuration the HBM-roofline metric is quoted on.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--T T]
+                  [--workload NAME] [--T T] [--fp8]
 
 Device timing: W untimed steps, then K steps each bracketed by CUDA events on
 the launch stream (stage boundaries come from moe_forward_staged); L2 is
@@ -87,6 +87,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="qwen3-30b-a3b-decode")
     p.add_argument("--T", type=int, default=None, help="override the token count")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--fp8", action="store_true",
+                   help="E4M3 expert weights with fp32 row scales (batches of up to 256)")
     p.add_argument("--eplb-redundant", type=int, default=0,
                    help="time the layer with this many redundant expert copies placed by "
                         "the EPLB-style plan (built from the counts of one warm-up call)")
@@ -103,9 +105,9 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(sources=None):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -118,7 +120,7 @@ def profiled_traffic(workload_key, kernel):
         with open(PROFILE_TRAFFIC) as fh:
             tab = json.load(fh)
         ent = tab[workload_key][kernel]
-        if ent.get("source_hash") != kernel_source_hash():
+        if ent.get("source_hash") != kernel_source_hash(ent.get("sources")):
             return None
         return float(ent["dram_bytes_per_launch"])
     except Exception:
@@ -335,17 +337,20 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ our arm
-def algorithmic(cfg, touched):
+def algorithmic(cfg, touched, fp8=False):
     """Algorithmic bytes and flops of one layer call: the touched experts'
-    weights, the router weight (+bias), x read and y written; flops of the
+    weights (2 bytes each in bf16; 1 byte each plus a 4-byte scale per row in
+    FP8), the router weight (+bias), x read and y written; flops of the
     expert FFN and router.  Intermediates (x_perm, h, z) are not counted."""
-    wbytes = touched * 3 * cfg.d * cfg.f * 2
+    wb = 1 if fp8 else 2
+    sb = 4 if fp8 else 0
+    g1 = touched * (2 * cfg.f * cfg.d * wb + 2 * cfg.f * sb)
+    g2 = touched * (cfg.f * cfg.d * wb + cfg.d * sb)
     router = cfg.d * cfg.E * 4 + (cfg.E * 4 if cfg.zipf_s is not None else 0)
     act = cfg.T * cfg.d * 2 * 2
     flops = 6 * cfg.P * cfg.d * cfg.f + 2 * cfg.T * cfg.d * cfg.E
-    return {"bytes": wbytes + router + act, "flops": flops,
-            "gemm1_bytes": touched * 2 * cfg.f * cfg.d * 2,
-            "gemm2_bytes": touched * cfg.f * cfg.d * 2,
+    return {"bytes": g1 + g2 + router + act, "flops": flops,
+            "gemm1_bytes": g1, "gemm2_bytes": g2,
             "gemm1_flops": 4 * cfg.P * cfg.d * cfg.f, "gemm2_flops": 2 * cfg.P * cfg.d * cfg.f}
 
 
@@ -367,9 +372,15 @@ def run_ours(args):
 
     # Same weights on every rank (replicas), a different batch per rank.
     w_g, bias = wl.make_router(cfg, dev, 0)
-    w13, w2 = wl.make_experts(cfg, dev, 0)
     x = wl.make_hidden(cfg, dev, rank)
-    layer = moe.MoELayer(w_g, bias, w13, w2, cfg.k, cfg.R)
+    if args.fp8:
+        if cfg.T > 256 or args.eplb_redundant:
+            raise SystemExit("--fp8 runs batches of up to 256 tokens, without --eplb-redundant")
+        w13, s13, w2, s2 = wl.make_experts_fp8(cfg, dev, 0)
+    else:
+        w13, w2 = wl.make_experts(cfg, dev, 0)
+        s13 = s2 = None
+    layer = moe.MoELayer(w_g, bias, w13, w2, cfg.k, cfg.R, w13_scale=s13, w2_scale=s2)
     shape = layer.shape(cfg.T)
     ws = moe.workspace(shape, dev)
     y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
@@ -390,7 +401,20 @@ def run_ours(args):
     # dominant kernel's launch time.  The extra event nodes cost a few
     # microseconds each, so pass-2 stage times are upper bounds.
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws)
+
+    def fwd(out, **kw):  # the layer through the C ABI (bf16 or FP8 experts)
+        if args.fp8:
+            moe.moe_forward_fp8(x, w_g, bias, w13, s13, w2, s2, out, shape, ws, **kw)
+        else:
+            moe.moe_forward(x, w_g, bias, w13, w2, out, shape, ws, **kw)
+
+    def fwd_staged(events):
+        if args.fp8:
+            moe.moe_forward_fp8_staged(x, w_g, bias, w13, s13, w2, s2, y, shape, ws, events)
+        else:
+            moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, events)
+
+    fwd(y)
     torch.cuda.synchronize(dev)
 
     eplb_info = None
@@ -418,9 +442,9 @@ def run_ours(args):
             if events is None and eplb_info is not None:
                 layer(x, out=y)
             elif events is None:
-                moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws)
+                fwd(y)
             else:
-                moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, events)
+                fwd_staged(events)
         return g
 
     plain = capture()
@@ -504,7 +528,7 @@ def run_ours(args):
     dedup_info = None
     if cfg.R > 1:
         idx_d = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
-        moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, idx_out=idx_d)
+        fwd(y, idx_out=idx_d)
         P = cfg.T * cfg.k
         rows_max = cfg.T * min(cfg.k, cfg.R)
         i32 = lambda n: torch.empty(n, dtype=torch.int32, device=dev)
@@ -549,9 +573,9 @@ def run_ours(args):
     # touched logical experts: the algorithmic bytes count each expert's
     # weights once even when replicas stream copies of them
     counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
-    moe.moe_forward(x, w_g, bias, w13, w2, y_dev, shape, ws, counts_out=counts)
+    fwd(y_dev, counts_out=counts)
     touched = int((counts > 0).sum().item())
-    alg = algorithmic(cfg, touched)
+    alg = algorithmic(cfg, touched, args.fp8)
     mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
     names = ["router", "topk_dispatch_gather", "gemm1_swiglu", "gemm2", "combine"]
     dom = max(range(len(mean_stage)), key=lambda j: mean_stage[j])
@@ -572,7 +596,8 @@ def run_ours(args):
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
     roof["kernel"] = kern
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-    roof["traffic"] = profiled_traffic(f"{cfg.name}@T{cfg.T}", kern)
+    roof["traffic"] = profiled_traffic(f"{cfg.name}@T{cfg.T}" + ("/fp8" if args.fp8 else ""),
+                                       kern)
     t_layer = ms_per_step / 1e3
     layer_roof = {
         "bytes": alg["bytes"], "flops": alg["flops"], "touched_experts": touched,
@@ -604,6 +629,9 @@ def run_ours(args):
         "gpu_launches": 2 * launches_per_forward(cfg) * args.steps,
         "clocks": clk,
     }
+    if args.fp8:
+        line["config"]["weights"] = "e4m3 codes, one fp32 scale per weight row"
+        line["dtype"] = "bf16 (tensor-core operands; expert weights stored e4m3)"
     if dedup_info is not None:
         line["dispatch_volume"] = dedup_info
     if eplb_info is not None:
@@ -612,7 +640,7 @@ def run_ours(args):
         line["stage_ms_note"] += "; with --eplb-redundant the stages are the plain layer's"
         line["gpu_launches"] = (launches_per_forward(cfg, args.eplb_redundant) +
                                 launches_per_forward(cfg)) * args.steps
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
         line["cpu_baseline"] = cpu_baseline(cfg, {"x": x, "w_g": w_g, "bias": bias,
                                                   "w13": w13, "w2": w2})
     if rank == 0:

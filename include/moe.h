@@ -77,7 +77,7 @@ typedef enum moe_status {
 MOE_API const char* moe_error_string(int status);
 
 /* Library ABI version (major * 100 + minor): 101 adds the EPLB calls and
- * moe_dispatch_dedup. */
+ * moe_dispatch_dedup; 102 the FP8-weight calls. */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -314,6 +314,40 @@ MOE_API int moe_forward_eplb(const moe_bf16* x, const float* w_g, const float* b
                              const int32_t* rep_phys, int32_t E_phys, moe_bf16* y,
                              int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
                              void* stream);
+
+/* FP8 expert weights ("Serving mixture-of-experts models: expert parallelism
+ * on H200", sections "Memory math for 8xH200" and "Quantization choices":
+ * native FP8 checkpoints store one byte per weight; the small-batch expert
+ * GEMMs are bound by reading them).  The pages fix no encoding; this library
+ * takes OCP FP8 E4M3 codes (bias 7, subnormals at exponent 0, S.1111.111 is
+ * NaN, no infinities) with one fp32 scale per weight row:
+ *   w13   [E, 2f, d] uint8 in   E4M3 codes, rows as moe_ffn's w13
+ *   w13_scale [E, 2f] fp32 in   W13[e, r, c] = e4m3(w13[e, r, c]) * w13_scale[e, r]
+ *   w2    [E, d, f] uint8 in    E4M3 codes, rows as moe_ffn's w2
+ *   w2_scale  [E, d] fp32 in    W2[e, r, c] = e4m3(w2[e, r, c]) * w2_scale[e, r]
+ * Activations, accumulation and rounding points are those of the bf16 calls:
+ * the result is moe_ffn / moe_forward on the dequantised weights (each row
+ * scale multiplies the fp32 accumulator before SwiGLU / the bf16 store).
+ * Code pointers 16-byte aligned, scales 4-byte aligned.  Supported for
+ * s->T <= 256 (the regime where the weights, not the tensor cores, bound the
+ * GEMMs); larger batches return MOE_ERR_UNSUPPORTED before any launch. */
+MOE_API int moe_ffn_fp8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w13,
+                        const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                        const moe_shape* s, moe_bf16* z, void* ws, void* stream);
+
+/* The whole layer (as moe_forward) with FP8 expert weights (as moe_ffn_fp8). */
+MOE_API int moe_forward_fp8(const moe_bf16* x, const float* w_g, const float* bias,
+                            const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
+                            const float* w2_scale, const moe_shape* s, moe_bf16* y,
+                            int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
+                            void* stream);
+
+/* moe_forward_fp8 with the stage events of moe_forward_staged. */
+MOE_API int moe_forward_fp8_staged(const moe_bf16* x, const float* w_g, const float* bias,
+                                   const uint8_t* w13, const float* w13_scale,
+                                   const uint8_t* w2, const float* w2_scale,
+                                   const moe_shape* s, moe_bf16* y, void* ws,
+                                   void* const* events, void* stream);
 
 /* Self-test of the failure path every device-side wait uses: launches one
  * kernel that waits on a barrier nothing will ever complete, through the same

@@ -14,5 +14,6 @@ from .binding import (EXPORTS, MOE_STAGE_EVENTS, STAGE_NAMES, MOE_ERR_CUDA, MOE_
                       moe_topk, moe_version,
                       moe_workspace_size, workspace, moe_eplb_plan, moe_eplb_remap,
                       moe_workspace_size_eplb, workspace_eplb, moe_forward_eplb,
-                      moe_dispatch_dedup)
+                      moe_dispatch_dedup, moe_ffn_fp8, moe_forward_fp8,
+                      moe_forward_fp8_staged)
 from .layer import MoELayer  # noqa: F401

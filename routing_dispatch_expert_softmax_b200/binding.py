@@ -30,7 +30,8 @@ EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router"
            "moe_topk", "moe_dispatch", "moe_ffn", "moe_combine", "moe_forward",
            "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check",
            "moe_dispatch_noalloc", "moe_eplb_plan", "moe_eplb_remap",
-           "moe_workspace_size_eplb", "moe_forward_eplb", "moe_dispatch_dedup")
+           "moe_workspace_size_eplb", "moe_forward_eplb", "moe_dispatch_dedup",
+           "moe_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_staged")
 
 
 class MoEError(RuntimeError):
@@ -105,6 +106,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_forward_eplb.restype = ctypes.c_int
     lib.moe_forward_eplb.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _i32, _P, _P, _P, _P,
                                      _P, _P]
+    lib.moe_ffn_fp8.restype = ctypes.c_int
+    lib.moe_ffn_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _S, _P, _P, _P]
+    lib.moe_forward_fp8.restype = ctypes.c_int
+    lib.moe_forward_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P]
+    lib.moe_forward_fp8_staged.restype = ctypes.c_int
+    lib.moe_forward_fp8_staged.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]
     _lib = lib
     return lib
 
@@ -296,12 +303,9 @@ def _event_handle(ev) -> int:
         return 0
 
 
-def moe_forward_staged(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, events, stream=None):
-    """``events``: MOE_STAGE_EVENTS torch.cuda.Event objects (or None entries)
-    recorded at the stage boundaries on the launch stream."""
+def _event_array(events, st):
     if len(events) != MOE_STAGE_EVENTS:
         raise ValueError(f"need {MOE_STAGE_EVENTS} events")
-    st = torch.cuda.current_stream() if stream is None else stream
     handles = []
     for ev in events:
         if ev is None:
@@ -310,12 +314,57 @@ def moe_forward_staged(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, events, st
         if not _event_handle(ev):
             ev.record(st)  # torch creates the CUDA event at its first record
         handles.append(ctypes.c_void_p(_event_handle(ev)))
-    arr = (ctypes.c_void_p * MOE_STAGE_EVENTS)(*handles)
+    return (ctypes.c_void_p * MOE_STAGE_EVENTS)(*handles)
+
+
+def moe_forward_staged(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, events, stream=None):
+    """``events``: MOE_STAGE_EVENTS torch.cuda.Event objects (or None entries)
+    recorded at the stage boundaries on the launch stream."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    arr = _event_array(events, st)
     _check(load_library().moe_forward_staged(
         _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
         _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.bfloat16, "w13"),
         _ptr(w2, torch.bfloat16, "w2"), ctypes.byref(shape), _ptr(y, torch.bfloat16, "y"),
         _ptr(ws, torch.uint8, "ws"), arr, _stream(st)), "moe_forward_staged")
+
+
+def moe_ffn_fp8(x_perm, offsets, w13, w13_scale, w2, w2_scale, z, shape: MoEShape, ws,
+                stream=None):
+    """Expert FFNs with E4M3 expert weights (uint8 codes) and fp32 row scales."""
+    _check(load_library().moe_ffn_fp8(
+        _ptr(x_perm, torch.bfloat16, "x_perm"), _ptr(offsets, torch.int32, "offsets"),
+        _ptr(w13, torch.uint8, "w13"), _ptr(w13_scale, torch.float32, "w13_scale"),
+        _ptr(w2, torch.uint8, "w2"), _ptr(w2_scale, torch.float32, "w2_scale"),
+        ctypes.byref(shape), _ptr(z, torch.bfloat16, "z"), _ptr(ws, torch.uint8, "ws"),
+        _stream(stream)), "moe_ffn_fp8")
+
+
+def moe_forward_fp8(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoEShape, ws,
+                    idx_out=None, w_out=None, counts_out=None, stream=None):
+    """The whole layer with E4M3 expert weights and fp32 row scales."""
+    _check(load_library().moe_forward_fp8(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.uint8, "w13"),
+        _ptr(w13_scale, torch.float32, "w13_scale"), _ptr(w2, torch.uint8, "w2"),
+        _ptr(w2_scale, torch.float32, "w2_scale"), ctypes.byref(shape),
+        _ptr(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
+        _ptr(w_out, torch.float32, "w_out"), _ptr(counts_out, torch.int32, "counts_out"),
+        _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_forward_fp8")
+
+
+def moe_forward_fp8_staged(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoEShape, ws,
+                           events, stream=None):
+    """moe_forward_fp8 with the stage events of moe_forward_staged."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    arr = _event_array(events, st)
+    _check(load_library().moe_forward_fp8_staged(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.uint8, "w13"),
+        _ptr(w13_scale, torch.float32, "w13_scale"), _ptr(w2, torch.uint8, "w2"),
+        _ptr(w2_scale, torch.float32, "w2_scale"), ctypes.byref(shape),
+        _ptr(y, torch.bfloat16, "y"), _ptr(ws, torch.uint8, "ws"), arr, _stream(st)),
+        "moe_forward_fp8_staged")
 
 
 def moe_selftest_bounded_wait(limit_ns: int, ws, stream=None):

@@ -9,7 +9,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kVersion = 101;
+constexpr int kVersion = 102;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
@@ -191,16 +191,20 @@ int moe_combine(const moe_bf16* z, const int32_t* row_of, const float* w, const 
                                     static_cast<cudaStream_t>(stream)));
 }
 
-static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
-                        const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
-                        moe_bf16* y, int32_t* idx_out, float* w_out, int32_t* counts_out,
-                        void* ws, void* stream, void* const* events) {
+// The whole layer: bf16 expert weights, or (fp8) E4M3 expert weights with one
+// fp32 scale per weight row (small batches only).
+static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const float* bias,
+                        const void* w13, const float* w13_scale, const void* w2,
+                        const float* w2_scale, const moe_shape* s, moe_bf16* y,
+                        int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
+                        void* stream, void* const* events) {
   if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  if (fp8 && s->T > kSwapMaxT) return MOE_ERR_UNSUPPORTED;
   if (s->T == 0) return MOE_OK;
   if (!ok16(x) || !ok4(w_g) || (bias && !aligned(bias, 4)) || !ok16(w13) || !ok16(w2) ||
       !ok16(y) || (idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4)) ||
-      (counts_out && !aligned(counts_out, 4)))
+      (counts_out && !aligned(counts_out, 4)) || (fp8 && (!ok4(w13_scale) || !ok4(w2_scale))))
     return MOE_ERR_INVALID_ARG;
   int sms = 0;
   int st = device_check(&sms);
@@ -243,9 +247,12 @@ static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
     e = launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
   if (e == cudaSuccess) e = mark(2);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  int r = launch_expert_ffn(x_perm, L.Ppad, reinterpret_cast<const __nv_bfloat16*>(w13),
-                            reinterpret_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms,
-                            cs, events ? events + 3 : nullptr);
+  int r = fp8 ? launch_expert_ffn_fp8(x_perm, L.Ppad, static_cast<const uint8_t*>(w13),
+                                       w13_scale, static_cast<const uint8_t*>(w2), w2_scale,
+                                       *s, L, wsb, z, sms, cs, events ? events + 3 : nullptr)
+              : launch_expert_ffn(x_perm, L.Ppad, static_cast<const __nv_bfloat16*>(w13),
+                                  static_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms,
+                                  cs, events ? events + 3 : nullptr);
   if (r != MOE_OK) return r;
   e = launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs);
   if (e == cudaSuccess) e = mark(5);
@@ -255,15 +262,53 @@ static int forward_impl(const moe_bf16* x, const float* w_g, const float* bias,
 int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const moe_bf16* w13,
                 const moe_bf16* w2, const moe_shape* s, moe_bf16* y, int32_t* idx_out,
                 float* w_out, int32_t* counts_out, void* ws, void* stream) {
-  return forward_impl(x, w_g, bias, w13, w2, s, y, idx_out, w_out, counts_out, ws, stream,
-                      nullptr);
+  return forward_impl(false, x, w_g, bias, w13, nullptr, w2, nullptr, s, y, idx_out, w_out,
+                      counts_out, ws, stream, nullptr);
 }
 
 int moe_forward_staged(const moe_bf16* x, const float* w_g, const float* bias,
                        const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
                        moe_bf16* y, void* ws, void* const* events, void* stream) {
-  return forward_impl(x, w_g, bias, w13, w2, s, y, nullptr, nullptr, nullptr, ws, stream,
-                      events);
+  return forward_impl(false, x, w_g, bias, w13, nullptr, w2, nullptr, s, y, nullptr, nullptr,
+                      nullptr, ws, stream, events);
+}
+
+int moe_ffn_fp8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w13,
+                const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                const moe_shape* s, moe_bf16* z, void* ws, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (s->T > kSwapMaxT) return MOE_ERR_UNSUPPORTED;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(x_perm) || !ok4(offsets) || !ok16(w13) || !ok4(w13_scale) || !ok16(w2) ||
+      !ok4(w2_scale) || !ok16(z) || !ws || !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*s, sms);
+  cudaError_t e = launch_tiles_from_offsets(offsets, *s, at<int>(ws, L.tiles),
+                                            at<int>(ws, L.err), cs);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_expert_ffn_fp8(reinterpret_cast<const __nv_bfloat16*>(x_perm), L.P, w13,
+                               w13_scale, w2, w2_scale, *s, L, static_cast<char*>(ws),
+                               reinterpret_cast<__nv_bfloat16*>(z), sms, cs);
+}
+
+int moe_forward_fp8(const moe_bf16* x, const float* w_g, const float* bias, const uint8_t* w13,
+                    const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                    const moe_shape* s, moe_bf16* y, int32_t* idx_out, float* w_out,
+                    int32_t* counts_out, void* ws, void* stream) {
+  return forward_impl(true, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, idx_out, w_out,
+                      counts_out, ws, stream, nullptr);
+}
+
+int moe_forward_fp8_staged(const moe_bf16* x, const float* w_g, const float* bias,
+                           const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
+                           const float* w2_scale, const moe_shape* s, moe_bf16* y, void* ws,
+                           void* const* events, void* stream) {
+  return forward_impl(true, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, nullptr, nullptr,
+                      nullptr, ws, stream, events);
 }
 
 size_t moe_workspace_size_eplb(const moe_shape* s, int32_t E_phys) {

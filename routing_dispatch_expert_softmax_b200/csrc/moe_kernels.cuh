@@ -38,6 +38,13 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       __nv_bfloat16* z, int num_sms, cudaStream_t st,
                       void* const* events = nullptr);
 
+// The same two GEMMs with E4M3 expert weights and one fp32 scale per weight
+// row (moe_gemm_fp8.cu); small batches (T <= kSwapMaxT) only.
+int launch_expert_ffn_fp8(const __nv_bfloat16* x_perm, long long x_rows, const uint8_t* w13,
+                          const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                          const moe_shape& s, const WsLayout& L, char* ws, __nv_bfloat16* z,
+                          int num_sms, cudaStream_t st, void* const* events = nullptr);
+
 // Logical -> physical expert ids of a replica plan (moe_eplb.cu).
 cudaError_t launch_eplb_remap(const int* idx, int T, int k, int E, const int* rep_offsets,
                               const int* rep_phys, int P, int* idx_phys, int* err,

@@ -38,12 +38,22 @@ class _Graphed:
 class MoELayer:
     """Routed MoE layer: router W_g (d, E) fp32 [+ bias (E,)], experts w13
     (E, 2f, d) bf16 (gate rows then up rows) and w2 (E, d, f) bf16, top-k.
-    ``R`` > 1 also computes the virtual expert-parallel layout."""
+    ``R`` > 1 also computes the virtual expert-parallel layout.
+
+    FP8 experts: pass w13 / w2 as uint8 E4M3 codes of the same shapes with
+    ``w13_scale`` (E, 2f) and ``w2_scale`` (E, d) fp32 row scales; the layer
+    then runs moe_forward_fp8 (batches of up to 256 tokens)."""
 
     def __init__(self, w_g: torch.Tensor, bias: Optional[torch.Tensor],
-                 w13: torch.Tensor, w2: torch.Tensor, k: int, R: int = 0):
+                 w13: torch.Tensor, w2: torch.Tensor, k: int, R: int = 0,
+                 w13_scale: Optional[torch.Tensor] = None,
+                 w2_scale: Optional[torch.Tensor] = None):
         B.load_library()
+        if (w13_scale is None) != (w2_scale is None):
+            raise ValueError("FP8 experts need both w13_scale and w2_scale")
         self.w_g, self.bias, self.w13, self.w2 = w_g, bias, w13, w2
+        self.w13_scale, self.w2_scale = w13_scale, w2_scale
+        self.fp8 = w13_scale is not None
         self.d, self.E = int(w_g.shape[0]), int(w_g.shape[1])
         self.f = int(w2.shape[2])
         self.k, self.R = int(k), int(R)
@@ -67,7 +77,11 @@ class MoELayer:
 
     def _call(self, x, y, ws, idx_out=None, w_out=None, counts_out=None, stream=None):
         shape = self.shape(int(x.shape[0]))
-        if self._eplb is None:
+        if self.fp8:
+            B.moe_forward_fp8(x, self.w_g, self.bias, self.w13, self.w13_scale, self.w2,
+                              self.w2_scale, y, shape, ws, idx_out=idx_out, w_out=w_out,
+                              counts_out=counts_out, stream=stream)
+        elif self._eplb is None:
             B.moe_forward(x, self.w_g, self.bias, self.w13, self.w2, y, shape, ws,
                           idx_out=idx_out, w_out=w_out, counts_out=counts_out, stream=stream)
         else:
@@ -84,6 +98,8 @@ class MoELayer:
         moe_forward_eplb, whose ``counts_out`` then has E + n_redundant
         entries (rows per physical expert).  Returns the plan
         (phys_to_logical, rep_offsets, rep_phys) as CPU int32 tensors."""
+        if self.fp8:
+            raise NotImplementedError("replica plans run on bf16 experts only")
         dev = self.w13.device
         p2l, off, phys = B.moe_eplb_plan(load, self.E, max(self.R, 1), n_redundant)
         sel = p2l.long().to(dev)

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_error_strings(lib):
-    assert moe.moe_version() == 101
+    assert moe.moe_version() == 102
     for code in range(6):
         assert moe.moe_error_string(code).startswith("MOE_")
     assert "unknown" in moe.moe_error_string(99)
@@ -130,6 +130,31 @@ def test_bad_arguments_are_rejected_before_launch(lib):
                 _P(A16), None, None, None, _P(A16), None) == INV
 
 
+def test_fp8_calls_reject_before_launch(lib):
+    s = ctypes.byref(B.MoEShape.of(**VALID))
+    big = ctypes.byref(B.MoEShape.of(**dict(VALID, T=257)))
+    INV, UNS = B.MOE_ERR_INVALID_ARG, B.MOE_ERR_UNSUPPORTED
+    ws = _P(A16)
+    # moe_ffn_fp8(x_perm, offsets, w13, w13_scale, w2, w2_scale, s, z, ws, stream)
+    assert _raw(lib, "moe_ffn_fp8", *[_P(A16)] * 6, big, _P(A16), ws, None) == UNS
+    assert _raw(lib, "moe_ffn_fp8", _P(A16), _P(A16), _P(A16), None, _P(A16), _P(A16), s,
+                _P(A16), ws, None) == INV                       # null w13 scales
+    assert _raw(lib, "moe_ffn_fp8", _P(A16), _P(A16), _P(A16 + 8), _P(A16), _P(A16), _P(A16),
+                s, _P(A16), ws, None) == INV                    # codes not 16-byte aligned
+    assert _raw(lib, "moe_ffn_fp8", _P(A16), _P(A16), _P(A16), _P(A16), _P(A16), _P(A16 + 2),
+                s, _P(A16), ws, None) == INV                    # misaligned w2 scales
+    # moe_forward_fp8(x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, idx, w, counts, ws, st)
+    fwd = [_P(A16), _P(A16), None, _P(A16), _P(A16), _P(A16), _P(A16)]
+    assert _raw(lib, "moe_forward_fp8", *fwd, big, _P(A16), None, None, None, ws, None) == UNS
+    assert _raw(lib, "moe_forward_fp8", *fwd[:6], None, s, _P(A16), None, None, None, ws,
+                None) == INV                                    # null w2 scales
+    assert _raw(lib, "moe_forward_fp8", *fwd, s, _P(A16), None, None, None, None, None) == INV
+    s0 = ctypes.byref(B.MoEShape.of(**dict(VALID, T=0)))
+    assert _raw(lib, "moe_forward_fp8", *[None] * 7, s0, None, None, None, None, ws,
+                None) == B.MOE_OK
+    assert _raw(lib, "moe_forward_fp8_staged", *fwd, big, _P(A16), ws, None, None) == UNS
+
+
 def test_empty_batch_is_a_no_op(lib):
     s0 = ctypes.byref(B.MoEShape.of(**dict(VALID, T=0)))
     # T = 0 launches nothing, so even null activation pointers are accepted.
@@ -147,6 +172,8 @@ def test_no_cpu_fallback_without_a_gpu(lib):
     assert _raw(lib, "moe_topk", _P(A16), s, _P(A16), _P(A16), None) == B.MOE_ERR_CUDA
     assert _raw(lib, "moe_forward", *[_P(A16)] * 5, s, _P(A16), None, None, None, _P(A16),
                 None) == B.MOE_ERR_CUDA
+    assert _raw(lib, "moe_forward_fp8", *[_P(A16)] * 7, s, _P(A16), None, None, None,
+                _P(A16), None) == B.MOE_ERR_CUDA
 
 
 def test_binding_refuses_cpu_tensors(lib):
