@@ -35,8 +35,10 @@ namespace {
 
 template <int NMAX, bool SWIGLU>
 struct F8Cfg {
-  // Raw e4m3 weight tiles in flight (8 KB each): as many weight bytes as the
-  // bf16 kernel keeps in flight, in half the shared memory per byte of K.
+  // Raw e4m3 weight tiles in flight (8 KB each: 96 / 80 KB, near the 112 KB of
+  // weights the bf16 kernel keeps in flight).  The token tile of a stage is
+  // loaded only once its MMA stage is free, so at most kMmaStages token loads
+  // are in flight.
   static constexpr int kRawStages = NMAX <= 64 ? 12 : 10;
   static constexpr int kMmaStages = 3;
   static constexpr int kRawBytes = 128 * kGemmBK;         // 8 KB of e4m3
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
       const int n = item_rows(i);
       const int e = et[3 * i + 2];
       if (n < 1 || n > NMAX) {
-        if (threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
+        if (threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 15);
         --it;
         continue;
       }
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x == 0 && *abort_flag) record_error(err, MOE_ERR_TIMEOUT, 13);
+  if (threadIdx.x == 0 && *abort_flag) record_error(err, MOE_ERR_TIMEOUT, 14);
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
