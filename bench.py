@@ -354,6 +354,23 @@ def algorithmic(cfg, touched, fp8=False):
             "gemm1_flops": 4 * cfg.P * cfg.d * cfg.f, "gemm2_flops": 2 * cfg.P * cfg.d * cfg.f}
 
 
+def routing_stats(counts, R):
+    """Load of one layer call ("Serving MoE models with expert parallelism on
+    8xH200", section "Routing imbalance"): rows per expert (max, mean over the
+    E experts, touched experts) and, with R > 1 virtual ranks, rows per rank
+    and the busiest-rank / mean ratio (the imbalance factor)."""
+    c = [int(v) for v in counts]
+    E, P = len(c), sum(c)
+    out = {"rows": P, "touched_experts": sum(1 for v in c if v > 0),
+           "max_rows_per_expert": max(c) if c else 0,
+           "mean_rows_per_expert": P / E if E else 0.0}
+    if R > 1:
+        per = [sum(c[r * E // R:(r + 1) * E // R]) for r in range(R)]
+        out["rows_per_rank"] = per
+        out["imbalance_factor"] = max(per) / (P / R) if P else 0.0
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -574,7 +591,8 @@ def run_ours(args):
     # weights once even when replicas stream copies of them
     counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
     fwd(y_dev, counts_out=counts)
-    touched = int((counts > 0).sum().item())
+    counts_h = counts.cpu().tolist()
+    touched = sum(1 for v in counts_h if v > 0)
     alg = algorithmic(cfg, touched, args.fp8)
     mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
     names = ["router", "topk_dispatch_gather", "gemm1_swiglu", "gemm2", "combine"]
@@ -621,6 +639,7 @@ def run_ours(args):
                              "stage events, then a second pass with them"},
         "roofline": roof,
         "layer_roofline": layer_roof,
+        "routing": routing_stats(counts_h, cfg.R),
         "stage_ms": dict(zip(names, mean_stage)),
         "stage_ms_note": "from the second timed pass with event nodes at every kernel boundary "
                          "(each adds a few us); the headline uses plain graph replays",

@@ -94,3 +94,27 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert rc0 == 0 and rc1 == 0
     assert '"impl": "reference"' in out0
     assert out1.strip() == ""
+
+
+def test_routing_stats_against_the_oracle_imbalance_factor():
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    import oracle
+    rng = np.random.default_rng(0)
+    for E, R in ((8, 4), (256, 8), (128, 0), (6, 1)):
+        counts = torch.from_numpy(rng.integers(0, 50, E).astype(np.int32))
+        st = bench.routing_stats(counts.tolist(), R)
+        c = counts.numpy()
+        assert st["rows"] == int(c.sum())
+        assert st["touched_experts"] == int((c > 0).sum())
+        assert st["max_rows_per_expert"] == int(c.max())
+        assert st["mean_rows_per_expert"] == c.sum() / E
+        if R > 1:
+            assert st["rows_per_rank"] == c.reshape(R, -1).sum(1).tolist()
+            assert st["imbalance_factor"] == oracle.imbalance_factor(c, R)
+        else:
+            assert "imbalance_factor" not in st
+    assert bench.routing_stats([0, 0, 0, 0], 2)["imbalance_factor"] == 0.0
