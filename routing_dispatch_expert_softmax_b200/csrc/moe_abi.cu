@@ -82,7 +82,9 @@ const char* moe_error_string(int status) {
   switch (status) {
     case MOE_OK: return "MOE_OK";
     case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null or misaligned pointer, or shape out of range";
-    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: the current device is not an sm_100 GPU";
+    case MOE_ERR_UNSUPPORTED:
+      return "MOE_ERR_UNSUPPORTED: the current device is not an sm_100 GPU, or the shape is "
+             "outside what this call runs (see the call's notes in moe.h)";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed or no CUDA device is usable";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait ran out";
     case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a device-side consistency check failed";
