@@ -245,8 +245,12 @@ def cpu_threads():
 
 
 def oracle_sample_run(cfg, host, tokens):
-    """One oracle pass over the given tokens of the batch (fp64, CPU)."""
+    """One oracle pass over the given tokens of the batch (fp64, CPU); FP8
+    experts are dequantised by the oracle inside the pass."""
     import oracle
+    if "w13_scale" in host:
+        return oracle.moe_forward_fp8(host["x"][tokens], host["w_g"], host["bias"], host["w13"],
+                                      host["w13_scale"], host["w2"], host["w2_scale"], cfg.k)
     return oracle.moe_forward(host["x"][tokens], host["w_g"], host["bias"], host["w13"],
                               host["w2"], cfg.k)
 
@@ -267,11 +271,15 @@ def host_inputs_for_oracle(cfg, dev_inputs, tokens):
     class Experts(dict):
         pass
 
-    w13, w2 = Experts(), Experts()
-    for e in touched.tolist():
-        w13[e] = f32(dev_inputs["w13"][e])
-        w2[e] = f32(dev_inputs["w2"][e])
-    return {"x": x, "w_g": w_g, "bias": bias, "w13": w13, "w2": w2}
+    fp8 = "w13_scale" in dev_inputs
+    raw = (lambda t: t.cpu().numpy()) if fp8 else f32  # FP8: codes and scales as stored
+    names = ("w13", "w2", "w13_scale", "w2_scale") if fp8 else ("w13", "w2")
+    host = {"x": x, "w_g": w_g, "bias": bias}
+    for name in names:
+        host[name] = Experts()
+        for e in touched.tolist():
+            host[name][e] = raw(dev_inputs[name][e])
+    return host
 
 
 def cpu_baseline(cfg, dev_inputs, budget_s=12.0):
@@ -306,7 +314,13 @@ def run_reference(args):
     from routing_dispatch_expert_softmax_b200 import workloads as wl
     cfg = workload_config(args.workload, args.T)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inputs = wl.make_layer(cfg, dev, 0)
+    w_g, bias = wl.make_router(cfg, dev, 0)
+    inputs = {"x": wl.make_hidden(cfg, dev, 0), "w_g": w_g, "bias": bias}
+    if args.fp8:
+        w13, s13, w2, s2 = wl.make_experts_fp8(cfg, dev, 0)
+        inputs.update(w13=w13, w13_scale=s13, w2=w2, w2_scale=s2)
+    else:
+        inputs["w13"], inputs["w2"] = wl.make_experts(cfg, dev, 0)
     n = min(cfg.T, 8)
     host = host_inputs_for_oracle(cfg, inputs, np.arange(cfg.T))
     del inputs
@@ -332,6 +346,8 @@ def run_reference(args):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+    if args.fp8:
+        line["config"]["weights"] = "e4m3 codes, one fp32 scale per weight row"
     print(json.dumps(line), flush=True)
     return 0
 
@@ -659,9 +675,11 @@ def run_ours(args):
         line["stage_ms_note"] += "; with --eplb-redundant the stages are the plain layer's"
         line["gpu_launches"] = (launches_per_forward(cfg, args.eplb_redundant) +
                                 launches_per_forward(cfg)) * args.steps
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
-        line["cpu_baseline"] = cpu_baseline(cfg, {"x": x, "w_g": w_g, "bias": bias,
-                                                  "w13": w13, "w2": w2})
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base_inputs = {"x": x, "w_g": w_g, "bias": bias, "w13": w13, "w2": w2}
+        if args.fp8:
+            base_inputs.update(w13_scale=s13, w2_scale=s2)
+        line["cpu_baseline"] = cpu_baseline(cfg, base_inputs)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

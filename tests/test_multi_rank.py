@@ -56,12 +56,12 @@ def _ref_worker(rank, world, port, out):
     sys.path.insert(0, ROOT)
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
                       MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    import argparse
     import contextlib
     import io
 
     import bench
-    args = argparse.Namespace(gpus=world, steps=1, warmup=1, workload="tiny", T=None)
+    args = bench.parse_args(["--gpus", str(world), "--steps", "1", "--warmup", "1",
+                             "--workload", "tiny"])
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         rc = bench.run_reference(args)
@@ -118,3 +118,21 @@ def test_routing_stats_against_the_oracle_imbalance_factor():
         else:
             assert "imbalance_factor" not in st
     assert bench.routing_stats([0, 0, 0, 0], 2)["imbalance_factor"] == 0.0
+
+
+@pytest.mark.parametrize("extra", [[], ["--fp8"]])
+def test_reference_arm_line_on_cpu(extra):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(k, None)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "0", *extra],
+                         capture_output=True, text=True, env=env, timeout=600, check=True).stdout
+    line = json.loads(out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert ("weights" in line["config"]) == bool(extra)
