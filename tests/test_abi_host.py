@@ -227,3 +227,34 @@ def test_eplb_workspace_size(lib):
     assert moe.moe_workspace_size_eplb(s, VALID["E"] + 8) >= moe.moe_workspace_size(s)
     assert moe.moe_workspace_size_eplb(s, VALID["E"] - 1) == 0
     assert moe.moe_workspace_size_eplb(s, 1025) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_plain_c_client_builds_links_and_runs(lib, tmp_path):
+    import shutil
+    import subprocess
+
+    import numpy as np
+
+    import oracle
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.dirname(B.LIB_PATH)
+    exe = str(tmp_path / "abi_from_c")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "abi_from_c.c"),
+                    "-L", pkg, "-l:" + os.path.basename(B.LIB_PATH), "-Wl,-rpath," + pkg,
+                    "-o", exe], check=True, capture_output=True, text=True)
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")  # no device: nothing may launch
+    out = subprocess.run([exe], check=True, capture_output=True, text=True, env=env,
+                         timeout=120).stdout
+    f = dict(kv.split("=", 1) for kv in out.split()[:6])
+    assert int(f["version"]) == moe.moe_version()
+    assert int(f["ws"]) == moe.moe_workspace_size(B.MoEShape.of(**VALID))
+    assert int(f["plan"]) == B.MOE_OK
+    p2l, _, _ = oracle.eplb_plan(np.array([9, 1, 1, 1, 1, 1, 1, 1]), 2, 2)  # (load, n_redundant, R)
+    assert int(f["p2l0"]) == int(p2l[0])
+    assert int(f["forward"]) == B.MOE_ERR_CUDA
+    assert int(f["bad"]) == B.MOE_ERR_INVALID_ARG
+    assert "MOE_ERR_CUDA" in out
