@@ -41,8 +41,11 @@ def e4m3_decode(codes):
 
 
 def dequantise_rows(codes, scale):
-    """W[..., r, c] = e4m3(codes[..., r, c]) * scale[..., r], fp64."""
-    return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[..., None]
+    """W[..., r, c] = e4m3(codes[..., r, c]) * scale[..., r], fp64.  The
+    codes are looked up in the decoded table of all 256 codes (the same
+    values as decoding each element, much faster on large matrices)."""
+    table = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return table[np.asarray(codes, dtype=np.uint8)] * np.asarray(scale, dtype=np.float64)[..., None]
 
 
 class LazyDequant:

@@ -588,6 +588,10 @@ def test_e4m3_decode_hand_values_and_library_cast():
     np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
     ok = ~np.isnan(ref)
     np.testing.assert_array_equal(got[ok], ref[ok])
+    # the table lookup in dequantise_rows gives the element-wise decode
+    rnd = np.random.default_rng(4).integers(0, 256, (7, 33), dtype=np.uint8)
+    np.testing.assert_array_equal(oracle.dequantise_rows(rnd, np.full(7, 2.0)),
+                                  2.0 * oracle.e4m3_decode(rnd))
 
 
 def _fp8_case(seed=0, T=24, d=64, E=4, k=2, f=64):
