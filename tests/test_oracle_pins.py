@@ -594,6 +594,21 @@ def test_e4m3_decode_hand_values_and_library_cast():
                                   2.0 * oracle.e4m3_decode(rnd))
 
 
+def test_fp8_single_expert_worked_by_hand():
+    # One expert (E = k = 1, gate weight 1), d = 2, f = 1, x = (1, 2).
+    # W13 codes: gate row (0x38, 0x40) = (1, 2) with scale 1/2; up row
+    # (0x3C, 0xB8) = (1.5, -1) with scale 2.  W2 codes: (0x40) = 2 with scale
+    # 1/4, (0x38) = 1 with scale 1.
+    #   g = (1*1 + 2*2) / 2 = 2.5,  u = 2 * (1.5 - 2) = -1,  h = silu(2.5) * u
+    #   y = (2/4 * h, 1 * h)
+    h = 2.5 / (1 + math.exp(-2.5)) * -1.0
+    c13 = np.array([[[0x38, 0x40], [0x3C, 0xB8]]], dtype=np.uint8)
+    c2 = np.array([[[0x40], [0x38]]], dtype=np.uint8)
+    out = oracle.moe_forward_fp8(np.array([[1.0, 2.0]]), np.zeros((2, 1)), None, c13,
+                                 np.array([[0.5, 2.0]]), c2, np.array([[0.25, 1.0]]), 1)
+    np.testing.assert_allclose(out["y"], [[0.5 * h, h]], rtol=1e-15, atol=0)
+
+
 def _fp8_case(seed=0, T=24, d=64, E=4, k=2, f=64):
     """Tiny layer with E4M3 weights and power-of-two row scales (so the
     dequantised weights are exact bf16 values)."""
@@ -660,6 +675,7 @@ def _fp8_pins_fail(monkeypatch, name, bad):
     monkeypatch.setattr(oracle, name, bad)
     failures = 0
     for fn in (test_e4m3_decode_hand_values_and_library_cast,
+               test_fp8_single_expert_worked_by_hand,
                test_fp8_layer_is_the_bf16_layer_on_library_dequantised_weights,
                test_fp8_row_scales_act_on_output_rows):
         try:
