@@ -208,8 +208,11 @@ MOE_API int moe_forward_staged(const moe_bf16* x, const float* w_g, const float*
  *     MOE_ERR_UNSUPPORTED before anything is launched (e.g. T = 16384,
  *     E = 256, R = 8 needs about 160 KB; T = 1<<20 with E = 256 does not fit).
  *   - The first call on a device looks up the array's device address with
- *     that device current (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture.
+ *     that device current (cudaGetSymbolAddress) and caches it for the life
+ *     of the process; make that first call before any stream capture.  A
+ *     cudaDeviceReset (or anything else that destroys the device's primary
+ *     context) invalidates the cached address: after one, unload and reload
+ *     the library before calling this entry point again.
  *   - Every call shares the one array and it keeps the last call's contents;
  *     the error word is cleared at the start of each call and the rest is
  *     rewritten.  Calls that overlap on the GPU (other streams, other threads)
@@ -251,10 +254,11 @@ MOE_API int moe_dispatch_dedup(const int32_t* idx, const moe_bf16* x, const moe_
 
 /* ---------------------------------------------------------------------------
  * Expert load balancing with replicated experts ("Serving MoE models with
- * expert parallelism on 8xH200", section "Routing imbalance": measure
- * per-expert load, place redundant copies of popular experts on less-loaded
- * GPUs, co-locate hot and cold experts; "vLLM Expert Parallel deployment",
- * EPLB section: load collected over a window, a number of redundant experts).
+ * expert parallelism on 8xH200", section "Routing imbalance": the busiest
+ * experts get extra copies on devices with spare capacity and busy and idle
+ * experts share devices; "vLLM Expert Parallel deployment", EPLB section:
+ * the load is taken over a window of steps, the number of extra copies is a
+ * setting).
  * The pages give no algorithm; these calls implement the plainest integer
  * reading (the oracle's tests/golden/eplb_worked_examples.json cases are
  * worked by hand from it):

@@ -6,9 +6,9 @@ CPU legs may use it; it shares nothing with the CUDA library.
 What the pages fix, and the reading taken where they are silent:
 
 * "Serving MoE models with expert parallelism on 8xH200", section "Routing
-  imbalance": measure per-expert load; replicate hot experts -- load
-  balancers place redundant copies of popular experts on less-loaded GPUs --
-  and re-shuffle placement so that hot and cold experts share GPUs.
+  imbalance": the per-expert load is measured, the busiest experts are given
+  extra copies on devices that have room, and placement is reshuffled so that
+  busy and idle experts share devices.
 * "vLLM Expert Parallel deployment" (EPLB section): the balancer collects
   load over a window and redistributes expert-to-rank mappings; the number of
   redundant experts is a parameter (num_redundant_experts).

@@ -15,17 +15,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
 bool ok4(const void* p) { return p != nullptr && aligned(p, 4); }
 
-bool shape_ok(const moe_shape* s) {
-  if (!s) return false;
-  if (s->T < 0 || s->T > (1 << 20)) return false;
-  if (s->d < 64 || s->d > 16384 || s->d % 64) return false;
-  if (s->E < 1 || s->E > kMaxE) return false;
-  if (s->k < 1 || s->k > kMaxK || s->k > s->E) return false;
-  if (s->f < 64 || s->f > 32768 || s->f % 64) return false;
-  if (s->R < 0 || s->R > kMaxR) return false;
-  if (s->R > 1 && s->E % s->R) return false;
-  return true;
-}
+bool shape_ok(const moe_shape* s) { return shape_valid(s); }
 
 // Current device: its SM count, and whether it is an sm_100 part.
 int device_check(int* num_sms) {

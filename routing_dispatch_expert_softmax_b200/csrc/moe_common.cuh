@@ -68,6 +68,19 @@ __device__ __forceinline__ void record_error(int* err, int code, int detail) {
   if (atomicCAS(err + kErrSlot, 0, code) == 0) err[kErrDetail] = detail;
 }
 
+// The shape limits every C-ABI entry point accepts (include/moe.h, moe_shape).
+inline bool shape_valid(const moe_shape* s) {
+  if (!s) return false;
+  if (s->T < 0 || s->T > (1 << 20)) return false;
+  if (s->d < 64 || s->d > 16384 || s->d % 64) return false;
+  if (s->E < 1 || s->E > kMaxE) return false;
+  if (s->k < 1 || s->k > kMaxK || s->k > s->E) return false;
+  if (s->f < 64 || s->f > 32768 || s->f % 64) return false;
+  if (s->R < 0 || s->R > kMaxR) return false;
+  if (s->R > 1 && s->E % s->R) return false;
+  return true;
+}
+
 // ----------------------------------------------------------------- workspace
 struct WsLayout {
   size_t err, w3, logit_part, logits, idx, idx_phys, w, counts, offsets, blockhist, blockbase,

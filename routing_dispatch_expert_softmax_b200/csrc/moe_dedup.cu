@@ -185,10 +185,7 @@ extern "C" int moe_dispatch_dedup(const int32_t* idx, const moe_bf16* x, const m
                                   int32_t* token_of, uint32_t* slot_mask,
                                   int32_t* rank_row_of, moe_bf16* x_dedup, void* ws,
                                   void* stream) {
-  if (!s || s->T < 0 || s->T > (1 << 20) || s->d < 64 || s->d > 16384 || s->d % 64 ||
-      s->E < 1 || s->E > kMaxE || s->k < 1 || s->k > kMaxK || s->k > s->E || s->f < 64 ||
-      s->f > 32768 || s->f % 64 || s->R < 2 || s->R > kMaxR || s->E % s->R)
-    return MOE_ERR_INVALID_ARG;
+  if (!shape_valid(s) || s->R < 2) return MOE_ERR_INVALID_ARG;
   if (!ws || !al(ws, 256) || !send_counts || !rank_offsets || !al(send_counts, 4) ||
       !al(rank_offsets, 4))
     return MOE_ERR_INVALID_ARG;

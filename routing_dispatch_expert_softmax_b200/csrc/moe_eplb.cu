@@ -2,10 +2,11 @@
 // logical -> physical expert remap on the device.
 //
 // "Serving MoE models with expert parallelism on 8xH200", section "Routing
-// imbalance": measure per-expert load, place redundant copies of popular
-// experts on less-loaded GPUs, co-locate hot and cold experts.  "vLLM Expert
-// Parallel deployment" (EPLB section): the balancer works from load collected
-// over a window, with the number of redundant experts as its knob.  The pages
+// imbalance": the load of each expert is measured, the busiest experts get
+// extra copies hosted by the devices with spare capacity, and busy and idle
+// experts are mixed on each device.  "vLLM Expert Parallel deployment" (EPLB
+// section): the load comes from a window of recent steps and the count of
+// extra copies is a setting.  The pages
 // give no algorithm; the plan below is the plainest integer reading:
 //   1. every expert starts with one copy; n_redundant times the expert with
 //      the largest load per copy gets another (ties: lower id);

@@ -81,10 +81,7 @@ extern "C" int moe_dispatch_noalloc(const int32_t* idx, const moe_bf16* x,
                                     int32_t* perm, int32_t* row_of, moe_bf16* x_perm,
                                     int32_t* send_counts, int32_t* rank_offsets,
                                     void* stream) {
-  if (!s || s->T < 0 || s->T > (1 << 20) || s->d < 64 || s->d > 16384 || s->d % 64 ||
-      s->E < 1 || s->E > kMaxE || s->k < 1 || s->k > kMaxK || s->k > s->E || s->f < 64 ||
-      s->f > 32768 || s->f % 64 || s->R < 0 || s->R > kMaxR || (s->R > 1 && s->E % s->R))
-    return MOE_ERR_INVALID_ARG;
+  if (!shape_valid(s)) return MOE_ERR_INVALID_ARG;
   if (!counts || !offsets || !al(counts, 4) || !al(offsets, 4)) return MOE_ERR_INVALID_ARG;
   if ((send_counts || rank_offsets) && s->R <= 1) return MOE_ERR_INVALID_ARG;
   if ((send_counts && !al(send_counts, 4)) || (rank_offsets && !al(rank_offsets, 4)))

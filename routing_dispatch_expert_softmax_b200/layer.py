@@ -13,26 +13,88 @@ from __future__ import annotations
 
 from typing import Dict, Optional
 
+import numpy as np
 import torch
 
 from . import binding as B
 
 
+class LoadWindow:
+    """Per-expert load over the last ``window`` layer calls, and the rule that
+    decides when to re-plan the replicas.
+
+    "vLLM Expert Parallel deployment" (EPLB section): the balancer works from
+    the load of a window of recent steps (window_size) and re-plans at a fixed
+    step interval (step_interval), adding a configured number of extra expert
+    copies.  "Serving MoE models with expert parallelism on 8xH200", section
+    "Routing imbalance": the imbalance factor is the busiest device's load over
+    the mean, and about 1.3 is where acting pays.  Readings taken: a re-plan
+    is considered every ``step_interval`` recorded calls, and adopted when the
+    window's imbalance factor over the current placement exceeds
+    ``threshold``; the window restarts after a re-plan (its counts described
+    the old placement).
+
+    Each call's per-(physical-)expert row counts are written by the layer's
+    own routing kernel into one slot of a device ring of ``window`` rows (the
+    ``counts_out`` of the layer call), so recording costs no extra work on the
+    device; only a re-plan decision copies the ring to the host."""
+
+    def __init__(self, n_experts: int, window: int, device):
+        if window < 1:
+            raise ValueError("window must be >= 1")
+        self.window = int(window)
+        self.ring = torch.zeros(self.window, int(n_experts), dtype=torch.int32, device=device)
+        self.calls = 0
+
+    def next_slot(self) -> torch.Tensor:
+        """The ring row the next call writes its counts into."""
+        slot = self.ring[self.calls % self.window]
+        self.calls += 1
+        return slot
+
+    def reset(self, n_experts: Optional[int] = None):
+        if n_experts is not None and n_experts != self.ring.shape[1]:
+            self.ring = torch.zeros(self.window, int(n_experts), dtype=torch.int32,
+                                    device=self.ring.device)
+        else:
+            self.ring.zero_()
+        self.calls = 0
+
+    def load(self) -> np.ndarray:
+        """Rows per expert summed over the recorded calls in the window
+        (int64, on the host)."""
+        n = min(self.calls, self.window)
+        return self.ring[:n].cpu().numpy().astype(np.int64).sum(axis=0)
+
+
+def imbalance_factor(load, R: int) -> float:
+    """Busiest rank's rows over the mean per rank, rank r owning experts
+    [r*P/R, (r+1)*P/R) of the P entries of ``load`` ("Serving MoE models with
+    expert parallelism on 8xH200", section "Routing imbalance")."""
+    load = np.asarray(load, dtype=np.int64)
+    R = max(int(R), 1)
+    per = load.reshape(R, -1).sum(axis=1)
+    mean = per.mean()
+    return float(per.max() / mean) if mean > 0 else 0.0
+
+
 class _Graphed:
-    """One captured layer call for a fixed T: static x / y buffers + graph."""
+    """One captured layer call for a fixed T: static x / y / counts buffers +
+    graph."""
 
     def __init__(self, layer: "MoELayer", T: int):
         dev = layer.w13.device
         self.x = torch.zeros(T, layer.d, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(T, layer.d, dtype=torch.bfloat16, device=dev)
+        self.counts = torch.zeros(layer.physical_experts, dtype=torch.int32, device=dev)
         self.ws = layer._new_workspace(T)
         # One eager call first: first-use set-up (kernel attributes, driver
         # entry points) must not happen under capture.
-        layer._call(self.x, self.y, self.ws)
+        layer._call(self.x, self.y, self.ws, counts_out=self.counts)
         torch.cuda.current_stream(dev).synchronize()
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
-            layer._call(self.x, self.y, self.ws)
+            layer._call(self.x, self.y, self.ws, counts_out=self.counts)
 
 
 class MoELayer:
@@ -61,6 +123,7 @@ class MoELayer:
         self._graphs: Dict[int, _Graphed] = {}
         self._last_ws: Optional[torch.Tensor] = None
         self._eplb: Optional[dict] = None
+        self._auto: Optional[dict] = None
 
     def shape(self, T: int) -> B.MoEShape:
         return B.MoEShape.of(T, self.d, self.E, self.k, self.f, self.R)
@@ -106,7 +169,7 @@ class MoELayer:
         self._eplb = dict(E_phys=self.E + int(n_redundant),
                           w13=self.w13.index_select(0, sel).contiguous(),
                           w2=self.w2.index_select(0, sel).contiguous(),
-                          off=off.to(dev), phys=phys.to(dev))
+                          off=off.to(dev), phys=phys.to(dev), p2l=p2l.numpy().astype(np.int64))
         self._ws.clear()
         self._graphs.clear()
         return p2l, off, phys
@@ -115,6 +178,49 @@ class MoELayer:
     def physical_experts(self) -> int:
         return self.E if self._eplb is None else self._eplb["E_phys"]
 
+    def enable_auto_rebalance(self, n_redundant: int, window: int = 1000,
+                              step_interval: int = 3000, threshold: float = 1.3):
+        """Keep a load window over the layer's calls and re-plan the replicas
+        by it (see ``LoadWindow``): every ``step_interval`` calls, if the
+        busiest of max(R, 1) ranks carries more than ``threshold`` times the
+        mean rows of the window, adopt ``rebalance(load, n_redundant)``.
+        The defaults are the example settings of the vLLM EPLB configuration
+        and the ~1.3 of the routing-imbalance discussion."""
+        if self.fp8:
+            raise NotImplementedError("replica plans run on bf16 experts only")
+        if step_interval < 1 or threshold < 1.0:
+            raise ValueError("step_interval >= 1 and threshold >= 1 required")
+        self._auto = dict(window=LoadWindow(self.physical_experts, window, self.w13.device),
+                          n_redundant=int(n_redundant), step_interval=int(step_interval),
+                          threshold=float(threshold), since=0, replans=0, last_factor=None)
+
+    @property
+    def load_window(self) -> Optional[LoadWindow]:
+        return None if self._auto is None else self._auto["window"]
+
+    def logical_load(self) -> np.ndarray:
+        """The window's rows per logical expert (replicas summed)."""
+        load = self._auto["window"].load()
+        if self._eplb is None:
+            return load
+        out = np.zeros(self.E, dtype=np.int64)
+        np.add.at(out, self._eplb["p2l"], load)
+        return out
+
+    def _after_call(self):
+        """Counts one recorded call; at each interval decides on a re-plan."""
+        a = self._auto
+        a["since"] += 1
+        if a["since"] < a["step_interval"]:
+            return
+        a["since"] = 0
+        factor = imbalance_factor(a["window"].load(), max(self.R, 1))
+        a["last_factor"] = factor
+        if factor > a["threshold"]:
+            self.rebalance(self.logical_load(), a["n_redundant"])
+            a["replans"] += 1
+            a["window"].reset(self.physical_experts)
+
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
                 idx_out=None, w_out=None, counts_out=None, stream=None) -> torch.Tensor:
         """Eager call: y = MoE(x) for a device tensor x (T, d) bf16."""
@@ -122,8 +228,13 @@ class MoELayer:
         y = out if out is not None else torch.empty_like(x)
         ws = self.workspace(T)
         self._last_ws = ws
-        self._call(x, y, ws, idx_out=idx_out, w_out=w_out, counts_out=counts_out,
-                   stream=stream)
+        slot = self._auto["window"].next_slot() if self._auto is not None else None
+        self._call(x, y, ws, idx_out=idx_out, w_out=w_out,
+                   counts_out=slot if slot is not None else counts_out, stream=stream)
+        if slot is not None:
+            if counts_out is not None:
+                counts_out.copy_(slot)
+            self._after_call()
         return y
 
     __call__ = forward
@@ -140,6 +251,7 @@ class MoELayer:
         g.x.copy_(x, non_blocking=True)
         g.graph.replay()
         self._last_ws = g.ws
+        self._record_graphed(g)
         if out is not None:
             out.copy_(g.y, non_blocking=True)
             return out
@@ -154,7 +266,13 @@ class MoELayer:
         g.graph.replay()
         y_host.copy_(g.y, non_blocking=True)
         self._last_ws = g.ws
+        self._record_graphed(g)
         return y_host
+
+    def _record_graphed(self, g: _Graphed):
+        if self._auto is not None:
+            self._auto["window"].next_slot().copy_(g.counts, non_blocking=True)
+            self._after_call()
 
     def check(self, stream=None) -> int:
         """Synchronises and returns (and clears) the last call's error word."""

@@ -48,18 +48,27 @@ def logit_bound(x64, wg64, bias64=None):
 
 
 def logit_bound_tensor_cores(x64, wg64, bias64=None):
-    """Bound for the tensor-core router (T > 256): W_g is carried as three
-    bf16 planes (residual below 2^-24 |W| per term, counted as one more
-    rounding) and the 3d products are accumulated in fp32 by the tensor cores,
-    whose internal rounding we allow twice the fp32 unit roundoff:
-    2 gamma_{3d+4} * (sum|x W| + |b|)."""
+    """Bound for the tensor-core router (T > 256).
+
+    W_g is carried as three bf16 planes hi + mid + lo; every product of a
+    bf16 x with a bf16 plane value is exact in fp32, and the planes leave a
+    residual below 2^-24 |W| per term, counted as one more rounding.  The
+    3d products are then accumulated in fp32 by the tensor cores.  Their
+    adds are not guaranteed to round to nearest; the reading taken is that
+    each add may truncate (round toward zero), whose relative error bound is
+    2^-23 = 2u instead of u.  n = 3d + 4 covers the 3d - 1 adds of the
+    products (in any grouping, the K partitions' partial sums included), the
+    plane residual and the bias add, with two to spare; the standard bound
+    with unit roundoff 2u is then
+    gamma_n(2u) (sum|x W| + |b|), gamma_n(2u) = 2nu / (1 - 2nu)."""
     d = x64.shape[1]
     n = 3 * d + 4
-    gamma = n * U32 / (1 - n * U32)
+    u2 = 2 * U32
+    gamma = n * u2 / (1 - n * u2)
     s = np.abs(x64) @ np.abs(wg64)
     if bias64 is not None:
         s = s + np.abs(bias64)[None, :]
-    return 2 * gamma * s
+    return gamma * s
 
 
 def selection_is_valid(L64_row, delta_row, sel):

@@ -266,17 +266,22 @@ def _ffn_case(cfg, seed=0, sample_rows=None):
     return assert_layer_close(got, ref, f"moe_ffn {cfg.name}")
 
 
-def _sample_rows(n_per_expert=3, max_experts=24, seed=0):
+def _sample_rows(n_random=256, seed=0):
+    """Rows of the expert-major buffer to check: the first and last row of
+    every touched expert, the rows on both sides of every 128-row tile
+    boundary inside an expert (where a tile-indexing mistake would show),
+    and a seeded random sample of n_random rows."""
     def pick(offsets, counts):
         rng = np.random.default_rng(seed)
+        offsets = np.asarray(offsets, dtype=np.int64)
         touched = np.nonzero(counts)[0]
-        hot = touched[np.argsort(-counts[touched], kind="stable")]
-        chosen = np.unique(np.concatenate([hot[:max_experts // 2], hot[-(max_experts // 2):]]))
-        rows = []
-        for e in chosen:
+        rows = [offsets[touched], offsets[touched + 1] - 1]
+        for e in touched:
             a, b = offsets[e], offsets[e + 1]
-            rows += [a, b - 1] + rng.integers(a, b, n_per_expert).tolist()
-        return np.unique(np.array(rows, dtype=np.int64))
+            edges = np.arange(a + 128, b, 128)
+            rows += [edges - 1, edges]
+        rows.append(rng.integers(0, offsets[-1], n_random))
+        return np.unique(np.concatenate(rows))
     return pick
 
 
@@ -331,11 +336,18 @@ def test_ffn_qwen_prefill_sampled():
 
 
 def test_ffn_mixtral_sampled():
-    _ffn_case(wl.MIXTRAL_8X7B.with_T(1024), sample_rows=_sample_rows(n_per_expert=6))
+    _ffn_case(wl.MIXTRAL_8X7B.with_T(1024), sample_rows=_sample_rows())
 
 
-def test_ffn_deepseek_sampled():
-    _ffn_case(wl.DEEPSEEK_V3_ROUTED.with_T(64), sample_rows=_sample_rows(max_experts=8))
+def test_ffn_deepseek_full():
+    # every row of every touched expert (512 rows over the experts the
+    # Zipf-skewed batch touches)
+    _ffn_case(wl.DEEPSEEK_V3_ROUTED.with_T(64))
+
+
+def test_ffn_deepseek_large_batch_sampled():
+    # T = 512: single-CTA 128-row tiles over sparse, skewed experts
+    _ffn_case(wl.DEEPSEEK_V3_ROUTED.with_T(512), sample_rows=_sample_rows())
 
 
 # ---------------------------------------------------------------- whole layer
@@ -402,32 +414,42 @@ def test_forward_qwen_decode(T):
     _check_forward(wl.QWEN3_30B_A3B_DECODE.with_T(T))
 
 
-def _token_sample(n=64, seed=0):
+def _token_sample(n=256, seed=0):
+    """A seeded sample of n tokens of the batch that always includes tokens
+    routed to the two hottest and the four coldest touched experts (the
+    first two and the last token of each), and the first and last token."""
     def pick(idx_h, counts):
         rng = np.random.default_rng(seed)
         T = idx_h.shape[0]
         touched = np.nonzero(counts)[0]
-        hottest, coldest = touched[np.argmax(counts[touched])], touched[np.argmin(counts[touched])]
-        must = [int(np.nonzero((idx_h == hottest).any(1))[0][0]),
-                int(np.nonzero((idx_h == coldest).any(1))[0][0]), 0, T - 1]
-        return np.unique(np.concatenate([must, rng.integers(0, T, n)]))
+        order = touched[np.argsort(-counts[touched], kind="stable")]
+        must = {0, T - 1}
+        for e in np.concatenate([order[:2], order[-4:]]):
+            toks = np.nonzero((idx_h == e).any(1))[0]
+            must.update(int(t) for t in toks[:2])
+            must.add(int(toks[-1]))
+        must = np.array(sorted(must), dtype=np.int64)
+        rest = np.setdiff1d(np.arange(T), must)
+        fill = rng.choice(rest, size=max(0, min(n - must.size, rest.size)), replace=False)
+        return np.unique(np.concatenate([must, fill]))
     return pick
 
 
 def test_forward_qwen_prefill_sampled():
-    _check_forward(wl.QWEN3_30B_A3B_PREFILL, sample=_token_sample(64))
+    _check_forward(wl.QWEN3_30B_A3B_PREFILL, sample=_token_sample())
 
 
 def test_forward_mixtral_sampled():
-    _check_forward(wl.MIXTRAL_8X7B, sample=_token_sample(24))
+    _check_forward(wl.MIXTRAL_8X7B, sample=_token_sample())
 
 
 @pytest.mark.parametrize("T", [1, 64, 512, 16384])
 def test_forward_deepseek(T):
-    # T = 512: single-CTA tiles over sparse experts; T = 16384: multi-block
-    # routing tables and CTA-pair tiles with E = 256.  The sampled tokens
-    # include ones routed to the hottest and the coldest expert.
-    _check_forward(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=None if T == 1 else _token_sample(6))
+    # T <= 64: every token.  T = 512: single-CTA tiles over sparse experts;
+    # T = 16384: multi-block routing tables and CTA-pair tiles with E = 256;
+    # both on a 256-token sample that includes tokens routed to the hottest
+    # and the coldest experts.
+    _check_forward(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=None if T <= 64 else _token_sample())
 
 
 @pytest.mark.parametrize("cfg", [

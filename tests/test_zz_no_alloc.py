@@ -4,10 +4,14 @@ Some callers cannot hand the library a workspace: their device memory is a
 fixed pool set up before serving starts, or they are a plugin that receives
 its inputs and outputs and may not call an allocator.  moe_dispatch_noalloc
 serves them by keeping its scratch in a fixed device array inside the
-library.  This test calls it through the C ABI and checks that its results
-equal moe_dispatch's (which uses a caller workspace) on two calls in a row,
-with different shapes, so the second call runs on the scratch the first one
-left behind.  Routing tables and the gathered rows must match bit for bit.
+library.  These tests call it through the C ABI and check that its results
+equal moe_dispatch's (which uses a caller workspace) and the oracle's on two
+calls in a row, with different shapes, so the second call runs on the scratch
+the first one left behind; routing tables and the gathered rows must match
+bit for bit.  They also check that a warmed-up call changes neither the free
+device memory nor PyTorch's allocation count, that an empty batch zeroes the
+tables, and what an out-of-range expert id does (it is left out of the
+counts, so offsets[E] comes out below T*k).
 
 This file is collected last on purpose; it passes alone in a fresh process as
 well as after the rest of the suite.
@@ -19,6 +23,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import routing_dispatch_expert_softmax_b200 as moe
 from routing_dispatch_expert_softmax_b200 import binding as B
 from routing_dispatch_expert_softmax_b200 import workloads as wl
@@ -62,6 +67,77 @@ def test_noalloc_dispatch_matches_workspace_dispatch(calls):
             if ref[name] is not None:
                 assert torch.equal(got[name], ref[name]), (n, name)
         assert int(got["offsets"][-1]) == T * k
+        # and against the oracle's dispatch of the same ids
+        idx_h = idx.cpu().numpy()
+        ref_counts = oracle.expert_counts(idx_h, E)
+        ref_perm, ref_row_of = oracle.dispatch_rows(idx_h, E)
+        np.testing.assert_array_equal(got["counts"].cpu().numpy(), ref_counts)
+        np.testing.assert_array_equal(got["offsets"].cpu().numpy(),
+                                      oracle.expert_offsets(ref_counts))
+        np.testing.assert_array_equal(got["perm"].cpu().numpy(), ref_perm)
+        np.testing.assert_array_equal(got["row_of"].cpu().numpy(), ref_row_of)
+        assert torch.equal(got["x_perm"], x[torch.from_numpy(ref_perm).long().to(DEV)])
+        if R > 1:
+            S, ro = oracle.virtual_ep_layout(idx_h, E, R)
+            np.testing.assert_array_equal(got["send"].cpu().numpy(), S)
+            np.testing.assert_array_equal(got["roff"].cpu().numpy(), ro)
+
+
+def _noalloc(idx, x, out, shape):
+    moe.moe_dispatch_noalloc(idx, x, out["counts"], out["offsets"], out["perm"],
+                             out["row_of"], out["x_perm"], shape, out["send"], out["roff"])
+
+
+def test_noalloc_dispatch_allocates_nothing():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    T, d, E, k, R = 256, 512, 64, 4, 4
+    idx = _routing(T, E, k, 3).to(DEV)
+    x = wl.make_hidden(wl.MoEConfig("x", T=T, d=d, E=E, k=k, f=64), DEV, 2)
+    shape = MoEShape.of(T, d, E, k, 64, R)
+    out = _outputs(T, d, E, k, R)
+    _noalloc(idx, x, out, shape)  # warm-up: kernels loaded, scratch address looked up
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    _noalloc(idx, x, out, shape)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0, (free0, free1)
+
+
+def test_noalloc_dispatch_empty_batch_zeroes_tables():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    E, R = 16, 4
+    shape = MoEShape.of(0, 64, E, 2, 64, R)
+    counts = torch.full((E,), 5, dtype=torch.int32, device=DEV)
+    offsets = torch.full((E + 1,), 5, dtype=torch.int32, device=DEV)
+    send = torch.full((R, R), 5, dtype=torch.int32, device=DEV)
+    roff = torch.full((R + 1,), 5, dtype=torch.int32, device=DEV)
+    moe.moe_dispatch_noalloc(None, None, counts, offsets, None, None, None, shape, send, roff)
+    torch.cuda.synchronize()
+    for t in (counts, offsets, send, roff):
+        assert int(t.abs().sum()) == 0
+
+
+def test_noalloc_dispatch_leaves_out_of_range_ids_uncounted():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    T, d, E, k = 50, 64, 8, 2
+    idx = _routing(T, E, k, 4)
+    idx[7, 1] = E + 3  # out of range: never dereferenced, not counted
+    shape = MoEShape.of(T, d, E, k, 64)
+    x = wl.make_hidden(wl.MoEConfig("x", T=T, d=d, E=E, k=k, f=64), DEV, 1)
+    out = _outputs(T, d, E, k, 0)
+    _noalloc(idx.to(DEV), x, out, shape)
+    torch.cuda.synchronize()
+    valid = idx.numpy().reshape(-1)
+    valid = valid[valid < E]
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), oracle.expert_counts(valid, E))
+    assert int(out["offsets"][-1]) == T * k - 1
+    torch.ones(1, device=DEV).sum().item()  # the context is still healthy
 
 
 def test_noalloc_dispatch_rejects_shapes_beyond_its_scratch():
