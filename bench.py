@@ -35,6 +35,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s; % of HBM (decode) or BF16 tensor-core (prefill) roofline"
+DEFAULT_WORKLOAD = "qwen3-30b-a3b-decode"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -44,38 +45,40 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ["routing_dispatch_expert_softmax_b200/csrc/moe_gemm_sm100.cu",
                   "routing_dispatch_expert_softmax_b200/csrc/moe_common.cuh"]
 
+def router_launches(cfg):
+    """Kernels of the router: one cluster kernel up to 256 tokens; above, the
+    W_g split and the tensor-core GEMM, plus a partial-sum kernel when the
+    GEMM's K is split into P > 1 partial planes (P is the largest divisor of
+    the 3d/64 K blocks, at most a quarter of them, with tiles * P <= 148)."""
+    if cfg.T <= 256:
+        return 1
+    bn = 128 if cfg.E <= 128 else 256
+    tiles = -(-cfg.T // 128) * -(-cfg.E // bn)
+    nk = 3 * cfg.d // 64
+    parts = 1
+    for p in range(2, nk // 4 + 1):
+        if nk % p:
+            continue
+        if tiles * p > 148:
+            break
+        parts = p
+    return 2 if parts == 1 else 3
+
+
 def launches_per_forward(cfg, eplb_redundant=0):
     """Kernels one moe_forward (moe_forward_eplb with eplb_redundant > 0)
-    launches: router (one cluster kernel up to 256 tokens; above, the W_g
-    split and the tensor-core GEMM, plus a partial-sum kernel when the GEMM's
-    K is split into P > 1 partial planes: P is the largest divisor of the
-    3d/64 K blocks, at most a quarter of them, with tiles * P <= 148),
-    routing (one fused kernel for T <= 1024, else top-k + histogram + scan +
-    scatter; with replicas top-k + remap + histogram + scan + scatter),
-    gather, the two expert GEMMs (each followed by the lone-tile kernel when
-    they run on CTA pairs), combine."""
+    launches: the router (router_launches), routing (one fused kernel for
+    T <= 1024, else top-k + histogram + scan + scatter; with replicas top-k +
+    remap + histogram + scan + scatter), gather, the two expert GEMMs (each
+    followed by the lone-tile kernel when they run on CTA pairs), combine."""
     T = cfg.T
-    if T <= 256:
-        router = 1
-    else:
-        bn = 128 if cfg.E <= 128 else 256
-        tiles = -(-T // 128) * -(-cfg.E // bn)
-        nk = 3 * cfg.d // 64
-        parts = 1
-        for p in range(2, nk // 4 + 1):
-            if nk % p:
-                continue
-            if tiles * p > 148:
-                break
-            parts = p
-        router = 2 if parts == 1 else 3
     routing = 1 if T <= 1024 else 4
     if eplb_redundant:
         routing = 5
     gemms = 2
     if T > 256 and T * cfg.k >= 128 * (cfg.E + eplb_redundant):
         gemms = 4
-    return router + routing + 1 + gemms + 1
+    return router_launches(cfg) + routing + 1 + gemms + 1
 
 
 def parse_args(argv=None):
@@ -84,11 +87,19 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="qwen3-30b-a3b-decode")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--T", type=int, default=None, help="override the token count")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-sweep", action="store_true",
+                   help="skip the sweep over every workload configuration that the default "
+                        "single-GPU run appends to its line")
     p.add_argument("--fp8", action="store_true",
                    help="E4M3 expert weights with fp32 row scales (batches of up to 256)")
+    p.add_argument("--ep", action="store_true",
+                   help="expert parallelism over the launched ranks: each rank holds E/N whole "
+                        "experts and its own batch; tokens are exchanged with NCCL all-to-all-v "
+                        "and the layer runs eagerly (one host synchronisation per call for the "
+                        "split sizes)")
     p.add_argument("--eplb-redundant", type=int, default=0,
                    help="time the layer with this many redundant expert copies placed by "
                         "the EPLB-style plan (built from the counts of one warm-up call)")
@@ -137,15 +148,19 @@ def workload_config(name, T):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi clock/throttle samples every 200 ms during the timed region."""
+    """nvidia-smi clock/throttle samples every 200 ms while running; each
+    sample carries its timestamp so a summary can be taken over any window
+    (a timed region) of the run."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
+        self.rows = []
         self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
 
     def start(self):
@@ -157,6 +172,7 @@ class ClockSampler:
                 stdout=self.tmp, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        return self
 
     def _ident(self):
         import torch
@@ -166,7 +182,20 @@ class ClockSampler:
         except Exception:
             return str(self.dev)
 
+    @staticmethod
+    def _parse(line):
+        import datetime
+        r = [c.strip() for c in line.split(",")]
+        try:
+            ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            reasons = {nm for nm, v in zip(ClockSampler.REASONS, r[6:10])
+                       if v.lower() == "active"}
+            return {"t": ts, "sm": float(r[2]), "max": float(r[3]), "reasons": reasons}
+        except (ValueError, IndexError):
+            return None
+
     def stop(self):
+        """Stops sampling; returns the summary of every sample (or None)."""
         if self.proc is None:
             return None
         time.sleep(0.25)
@@ -177,23 +206,33 @@ class ClockSampler:
             self.proc.kill()
         self.tmp.flush()
         self.tmp.seek(0)
-        rows = [r.strip().split(",") for r in self.tmp.read().splitlines() if r.strip()]
+        self.rows = [r for r in (self._parse(ln) for ln in self.tmp.read().splitlines()
+                                 if ln.strip()) if r]
         os.unlink(self.tmp.name)
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                sm.append(float(r[1]))
-                mx = max(mx, float(r[2]))
-                for nm, v in zip(names, r[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(nm)
-            except (ValueError, IndexError):
-                continue
-        if not sm:
+        return self.summary()
+
+    def summary(self, t0=None, t1=None):
+        """Median SM clock, max clock and active reasons of the samples taken
+        in [t0, t1] (all samples without a window).  A window shorter than
+        the sampling period may hold none: then the nearest sample stands in
+        and its distance is given."""
+        rows = self.rows
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sel = rows if t0 is None else [r for r in rows if t0 <= r["t"] <= t1]
+        out = {}
+        if not sel:
+            mid = 0.5 * (t0 + t1)
+            near = min(rows, key=lambda r: abs(r["t"] - mid))
+            sel = [near]
+            out["nearest_sample_s"] = round(abs(near["t"] - mid), 3)
+        reasons = set()
+        for r in sel:
+            reasons |= r["reasons"]
+        out.update({"sm_mhz": statistics.median(r["sm"] for r in sel),
+                    "sm_max_mhz": max(r["max"] for r in sel), "reasons": sorted(reasons),
+                    "samples": len(sel) if "nearest_sample_s" not in out else 0})
+        return out
 
 
 # ------------------------------------------------------------------ distributed
@@ -387,6 +426,176 @@ def routing_stats(counts, R):
     return out
 
 
+STAGES = ["router", "topk_dispatch_gather", "gemm1_swiglu", "gemm2", "combine"]
+
+# Every configuration of the workload list, timed in the default run: the
+# tiny layer, Qwen3-30B-A3B decode at four batch sizes, Qwen3-30B-A3B
+# prefill, Mixtral-8x7B and the DeepSeek-V3 routed experts at four batch
+# sizes (each model's weights are generated once and freed before the next).
+SWEEP = (("tiny", (64,)), ("qwen3-30b-a3b-decode", (1, 8, 64, 256)),
+         ("qwen3-30b-a3b-prefill", (8192,)), ("mixtral-8x7b", (4096,)),
+         ("deepseek-v3-routed", (1, 64, 512, 16384)))
+
+
+def capture_graph(fn):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def timed_passes(plain_fn, staged_fn, steps, warmup, flush_l2, stream, dist, dev, check):
+    """The timed region: W warm-up replays, then K steps of one CUDA graph of
+    the plain layer call between two events (the headline pass), then K steps
+    of graphs captured with stage events at the kernel boundaries (pass 2;
+    its event nodes cost a few microseconds each, so stage times are upper
+    bounds).  L2 is flushed before every step, outside the events.  Returns
+    (per-step ms, per-step stage ms, wall-clock window of the timed region)."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    plain = capture_graph(plain_fn)
+    for _ in range(warmup):
+        flush_l2()
+        plain.replay()
+    torch.cuda.synchronize(dev)
+    check()
+    step_ev = [(ev(), ev()) for _ in range(steps)]
+    events = [[ev() for _ in range(STAGE_EVENTS)] for _ in range(steps)]
+    staged = [capture_graph(lambda e=e: staged_fn(e)) for e in events]
+    for g in staged[:2]:
+        flush_l2()
+        g.replay()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for i in range(steps):
+        flush_l2()
+        step_ev[i][0].record(stream)
+        plain.replay()
+        step_ev[i][1].record(stream)
+    for i in range(steps):
+        flush_l2()
+        staged[i].replay()
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if dist:
+        dist.barrier()
+    check()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    stage_ms = [[e[j].elapsed_time(e[j + 1]) for j in range(STAGE_EVENTS - 1)] for e in events]
+    del staged, plain
+    return step_ms, stage_ms, (t0, t1)
+
+
+STAGE_EVENTS = 6
+
+
+def kernel_roofline(cfg, alg, mean_stage, peaks, peak_src, traffic_key):
+    """Roofline of the dominant stage: its algorithmic bytes (or flops, for
+    an expert GEMM at a tensor-bound batch) over its mean event time."""
+    decode = cfg.P / cfg.E < 64
+    dom = max(range(len(mean_stage)), key=lambda j: mean_stage[j])
+    kern = STAGES[dom]
+    t_kern = mean_stage[dom] / 1e3
+    if kern in ("gemm1_swiglu", "gemm2") and not decode:
+        fl = alg["gemm1_flops"] if kern == "gemm1_swiglu" else alg["gemm2_flops"]
+        achieved = fl / t_kern / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        by = {"gemm1_swiglu": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(
+            kern, cfg.T * cfg.d * 2 * 2)
+        achieved = by / t_kern / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
+    roof["kernel"] = kern
+    roof["peak_source"] = (f"{peak_src} ("
+                           f"{'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})")
+    roof["traffic"] = profiled_traffic(traffic_key, kern)
+    return roof
+
+
+def layer_roofline(cfg, alg, touched, ms_per_step, peaks):
+    """The whole layer's algorithmic bytes and flops against the measured
+    peaks and the spec denominators (~8 TB/s HBM, 2.25 PF/s dense bf16)."""
+    t_layer = ms_per_step / 1e3
+    decode = cfg.P / cfg.E < 64
+    return {
+        "bytes": alg["bytes"], "flops": alg["flops"], "touched_experts": touched,
+        "hbm_frac_measured": alg["bytes"] / t_layer / (peaks["hbm_gbs"] * 1e9),
+        "hbm_frac_spec_8TBs": alg["bytes"] / t_layer / 8e12,
+        "tensor_frac_measured": alg["flops"] / t_layer / (peaks["bf16_tflops"] * 1e12),
+        "tensor_frac_spec_2250TF": alg["flops"] / t_layer / 2.25e15,
+        "bound": "hbm" if decode else "tensor",
+    }
+
+
+def run_sweep(args, dev, local, peaks, peak_src, flush_l2, stream):
+    """Every configuration of SWEEP, each timed like the headline (plain and
+    staged graph passes, L2 flushed before every step); one clock sampler
+    runs across the sweep and each point gets the samples of its own timed
+    region."""
+    import torch
+
+    import routing_dispatch_expert_softmax_b200 as moe
+    from routing_dispatch_expert_softmax_b200 import workloads as wl
+    points = []
+    clocks = ClockSampler(local).start()
+    steps, warmup = max(args.steps, 1), max(args.warmup, 3)
+    for name, Ts in SWEEP:
+        base = wl.CONFIGS[name]
+        w_g, bias = wl.make_router(base, dev, 0)
+        w13, w2 = wl.make_experts(base, dev, 0)
+        for T in Ts:
+            cfg = base.with_T(T)
+            x = wl.make_hidden(cfg, dev, 0)
+            shape = moe.MoEShape.from_config(cfg)
+            ws = moe.workspace(shape, dev)
+            y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
+            counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+            moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, counts_out=counts)
+            torch.cuda.synchronize(dev)
+
+            def check():
+                st = moe.moe_check(ws)
+                if st != moe.MOE_OK:
+                    raise RuntimeError(f"{cfg.name}: {moe.moe_error_string(st)}")
+
+            step_ms, stage_ms, win = timed_passes(
+                lambda: moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws),
+                lambda e: moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, e),
+                steps, warmup, flush_l2, stream, None, dev, check)
+            counts_h = counts.cpu().tolist()
+            touched = sum(1 for v in counts_h if v > 0)
+            alg = algorithmic(cfg, touched)
+            ms = statistics.fmean(step_ms)
+            mean_stage = [statistics.fmean(s[j] for s in stage_ms)
+                          for j in range(len(stage_ms[0]))]
+            points.append({
+                "workload": base.name, "T": cfg.T, "us_per_layer": ms * 1e3,
+                "tokens_per_s": cfg.T / (ms / 1e3),
+                "layer_roofline": layer_roofline(cfg, alg, touched, ms, peaks),
+                "roofline": kernel_roofline(cfg, alg, mean_stage, peaks, peak_src,
+                                            f"{base.name}@T{cfg.T}"),
+                "stage_us": {k: v * 1e3 for k, v in zip(STAGES, mean_stage)},
+                "routing": routing_stats(counts_h, cfg.R), "window": win})
+            del x, ws, y, counts
+        del w_g, bias, w13, w2
+        torch.cuda.empty_cache()
+    overall = clocks.stop()
+    for p in points:
+        t0, t1 = p.pop("window")
+        p["clocks"] = clocks.summary(t0, t1)
+    return {"points": points, "clocks": overall, "steps": steps, "warmup": warmup,
+            "note": "each point: mean of K plain CUDA-graph replays of moe_forward, L2 flushed "
+                    "before every step; stage_us from the staged pass (event nodes add a few "
+                    "us each); roofline = dominant stage vs MEASURED_PEAKS.json; clocks = "
+                    "samples inside the point's timed region, else the nearest sample"}
+
+
 def run_ours(args):
     import torch
 
@@ -427,12 +636,6 @@ def run_ours(args):
         # starts cold and pays no write-back of data the flush left dirty.
         flush_i32.sum()
 
-    # The timed region has two passes of K steps.  Pass 1 (the headline):
-    # per step, one CUDA graph of the plain layer call between two events.
-    # Pass 2: the same steps captured with stage events at the kernel
-    # boundaries (moe_forward_staged); the per-stage durations give the
-    # dominant kernel's launch time.  The extra event nodes cost a few
-    # microseconds each, so pass-2 stage times are upper bounds.
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def fwd(out, **kw):  # the layer through the C ABI (bf16 or FP8 experts)
@@ -451,6 +654,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
 
     eplb_info = None
+    ws_e = None
     if args.eplb_redundant:
         # Replicated experts: the plan comes from one call's counts (the load
         # window), the layer then runs moe_forward_eplb.  The staged pass
@@ -469,64 +673,24 @@ def run_ours(args):
                      "imbalance_plain": float(cl.max() / cl.float().mean()),
                      "imbalance_eplb": float(cp.max() / cp.float().mean())}
 
-    def capture(events=None):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            if events is None and eplb_info is not None:
-                layer(x, out=y)
-            elif events is None:
-                fwd(y)
-            else:
-                fwd_staged(events)
-        return g
+    def check():
+        st = moe.moe_check(ws)
+        if st == moe.MOE_OK and ws_e is not None:
+            st = moe.moe_check(ws_e)
+        if st != moe.MOE_OK:
+            raise RuntimeError(moe.moe_error_string(st))
 
-    plain = capture()
-    for i in range(args.warmup):
-        flush_l2()
-        plain.replay()
-    torch.cuda.synchronize(dev)
-    st = moe.moe_check(ws)
-    if st == moe.MOE_OK and eplb_info is not None:
-        st = moe.moe_check(ws_e)
-    if st != moe.MOE_OK:
-        raise RuntimeError(moe.moe_error_string(st))
+    plain_fn = (lambda: layer(x, out=y)) if eplb_info is not None else (lambda: fwd(y))
 
-    # ---------------- timed region (device)
-    step_ev = [(ev(), ev()) for _ in range(args.steps)]
-    events = [[ev() for _ in range(moe.MOE_STAGE_EVENTS)] for _ in range(args.steps)]
-    staged = [capture(e) for e in events]
-    for g in staged[:2]:
-        flush_l2()
-        g.replay()
-    torch.cuda.synchronize(dev)
-    clocks = ClockSampler(local)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    for i in range(args.steps):
-        flush_l2()
-        step_ev[i][0].record(stream)
-        plain.replay()
-        step_ev[i][1].record(stream)
-    for i in range(args.steps):
-        flush_l2()
-        staged[i].replay()
-    torch.cuda.synchronize(dev)
-    if dist:
-        dist.barrier()
-    clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    stage_ms = [[e[s].elapsed_time(e[s + 1]) for s in range(moe.MOE_STAGE_EVENTS - 1)]
-                for e in events]
+    # ---------------- timed region (device); the clock sampler runs from
+    # before the warm-up to the end of the end-to-end pass below
+    clocks = ClockSampler(local).start()
+    step_ms, stage_ms, _ = timed_passes(plain_fn, fwd_staged, args.steps, args.warmup,
+                                        flush_l2, stream, dist, dev, check)
     total_ms = max_over_ranks(dist, sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     tokens = sum_over_ranks(dist, cfg.T * args.steps, dev)
     value = tokens / (total_ms / 1e3)
-    st = moe.moe_check(ws)
-    if st != moe.MOE_OK:
-        raise RuntimeError(moe.moe_error_string(st))
-    del staged, plain
 
     # ---------------- end to end through the public API, host buffers
     # MoELayer.forward_host: pinned x -> device, graph replay of the layer,
@@ -549,6 +713,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
+    clk = clocks.stop()
     e2e_ms = max_over_ranks(dist, sum(a.elapsed_time(b) for a, b in e2e_ev), dev)
     e2e_value = tokens / (e2e_ms / 1e3)
     y_dev = torch.empty_like(y)
@@ -611,36 +776,9 @@ def run_ours(args):
     touched = sum(1 for v in counts_h if v > 0)
     alg = algorithmic(cfg, touched, args.fp8)
     mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
-    names = ["router", "topk_dispatch_gather", "gemm1_swiglu", "gemm2", "combine"]
-    dom = max(range(len(mean_stage)), key=lambda j: mean_stage[j])
-    tokens_per_expert = cfg.P / cfg.E
-    decode = tokens_per_expert < 64
-    kern = names[dom]
-    t_kern = mean_stage[dom] / 1e3
-    if kern in ("gemm1_swiglu", "gemm2") and not decode:
-        fl = alg["gemm1_flops"] if kern == "gemm1_swiglu" else alg["gemm2_flops"]
-        achieved = fl / t_kern / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
-    else:
-        by = {"gemm1_swiglu": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(
-            kern, cfg.T * cfg.d * 2 * 2)
-        achieved = by / t_kern / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"]}
-    roof["kernel"] = kern
-    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-    roof["traffic"] = profiled_traffic(f"{cfg.name}@T{cfg.T}" + ("/fp8" if args.fp8 else ""),
-                                       kern)
-    t_layer = ms_per_step / 1e3
-    layer_roof = {
-        "bytes": alg["bytes"], "flops": alg["flops"], "touched_experts": touched,
-        "hbm_frac_measured": alg["bytes"] / t_layer / (peaks["hbm_gbs"] * 1e9),
-        "hbm_frac_spec_8TBs": alg["bytes"] / t_layer / 8e12,
-        "tensor_frac_measured": alg["flops"] / t_layer / (peaks["bf16_tflops"] * 1e12),
-        "tensor_frac_spec_2250TF": alg["flops"] / t_layer / 2.25e15,
-        "bound": "hbm" if decode else "tensor",
-    }
+    roof = kernel_roofline(cfg, alg, mean_stage, peaks, peak_src,
+                           f"{cfg.name}@T{cfg.T}" + ("/fp8" if args.fp8 else ""))
+    layer_roof = layer_roofline(cfg, alg, touched, ms_per_step, peaks)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -656,7 +794,7 @@ def run_ours(args):
         "roofline": roof,
         "layer_roofline": layer_roof,
         "routing": routing_stats(counts_h, cfg.R),
-        "stage_ms": dict(zip(names, mean_stage)),
+        "stage_ms": dict(zip(STAGES, mean_stage)),
         "stage_ms_note": "from the second timed pass with event nodes at every kernel boundary "
                          "(each adds a few us); the headline uses plain graph replays",
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * cfg.d * 2,
@@ -680,6 +818,12 @@ def run_ours(args):
         if args.fp8:
             base_inputs.update(w13_scale=s13, w2_scale=s2)
         line["cpu_baseline"] = cpu_baseline(cfg, base_inputs)
+    default_run = (args.workload == DEFAULT_WORKLOAD and args.T is None and not args.fp8
+                   and not args.eplb_redundant)
+    if world == 1 and default_run and not args.no_sweep:
+        del layer, w13, w2, ws, y, y_dev
+        torch.cuda.empty_cache()
+        line["sweep"] = run_sweep(args, dev, local, peaks, peak_src, flush_l2, stream)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -688,10 +832,130 @@ def run_ours(args):
     return 0
 
 
+def run_ep(args):
+    """--ep: the expert-parallel layer (EPMoELayer) over the launched ranks."""
+    import torch
+
+    import routing_dispatch_expert_softmax_b200 as moe
+    from routing_dispatch_expert_softmax_b200 import workloads as wl
+    from routing_dispatch_expert_softmax_b200.ep import EPMoELayer, TorchDistComm
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    moe.load_library()
+    cfg = workload_config(args.workload, args.T)
+    if cfg.E % world:
+        raise SystemExit(f"--ep needs E ({cfg.E}) divisible by the rank count ({world})")
+    E_loc = cfg.E // world
+    w_g, bias = wl.make_router(cfg, dev, 0)
+    w13, w2 = wl.make_experts(cfg, dev, 0)
+    w13 = w13[rank * E_loc:(rank + 1) * E_loc].clone()
+    w2 = w2[rank * E_loc:(rank + 1) * E_loc].clone()
+    torch.cuda.empty_cache()
+    x = wl.make_hidden(cfg, dev, rank)
+    comm = TorchDistComm() if world > 1 else _LoopbackComm()
+    layer = EPMoELayer(w_g, bias, w13, w2, cfg.k, rank, world, comm=comm)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev).view(torch.int32)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(max(args.warmup, 3)):
+        flush.sum()
+        layer(x)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local).start()
+    times = []
+    if dist:
+        dist.barrier()
+    for _ in range(args.steps):
+        flush.sum()
+        a, b = ev(), ev()
+        a.record(stream)
+        layer(x)
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+    e2e = []
+    for _ in range(args.steps):
+        flush.sum()
+        a, b = ev(), ev()
+        a.record(stream)
+        xd = x_host.to(dev, non_blocking=True)
+        y_host.copy_(layer(xd), non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e.append(a.elapsed_time(b))
+    clk = clocks.stop()
+    keep = {}
+    layer(x, keep=keep)
+    st = layer.check(keep["st"])
+    if st == moe.MOE_OK:
+        st = layer.check(keep["grp"])
+    if st != moe.MOE_OK:
+        raise RuntimeError(moe.moe_error_string(st))
+    total_ms = max_over_ranks(dist, sum(times), dev)
+    e2e_ms = max_over_ranks(dist, sum(e2e), dev)
+    tokens = sum_over_ranks(dist, cfg.T * args.steps, dev)
+    rows_in = sum_over_ranks(dist, float(sum(keep["recv_rows"])), dev)
+    line = {
+        "metric": METRIC, "value": tokens / (total_ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "global_batch": cfg.T * world, "parallelism": f"ep{world}",
+                   "experts_per_rank": E_loc,
+                   "l2": "flushed before every step (256 MiB read, outside the timed events)",
+                   "launch": "eager: router, top-k, dispatch, count all-to-all, host split "
+                             "sizes, row all-to-all-v, regroup, expert GEMMs, return "
+                             "all-to-all-v, combine"},
+        "exchange": {"rows_received_per_step_all_ranks": rows_in,
+                     "bytes_each_way_per_step_all_ranks": rows_in * cfg.d * 2},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+        "gpu_launches": ep_launches_per_forward(cfg, world) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def ep_launches_per_forward(cfg, world):
+    """Library kernels of one EPMoELayer call on one rank: router (1, or the
+    tensor-core router's 2-3 above 256 tokens) and top-k; the dispatch
+    (histogram, scan, scatter, gather); the received-row labels; the regroup
+    dispatch (4 again); moe_ffn (work lists and two GEMMs, each followed by
+    the lone-tile kernel in the CTA-pair regime, judged at the balanced
+    T*k rows per rank); the copy back to received order and the combine."""
+    router = router_launches(cfg)
+    E_loc = cfg.E // world
+    n = cfg.T * cfg.k
+    gemms = 4 if (n > 256 and n >= 128 * E_loc) else 2
+    return router + 1 + 4 + 1 + 4 + 1 + gemms + 1 + 1
+
+
+class _LoopbackComm:
+    """The one-rank exchange: every all-to-all is a copy to itself."""
+
+    def all_to_all(self, out, inp, out_splits=None, in_splits=None):
+        out.copy_(inp)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.ep:
+        return run_ep(args)
     return run_ours(args)
 
 

@@ -77,7 +77,7 @@ typedef enum moe_status {
 MOE_API const char* moe_error_string(int status);
 
 /* Library ABI version (major * 100 + minor): 101 adds the EPLB calls and
- * moe_dispatch_dedup; 102 the FP8-weight calls. */
+ * moe_dispatch_dedup; 102 the FP8-weight calls; 103 moe_ep_recv_experts. */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -251,6 +251,29 @@ MOE_API int moe_dispatch_dedup(const int32_t* idx, const moe_bf16* x, const moe_
                                int32_t* token_of, uint32_t* slot_mask,
                                int32_t* rank_row_of, moe_bf16* x_dedup, void* ws,
                                void* stream);
+
+/* Receive side of a real expert-parallel exchange ("Serving MoE models with
+ * expert parallelism on 8xH200", section "Tensor parallel vs expert
+ * parallel": tokens travel to the devices holding their experts and the
+ * results travel back; "Wide Expert Parallelism", section "All-to-all
+ * communication: the essential tradeoff").  With R ranks each owning E_loc =
+ * E / R whole experts, every rank dispatches its own tokens with moe_dispatch
+ * (s->R = R): its expert-major buffer is then rank-contiguous, and the slice
+ * for rank r is ordered by r's local expert.  After an all-to-all-v of those
+ * slices (and of the per-expert counts), rank r holds rows ordered by
+ * (source rank, local expert, token).  This call labels each received row
+ * with its local expert, so that moe_dispatch with k = 1 and these labels as
+ * ids regroups the rows expert-major (rows of one expert across all sources
+ * contiguous, source-ascending) for moe_ffn.
+ *   recv_counts   [R, E_loc] int32 in (device): rows source s sent for local
+ *                 expert e (the slices of each source's `counts`)
+ *   N             rows received (host-known; the sum of recv_counts)
+ *   expert_of_row [N] int32 out: local expert in [0, E_loc) of each row
+ * R <= 64, R * E_loc <= 1024.  Rows beyond the counts' total, or every row
+ * when a count is negative, get -1; moe_dispatch then reports them as
+ * MOE_ERR_DEVICE_CHECK.  Allocates nothing; no workspace. */
+MOE_API int moe_ep_recv_experts(const int32_t* recv_counts, int32_t R, int32_t E_loc,
+                                int32_t N, int32_t* expert_of_row, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Expert load balancing with replicated experts ("Serving MoE models with

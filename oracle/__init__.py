@@ -9,10 +9,12 @@ from .moe_oracle import *  # noqa: F401,F403
 from .eplb_oracle import *  # noqa: F401,F403
 from .dedup_oracle import *  # noqa: F401,F403
 from .fp8_oracle import *  # noqa: F401,F403
+from .ep_oracle import *  # noqa: F401,F403
 from . import dedup_oracle as _dedup
+from . import ep_oracle as _ep
 from . import eplb_oracle as _eplb
 from . import fp8_oracle as _fp8
 from . import moe_oracle as _moe
 
 __all__ = (list(_moe.__all__) + list(_eplb.__all__) + list(_dedup.__all__)
-           + list(_fp8.__all__))
+           + list(_fp8.__all__) + list(_ep.__all__))

@@ -31,7 +31,7 @@ EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router"
            "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check",
            "moe_dispatch_noalloc", "moe_eplb_plan", "moe_eplb_remap",
            "moe_workspace_size_eplb", "moe_forward_eplb", "moe_dispatch_dedup",
-           "moe_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_staged")
+           "moe_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_staged", "moe_ep_recv_experts")
 
 
 class MoEError(RuntimeError):
@@ -103,6 +103,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_workspace_size_eplb.argtypes = [_S, _i32]
     lib.moe_dispatch_dedup.restype = ctypes.c_int
     lib.moe_dispatch_dedup.argtypes = [_P, _P, _S, _P, _P, _P, _P, _P, _P, _P, _P]
+    lib.moe_ep_recv_experts.restype = ctypes.c_int
+    lib.moe_ep_recv_experts.argtypes = [_P, _i32, _i32, _i32, _P, _P]
     lib.moe_forward_eplb.restype = ctypes.c_int
     lib.moe_forward_eplb.argtypes = [_P, _P, _P, _P, _P, _S, _P, _P, _i32, _P, _P, _P, _P,
                                      _P, _P]
@@ -241,6 +243,15 @@ def moe_dispatch_dedup(idx, x, send_counts, rank_offsets, token_of, slot_mask, s
         _ptr(slot_mask, torch.int32, "slot_mask"), _ptr(rank_row_of, torch.int32, "rank_row_of"),
         _ptr(x_dedup, torch.bfloat16, "x_dedup"), _ptr(ws, torch.uint8, "ws"),
         _stream(stream)), "moe_dispatch_dedup")
+
+
+def moe_ep_recv_experts(recv_counts, R: int, E_loc: int, N: int, expert_of_row, stream=None):
+    """Local expert of each row an expert-parallel rank received (rows ordered
+    by source rank, then local expert)."""
+    _check(load_library().moe_ep_recv_experts(
+        _ptr(recv_counts, torch.int32, "recv_counts"), int(R), int(E_loc), int(N),
+        _ptr(expert_of_row, torch.int32, "expert_of_row"), _stream(stream)),
+        "moe_ep_recv_experts")
 
 
 def moe_eplb_plan(load, E: int, R: int, n_redundant: int):

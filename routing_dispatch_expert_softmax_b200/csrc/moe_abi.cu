@@ -9,7 +9,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kVersion = 102;
+constexpr int kVersion = 103;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
