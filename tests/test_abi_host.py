@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_error_strings(lib):
-    assert moe.moe_version() == 102
+    assert moe.moe_version() == 103
     for code in range(6):
         assert moe.moe_error_string(code).startswith("MOE_")
     assert "unknown" in moe.moe_error_string(99)
