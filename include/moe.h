@@ -77,7 +77,8 @@ typedef enum moe_status {
 MOE_API const char* moe_error_string(int status);
 
 /* Library ABI version (major * 100 + minor): 101 adds the EPLB calls and
- * moe_dispatch_dedup; 102 the FP8-weight calls; 103 moe_ep_recv_experts. */
+ * moe_dispatch_dedup; 102 the FP8-weight calls; 103 moe_ep_recv_experts and
+ * FP8 weights at every batch size. */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -342,8 +343,8 @@ MOE_API int moe_forward_eplb(const moe_bf16* x, const float* w_g, const float* b
                              int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
                              void* stream);
 
-/* FP8 expert weights ("Serving mixture-of-experts models: expert parallelism
- * on H200", sections "Memory math for 8xH200" and "Quantization choices":
+/* FP8 expert weights ("Serving MoE models with expert parallelism on
+ * 8xH200", sections "Memory math for 8xH200" and "Quantization choices":
  * native FP8 checkpoints store one byte per weight; the small-batch expert
  * GEMMs are bound by reading them).  The pages fix no encoding; this library
  * takes OCP FP8 E4M3 codes (bias 7, subnormals at exponent 0, S.1111.111 is
@@ -355,9 +356,12 @@ MOE_API int moe_forward_eplb(const moe_bf16* x, const float* w_g, const float* b
  * Activations, accumulation and rounding points are those of the bf16 calls:
  * the result is moe_ffn / moe_forward on the dequantised weights (each row
  * scale multiplies the fp32 accumulator before SwiGLU / the bf16 store).
- * Code pointers 16-byte aligned, scales 4-byte aligned.  Supported for
- * s->T <= 256 (the regime where the weights, not the tensor cores, bound the
- * GEMMs); larger batches return MOE_ERR_UNSUPPORTED before any launch. */
+ * Code pointers 16-byte aligned, scales 4-byte aligned.  Every batch size
+ * runs the weights-as-M (swap-AB) form: a converter warpgroup widens each
+ * streamed e4m3 weight tile to bf16 for the tensor cores; above 64 tokens the
+ * work items are 128-row token tiles of an expert, each streaming the
+ * expert's (one-byte) weights again, so large batches trade repeated weight
+ * reads for the halved weight bytes. */
 MOE_API int moe_ffn_fp8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w13,
                         const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                         const moe_shape* s, moe_bf16* z, void* ws, void* stream);

@@ -192,7 +192,6 @@ static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const flo
                         void* stream, void* const* events) {
   if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
-  if (fp8 && s->T > kSwapMaxT) return MOE_ERR_UNSUPPORTED;
   if (s->T == 0) return MOE_OK;
   if (!ok16(x) || !ok4(w_g) || (bias && !aligned(bias, 4)) || !ok16(w13) || !ok16(w2) ||
       !ok16(y) || (idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4)) ||
@@ -227,12 +226,13 @@ static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const flo
     if (s->T <= kFusedRouteMaxT) {
       e = launch_route_fused(logits, *s, idx, gw, counts, offsets, at<int>(ws, L.tiles),
                              at<int>(ws, L.send), at<int>(ws, L.rank_off), row_of, perm,
-                             at<int>(ws, L.err), cs);
+                             at<int>(ws, L.err), cs, fp8 ? 0 : -1);
     } else {
       e = launch_topk(logits, *s, idx, gw, cs);
       if (e == cudaSuccess)
         e = launch_route_tables(idx, *s, L, wsb, counts, offsets, row_of, perm,
-                                at<int>(ws, L.send), at<int>(ws, L.rank_off), cs);
+                                at<int>(ws, L.send), at<int>(ws, L.rank_off), cs,
+                                fp8 ? 0 : -1);
     }
   }
   if (e == cudaSuccess)
@@ -269,7 +269,6 @@ int moe_ffn_fp8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w
                 const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                 const moe_shape* s, moe_bf16* z, void* ws, void* stream) {
   if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
-  if (s->T > kSwapMaxT) return MOE_ERR_UNSUPPORTED;
   if (s->T == 0) return MOE_OK;
   if (!ok16(x_perm) || !ok4(offsets) || !ok16(w13) || !ok4(w13_scale) || !ok16(w2) ||
       !ok4(w2_scale) || !ok16(z) || !ws || !aligned(ws, 256))
@@ -280,7 +279,7 @@ int moe_ffn_fp8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(*s, sms);
   cudaError_t e = launch_tiles_from_offsets(offsets, *s, at<int>(ws, L.tiles),
-                                            at<int>(ws, L.err), cs);
+                                            at<int>(ws, L.err), cs, 0);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return launch_expert_ffn_fp8(reinterpret_cast<const __nv_bfloat16*>(x_perm), L.P, w13,
                                w13_scale, w2, w2_scale, *s, L, static_cast<char*>(ws),

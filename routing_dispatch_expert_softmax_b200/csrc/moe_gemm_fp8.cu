@@ -16,12 +16,17 @@
 //
 // Same work items and roles as the bf16 swap-AB kernel (weights are the M = 128
 // operand, the expert's token rows the N operand), plus a converter warpgroup:
-//   warp 0      TMA producer of the raw e4m3 weight tiles (128 rows x 64 bytes,
-//               unswizzled) into a deep ring;
-//   warps 6-9   widen each raw tile to bf16 (exact: every E4M3 value is a bf16
-//               value) and write it 128-byte swizzled, K-major, into a short
-//               ring of MMA stages; one of them loads the stage's token tile;
-//   warp 1      owns TMEM and issues tcgen05.mma kind::f16 on the MMA stages;
+//   warp 0      TMA producer: each raw stage receives the e4m3 weight tile
+//               (128 rows x 64 bytes, unswizzled) and, beside it, the stage's
+//               bf16 token tile (128-byte swizzled, the MMA layout), so both
+//               stream through the same deep ring;
+//   warps 6-9   widen each raw weight tile to bf16 (exact: every E4M3 value is
+//               a bf16 value) and write it 128-byte swizzled, K-major, into a
+//               short ring of converted-weight stages;
+//   warp 1      owns TMEM and issues tcgen05.mma kind::f16 with A = converted
+//               weights, B = the token tile still in its raw stage; a raw
+//               stage is free once the four converter warps and the MMA are
+//               done with it;
 //   warps 2-5   drain the accumulator, apply the row scales (and SwiGLU), store.
 // Activations stay bf16, so the result is the bf16 path's arithmetic applied to
 // the dequantised weights.  Every wait is bounded (error word MOE_ERR_TIMEOUT,
@@ -35,23 +40,23 @@ namespace {
 
 template <int NMAX, bool SWIGLU>
 struct F8Cfg {
-  // Raw e4m3 weight tiles in flight (8 KB each: 96 / 80 KB, near the 112 KB of
-  // weights the bf16 kernel keeps in flight).  The token tile of a stage is
-  // loaded only once its MMA stage is free, so at most kMmaStages token loads
-  // are in flight.
-  static constexpr int kRawStages = NMAX <= 64 ? 12 : 10;
-  static constexpr int kMmaStages = 3;
-  static constexpr int kRawBytes = 128 * kGemmBK;         // 8 KB of e4m3
-  static constexpr int kWBytes = 128 * kGemmBK * 2;       // 16 KB of bf16
+  // Raw stages in flight: 9 x (8 KB e4m3 + 8 KB tokens) at NMAX = 64,
+  // 6 x (8 + 16 KB) at NMAX = 128; two converted-weight stages.
+  static constexpr int kRawStages = NMAX <= 64 ? 9 : 6;
+  static constexpr int kMmaStages = 2;
+  static constexpr int kRawWBytes = 128 * kGemmBK;        // 8 KB of e4m3
   static constexpr int kXBytes = NMAX * kGemmBK * 2;      // token rows, bf16
-  static constexpr int kMmaBytes = kWBytes + kXBytes;
+  static constexpr int kRawBytes = kRawWBytes + kXBytes;  // one raw stage
+  static constexpr int kWBytes = 128 * kGemmBK * 2;       // 16 KB of bf16
+  static constexpr int kMmaBytes = kWBytes;
   static constexpr int kTmemCols = 2 * NMAX;
   static constexpr int kXchBytes = SWIGLU ? 2 * 64 * 16 * 4 : 0;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes =
       kMmaStages * kMmaBytes + kRawStages * kRawBytes + kXchBytes + kBarBytes + 1024;
   static constexpr int kThreads = 320;
-  static_assert(8 * (2 * kRawStages + 3 * kMmaStages + 5) + 8 <= kBarBytes, "barriers");
+  static_assert(8 * (2 * kRawStages + 2 * kMmaStages + 5) + 8 <= kBarBytes, "barriers");
+  static_assert(kRawBytes % 1024 == 0 && kWBytes % 1024 == 0, "swizzled tiles 1024-aligned");
 };
 
 __device__ __forceinline__ bool wait_limit(uint64_t* bar, uint32_t parity,
@@ -110,14 +115,13 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* mma_st = smem;                                  // MS x (bf16 W | tokens)
-  uint8_t* raw_st = smem + MS * C::kMmaBytes;              // RS x e4m3 W
+  uint8_t* mma_st = smem;                                  // MS x bf16 W
+  uint8_t* raw_st = smem + MS * C::kMmaBytes;              // RS x (e4m3 W | bf16 tokens)
   float* xch = reinterpret_cast<float*>(raw_st + RS * C::kRawBytes);
   uint64_t* rfull = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + C::kXchBytes);
-  uint64_t* rempty = rfull + RS;
+  uint64_t* rempty = rfull + RS;   // 4 converter warps + the MMA commit
   uint64_t* wfull = rempty + RS;   // converted weights written (4 converter warps)
-  uint64_t* xfull = wfull + MS;    // token tile landed (TMA)
-  uint64_t* mempty = xfull + MS;   // MMA stage free (tcgen05.commit)
+  uint64_t* mempty = wfull + MS;   // converted-weight stage free (tcgen05.commit)
   uint64_t* tfull = mempty + MS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
@@ -128,11 +132,10 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
   if (threadIdx.x == 0) {
     for (int s2 = 0; s2 < RS; ++s2) {
       mbar_init(&rfull[s2], 1);
-      mbar_init(&rempty[s2], 4);
+      mbar_init(&rempty[s2], 5);
     }
     for (int s2 = 0; s2 < MS; ++s2) {
       mbar_init(&wfull[s2], 4);
-      mbar_init(&xfull[s2], 1);
       mbar_init(&mempty[s2], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -167,8 +170,9 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ e4m3 weight producer
+      // ------------------------------------------------ producer: e4m3 weights + tokens
       const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
       int fills[RS];
 #pragma unroll
       for (int s2 = 0; s2 < RS; ++s2) fills[s2] = 0;
@@ -177,9 +181,11 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
+        const int row0 = et[3 * i + 0];
         const int n = item_rows(i);
         const int e = et[3 * i + 2];
         if (n < 1 || n > NMAX) continue;  // recorded by the epilogue
+        const int nb = (n + 15) >> 4;
         const int wrow = e * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&rempty[stage], phase ^ 1u, abort_flag)) {
@@ -187,7 +193,8 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
             break;
           }
           uint8_t* dst = raw_st + stage * C::kRawBytes;
-          mbar_arrive_expect_tx(&rfull[stage], (uint32_t)C::kRawBytes);
+          uint8_t* xdst = dst + C::kRawWBytes;
+          mbar_arrive_expect_tx(&rfull[stage], (uint32_t)(C::kRawWBytes + nb * 16 * 128));
           if (SWIGLU) {
             tma_load_2d(dst, &tmW, &rfull[stage], kb * kGemmBK, wrow, pol_w);
             tma_load_2d(dst + 64 * kGemmBK, &tmW, &rfull[stage], kb * kGemmBK, wrow + up_offset,
@@ -195,6 +202,9 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
           } else {
             tma_load_2d(dst, &tmW, &rfull[stage], kb * kGemmBK, wrow, pol_w);
           }
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d(xdst + b * 16 * 128, &tmX, &rfull[stage], kb * kGemmBK, row0 + 16 * b,
+                        pol_x);
           ++fills[stage];
           if (++stage == RS) {
             stage = 0;
@@ -211,8 +221,8 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, rs = 0;
+      uint32_t phase = 0, rph = 0;
       int it = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
@@ -230,21 +240,26 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
         const uint32_t d_tmem = tmem_base + (uint32_t)(ab * NMAX);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&wfull[stage], phase, abort_flag) ||
-              !mbar_wait_bounded(&xfull[stage], phase, abort_flag)) {
+              !mbar_wait_bounded(&rfull[rs], rph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(mma_st + stage * C::kMmaBytes);
-          const uint32_t b_addr = a_addr + C::kWBytes;
+          const uint32_t b_addr = smem_u32(raw_st + rs * C::kRawBytes + C::kRawWBytes);
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 16; ++kk)
             umma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
                          sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(&mempty[stage]);
+          umma_commit(&rempty[rs]);  // the raw stage's token tile is read
           if (++stage == MS) {
             stage = 0;
             phase ^= 1u;
+          }
+          if (++rs == RS) {
+            rs = 0;
+            rph ^= 1u;
           }
         }
         if (ok) umma_commit(&tfull[ab]);
@@ -257,32 +272,19 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
   } else if (warp >= 6) {
     // ------------------------------------------------ converters (warps 6..9)
     const int ct = threadIdx.x - 192;  // 0..127
-    const uint64_t pol_x = policy_evict_last();
-    int xfills[MS];
-#pragma unroll
-    for (int s2 = 0; s2 < MS; ++s2) xfills[s2] = 0;
     int rs = 0, ms = 0;
     uint32_t rph = 0, mph = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int i = w / n_tiles;
-      const int row0 = et[3 * i + 0];
       const int n = item_rows(i);
       if (n < 1 || n > NMAX) continue;
-      const int nb = (n + 15) >> 4;
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait_bounded(&mempty[ms], mph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         uint8_t* wdst = mma_st + ms * C::kMmaBytes;
-        if (ct == 0) {
-          uint8_t* xdst = wdst + C::kWBytes;
-          mbar_arrive_expect_tx(&xfull[ms], (uint32_t)(nb * 16 * 128));
-          for (int b = 0; b < nb; ++b)
-            tma_load_2d(xdst + b * 16 * 128, &tmX, &xfull[ms], kb * kGemmBK, row0 + 16 * b, pol_x);
-          ++xfills[ms];
-        }
         if (!mbar_wait_bounded(&rfull[rs], rph, abort_flag)) {
           ok = false;
           break;
@@ -323,11 +325,6 @@ __global__ void __launch_bounds__(320, 1) k_expert_gemm_swap_f8(
           mph ^= 1u;
         }
       }
-    }
-    if (ct == 0 && *abort_flag) {
-#pragma unroll
-      for (int s2 = 0; s2 < MS; ++s2)
-        if (xfills[s2] > 0) wait_limit(&xfull[s2], (uint32_t)((xfills[s2] - 1) & 1), 100000000ull);
     }
   } else {
     // ------------------------------------------------ epilogue (warps 2..5)
@@ -484,7 +481,6 @@ int launch_expert_ffn_fp8(const __nv_bfloat16* x_perm, long long x_rows, const u
                           const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                           const moe_shape& s, const WsLayout& L, char* ws, __nv_bfloat16* z,
                           int num_sms, cudaStream_t st, void* const* events) {
-  if (s.T > kSwapMaxT) return MOE_ERR_UNSUPPORTED;
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
     return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,

@@ -17,15 +17,19 @@ cudaError_t launch_topk(const float* logits, const moe_shape& s, int* idx, float
                         cudaStream_t st);
 // Selection + dispatch tables in one block; valid for T <= kFusedRouteMaxT.
 constexpr int kFusedRouteMaxT = 1024;
+// `pair`: 1 = the work lists of the CTA-pair expert GEMMs (tile pairs plus a
+// leftover list), 0 = plain 128-row tiles, -1 = pair_tiles(s) (the bf16 GEMMs'
+// choice; the FP8 GEMMs always take plain tiles).
 cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
                                int* counts, int* offsets, int* tiles, int* send,
                                int* rank_off, int* row_of, int* perm, int* err,
-                               cudaStream_t st);
+                               cudaStream_t st, int pair = -1);
 cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayout& L,
                                 char* ws, int* counts, int* offsets, int* row_of,
-                                int* perm, int* send, int* rank_off, cudaStream_t st);
+                                int* perm, int* send, int* rank_off, cudaStream_t st,
+                                int pair = -1);
 cudaError_t launch_tiles_from_offsets(const int* offsets, const moe_shape& s,
-                                      int* tiles, int* err, cudaStream_t st);
+                                      int* tiles, int* err, cudaStream_t st, int pair = -1);
 cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, int T,
                           int d, __nv_bfloat16* x_perm, int* err, cudaStream_t st);
 cudaError_t launch_selftest_bounded_wait(unsigned long long limit_ns, int* err,
@@ -39,7 +43,8 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       void* const* events = nullptr);
 
 // The same two GEMMs with E4M3 expert weights and one fp32 scale per weight
-// row (moe_gemm_fp8.cu); small batches (T <= kSwapMaxT) only.
+// row (moe_gemm_fp8.cu): swap-AB form at every batch size, over the plain
+// 128-row tile list above 64 tokens.
 int launch_expert_ffn_fp8(const __nv_bfloat16* x_perm, long long x_rows, const uint8_t* w13,
                           const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                           const moe_shape& s, const WsLayout& L, char* ws, __nv_bfloat16* z,

@@ -940,7 +940,7 @@ template <int VPL>
 static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R, int chunk,
                                  size_t smem, int* idx, float* w, int* counts, int* offsets,
                                  int* tiles, int* send, int* rank_off, int* row_of, int* perm,
-                                 int* err, cudaStream_t st) {
+                                 int* err, int pair, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_route_fused<VPL>,
@@ -953,13 +953,14 @@ static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R,
   const unsigned blocks = (unsigned)((s.T + kFusedSelTokens - 1) / kFusedSelTokens);
   return launch_kernel(k_route_fused<VPL>, dim3(blocks), dim3(1024), smem, st, 1, logits, s.T,
                        s.E, s.k, R, chunk, idx, w, counts, offsets, tiles, send, rank_off, row_of,
-                       perm, err, err + kRouteTicket, pair_tiles(s) ? 1 : 0);
+                       perm, err, err + kRouteTicket, pair);
 }
 
 cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
                                int* counts, int* offsets, int* tiles, int* send,
                                int* rank_off, int* row_of, int* perm, int* err,
-                               cudaStream_t st) {
+                               cudaStream_t st, int pair) {
+  if (pair < 0) pair = pair_tiles(s) ? 1 : 0;
   const int R = s.R > 1 ? s.R : 0;
   const int chunk = R ? (s.T + R - 1) / R : 1;
   const long long tk = (long long)s.T * s.k;
@@ -968,14 +969,16 @@ cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx
   const int vpl = (s.E + 31) / 32;
 #define MOE_FUSED_CALL(V)                                                                 \
   return route_fused_t<V>(logits, s, R, chunk, smem, idx, w, counts, offsets, tiles, send, \
-                          rank_off, row_of, perm, err, st)
+                          rank_off, row_of, perm, err, pair, st)
   MOE_VPL_DISPATCH(vpl, MOE_FUSED_CALL);
 #undef MOE_FUSED_CALL
 }
 
 cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayout& L,
                                 char* ws, int* counts, int* offsets, int* row_of,
-                                int* perm, int* send, int* rank_off, cudaStream_t st) {
+                                int* perm, int* send, int* rank_off, cudaStream_t st,
+                                int pair) {
+  if (pair < 0) pair = pair_tiles(s) ? 1 : 0;
   int* err = reinterpret_cast<int*>(ws + L.err);
   int* blockhist = reinterpret_cast<int*>(ws + L.blockhist);
   int* blockbase = reinterpret_cast<int*>(ws + L.blockbase);
@@ -988,8 +991,7 @@ cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayo
                                 st, 1, idx, s.T, s.E, s.k, R, chunk, blockhist, blocksend, err);
   if (e != cudaSuccess) return e;
   e = launch_kernel(k_scan, dim3(1), dim3(1024), 0, st, 1, blockhist, L.nblocks, s.E, R,
-                    blocksend, blockbase, counts, offsets, tiles, send, rank_off,
-                    pair_tiles(s) ? 1 : 0);
+                    blocksend, blockbase, counts, offsets, tiles, send, rank_off, pair);
   if (e != cudaSuccess) return e;
   const size_t scat_smem = sizeof(uint32_t) * (kTokensPerRouteBlock / 32) * s.E;
   return launch_kernel(k_scatter, dim3(L.nblocks), dim3(kTokensPerRouteBlock), scat_smem, st, 1,
@@ -997,9 +999,10 @@ cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayo
 }
 
 cudaError_t launch_tiles_from_offsets(const int* offsets, const moe_shape& s,
-                                      int* tiles, int* err, cudaStream_t st) {
+                                      int* tiles, int* err, cudaStream_t st, int pair) {
+  if (pair < 0) pair = pair_tiles(s) ? 1 : 0;
   return launch_kernel(k_tiles_from_offsets, dim3(1), dim3(1024), 0, st, 1, offsets, s.E,
-                       (int)((long long)s.T * s.k), tiles, err, pair_tiles(s) ? 1 : 0);
+                       (int)((long long)s.T * s.k), tiles, err, pair);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, int T,

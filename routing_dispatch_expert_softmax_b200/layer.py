@@ -104,7 +104,7 @@ class MoELayer:
 
     FP8 experts: pass w13 / w2 as uint8 E4M3 codes of the same shapes with
     ``w13_scale`` (E, 2f) and ``w2_scale`` (E, d) fp32 row scales; the layer
-    then runs moe_forward_fp8 (batches of up to 256 tokens)."""
+    then runs moe_forward_fp8."""
 
     def __init__(self, w_g: torch.Tensor, bias: Optional[torch.Tensor],
                  w13: torch.Tensor, w2: torch.Tensor, k: int, R: int = 0,

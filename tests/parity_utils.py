@@ -115,3 +115,24 @@ class LazyExperts:
 
     def __getitem__(self, e):
         return self.t[int(e)].float().cpu().numpy().astype(np.float64)
+
+
+def token_sample(n=256, seed=0):
+    """A seeded sample of n tokens of the batch that always includes tokens
+    routed to the two hottest and the four coldest touched experts (the
+    first two and the last token of each), and the first and last token."""
+    def pick(idx_h, counts):
+        rng = np.random.default_rng(seed)
+        T = idx_h.shape[0]
+        touched = np.nonzero(counts)[0]
+        order = touched[np.argsort(-counts[touched], kind="stable")]
+        must = {0, T - 1}
+        for e in np.concatenate([order[:2], order[-4:]]):
+            toks = np.nonzero((idx_h == e).any(1))[0]
+            must.update(int(t) for t in toks[:2])
+            must.add(int(toks[-1]))
+        must = np.array(sorted(must), dtype=np.int64)
+        rest = np.setdiff1d(np.arange(T), must)
+        fill = rng.choice(rest, size=max(0, min(n - must.size, rest.size)), replace=False)
+        return np.unique(np.concatenate([must, fill]))
+    return pick

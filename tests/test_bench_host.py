@@ -37,8 +37,11 @@ def test_launch_counts_match_the_profiled_launch_lists():
     # profiles/launches_qwen3_decode_T64.md: 6 kernels per layer call;
     # profiles/launches_qwen3_prefill_T8192.md: 13 (split router with a
     # finish kernel, four routing kernels, gather, two pair GEMMs each with
-    # its lone-tile kernel, combine).
+    # its lone-tile kernel, combine); the FP8 layer runs its two 128-row-tile
+    # GEMMs at every batch size (11 at prefill).
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE) == 6
+    assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE, fp8=True) == 6
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_PREFILL) == 13
+    assert bench.launches_per_forward(wl.QWEN3_30B_A3B_PREFILL, fp8=True) == 11
     # replicas: top-k, remap, histogram, scan, scatter instead of the fused kernel
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE, eplb_redundant=16) == 10

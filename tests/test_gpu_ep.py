@@ -100,7 +100,7 @@ def _emulated_exchange(layers, xs):
 @pytest.mark.parametrize("cfg,R,T_of", [
     (wl.MoEConfig("ep-small", T=1, d=256, E=16, k=4, f=256, zipf_s=1.2), 4, lambda r: 9 + 7 * r),
     (wl.DEEPSEEK_V3_ROUTED, 8, lambda r: 8),
-    (wl.QWEN3_30B_A3B_DECODE, 2, lambda r: 200 + 50 * r),
+    (wl.QWEN3_30B_A3B_DECODE, 2, lambda r: 90 + 20 * r),
 ], ids=["small", "deepseek-8x8", "qwen-2ranks"])
 def test_emulated_ranks_match_the_single_gpu_layer(cfg, R, T_of):
     xs, w_g, bias, w13, w2, layers = _ranks(cfg, R, T_of)

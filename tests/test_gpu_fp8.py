@@ -16,8 +16,8 @@ import routing_dispatch_expert_softmax_b200 as moe
 from routing_dispatch_expert_softmax_b200 import workloads as wl
 from routing_dispatch_expert_softmax_b200.binding import MoEShape
 
-from parity_utils import (assert_layer_close, logit_bound, np64, order_by_logit,
-                          selection_is_valid, unique_selection)
+from parity_utils import (assert_layer_close, logit_bound, logit_bound_tensor_cores, np64,
+                          order_by_logit, selection_is_valid, token_sample, unique_selection)
 
 pytestmark = pytest.mark.gpu
 
@@ -102,11 +102,18 @@ def _forward_fp8_case(cfg, sample=None, seed=0):
     moe.moe_forward_fp8(x, w_g, bias, c13, s13, c2, s2, y, shape, ws, idx_out=idx, w_out=gw)
     _check_clean(ws)
     idx_h = idx.cpu().numpy()
-    toks = np.arange(cfg.T) if sample is None else sample
+    if sample is None:
+        toks = np.arange(cfg.T)
+    elif callable(sample):
+        toks = sample(idx_h, oracle.expert_counts(idx_h, cfg.E))
+    else:
+        toks = sample
     x64 = np64(x[torch.from_numpy(toks).long().to(DEV)])
     wg64, b64 = np64(w_g), None if bias is None else np64(bias)
     L64 = oracle.router_logits(x64, wg64, b64)
-    delta = logit_bound(x64, wg64, b64)
+    # above 256 tokens the router runs on the tensor cores
+    bound = logit_bound_tensor_cores if cfg.T > 256 else logit_bound
+    delta = bound(x64, wg64, b64)
     sel = []
     for i, t in enumerate(toks):
         g = idx_h[t].tolist()
@@ -137,15 +144,38 @@ def test_forward_fp8_deepseek(T):
     _forward_fp8_case(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=sample)
 
 
-def test_forward_fp8_rejects_large_batches():
-    cfg = wl.QWEN3_30B_A3B_DECODE.with_T(257)
+@pytest.mark.parametrize("cfg", [wl.QWEN3_30B_A3B_DECODE.with_T(257),
+                                 wl.QWEN3_30B_A3B_PREFILL,
+                                 wl.DEEPSEEK_V3_ROUTED.with_T(512)], ids=lambda c: c.name)
+def test_forward_fp8_large_batches(cfg):
+    # above 256 tokens: tensor-core router, plain 128-row token tiles (an
+    # expert with more rows is several work items); a 256-token sample with
+    # tokens of the hottest and coldest experts
+    _forward_fp8_case(cfg, sample=None if cfg.T <= 257 else token_sample())
+
+
+def test_ffn_fp8_large_batch_ragged_tiles():
+    # caller offsets: experts of 0, 1, 127, 128, 129, 300 and 640 rows
+    counts = np.array([0, 1, 127, 128, 129, 300, 640], dtype=np.int64)
+    E, P = counts.size, int(counts.sum())
+    cfg = wl.MoEConfig("fp8-tiles", T=P, d=256, E=E, k=1, f=384)
+    x_perm = wl.make_hidden(cfg, DEV, 3)
+    c13, s13, c2, s2 = wl.make_experts_fp8(cfg, DEV, 3)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     shape = MoEShape.from_config(cfg)
-    c13, s13, c2, s2 = wl.make_experts_fp8(wl.TINY, DEV, 0)  # never read
-    x = torch.zeros(cfg.T, cfg.d, dtype=torch.bfloat16, device=DEV)
-    w_g = torch.zeros(cfg.d, cfg.E, device=DEV)
-    with pytest.raises(moe.MoEError) as ei:
-        moe.moe_forward_fp8(x, w_g, None, c13, s13, c2, s2, x, shape, moe.workspace(shape))
-    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+    ws = moe.workspace(shape)
+    z = torch.empty(P, cfg.d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn_fp8(x_perm, torch.from_numpy(offsets).to(DEV), c13, s13, c2, s2, z, shape, ws)
+    _check_clean(ws)
+    xp = np64(x_perm)
+    ref = np.zeros((P, cfg.d))
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if b > a:
+            w13 = oracle.dequantise_rows(c13[e].cpu().numpy(), s13[e].cpu().numpy())
+            w2 = oracle.dequantise_rows(c2[e].cpu().numpy(), s2[e].cpu().numpy())
+            ref[a:b] = oracle.swiglu_ffn(xp[a:b], w13, w2)
+    assert_layer_close(z, ref, "moe_ffn_fp8 tiles")
 
 
 def test_forward_fp8_graph_replay_is_deterministic():

@@ -20,7 +20,7 @@ from routing_dispatch_expert_softmax_b200.binding import MoEShape
 
 from parity_utils import (LazyExperts, assert_layer_close, logit_bound,
                           logit_bound_tensor_cores, np64, order_by_logit,
-                          selection_is_valid, unique_selection)
+                          selection_is_valid, token_sample, unique_selection)
 
 ROUTER_TC_MIN_T = 257  # from this batch size the router runs on the tensor cores
 
@@ -414,33 +414,12 @@ def test_forward_qwen_decode(T):
     _check_forward(wl.QWEN3_30B_A3B_DECODE.with_T(T))
 
 
-def _token_sample(n=256, seed=0):
-    """A seeded sample of n tokens of the batch that always includes tokens
-    routed to the two hottest and the four coldest touched experts (the
-    first two and the last token of each), and the first and last token."""
-    def pick(idx_h, counts):
-        rng = np.random.default_rng(seed)
-        T = idx_h.shape[0]
-        touched = np.nonzero(counts)[0]
-        order = touched[np.argsort(-counts[touched], kind="stable")]
-        must = {0, T - 1}
-        for e in np.concatenate([order[:2], order[-4:]]):
-            toks = np.nonzero((idx_h == e).any(1))[0]
-            must.update(int(t) for t in toks[:2])
-            must.add(int(toks[-1]))
-        must = np.array(sorted(must), dtype=np.int64)
-        rest = np.setdiff1d(np.arange(T), must)
-        fill = rng.choice(rest, size=max(0, min(n - must.size, rest.size)), replace=False)
-        return np.unique(np.concatenate([must, fill]))
-    return pick
-
-
 def test_forward_qwen_prefill_sampled():
-    _check_forward(wl.QWEN3_30B_A3B_PREFILL, sample=_token_sample())
+    _check_forward(wl.QWEN3_30B_A3B_PREFILL, sample=token_sample())
 
 
 def test_forward_mixtral_sampled():
-    _check_forward(wl.MIXTRAL_8X7B, sample=_token_sample())
+    _check_forward(wl.MIXTRAL_8X7B, sample=token_sample())
 
 
 @pytest.mark.parametrize("T", [1, 64, 512, 16384])
@@ -449,7 +428,7 @@ def test_forward_deepseek(T):
     # T = 16384: multi-block routing tables and CTA-pair tiles with E = 256;
     # both on a 256-token sample that includes tokens routed to the hottest
     # and the coldest experts.
-    _check_forward(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=None if T <= 64 else _token_sample())
+    _check_forward(wl.DEEPSEEK_V3_ROUTED.with_T(T), sample=None if T <= 64 else token_sample())
 
 
 @pytest.mark.parametrize("cfg", [
