@@ -252,8 +252,10 @@ def swiglu_ffn(X, w13_e, w2_e):
     return (silu(g) * u) @ w2_e.T
 
 
-def expert_outputs(x, perm, offsets, w13, w2):
-    """Run every expert's FFN over its contiguous rows; returns Z (P, d)."""
+def expert_outputs(x, perm, offsets, w13, w2, ffn=None):
+    """Run every expert's FFN (``ffn``, default swiglu_ffn) over its
+    contiguous rows; returns Z (P, d)."""
+    ffn = swiglu_ffn if ffn is None else ffn
     x = _f64(x)
     offsets = np.asarray(offsets, dtype=np.int64)
     E = offsets.shape[0] - 1
@@ -262,8 +264,7 @@ def expert_outputs(x, perm, offsets, w13, w2):
     for e in range(E):
         a, b = int(offsets[e]), int(offsets[e + 1])
         if b > a:
-            Z[a:b] = swiglu_ffn(x[np.asarray(perm[a:b], dtype=np.int64)],
-                                w13[e], w2[e])
+            Z[a:b] = ffn(x[np.asarray(perm[a:b], dtype=np.int64)], w13[e], w2[e])
     return Z
 
 
@@ -295,7 +296,7 @@ def imbalance_factor(counts, R):
 
 
 def moe_forward(x, w_g, bias, w13, w2, k, R=0, select_dtype=np.float32,
-                idx=None):
+                idx=None, ffn=None):
     """The whole layer, step by step, in the order the pages describe it.
 
     1. router logits in fp64;
@@ -304,7 +305,8 @@ def moe_forward(x, w_g, bias, w13, w2, k, R=0, select_dtype=np.float32,
        (the tests pass oracle-made alternatives for near-ties here);
     3. gates from the fp64 logits;
     4. counts, offsets, dispatch rows (and the virtual-EP layout if R > 1);
-    5. expert SwiGLU FFNs on each expert's rows;
+    5. expert SwiGLU FFNs on each expert's rows (``ffn`` replaces
+       swiglu_ffn, e.g. with a quantised variant);
     6. gate-weighted combine.
     Returns a dict of every intermediate.
     """
@@ -324,7 +326,7 @@ def moe_forward(x, w_g, bias, w13, w2, k, R=0, select_dtype=np.float32,
     if R and R > 1:
         S, rank_offsets = virtual_ep_layout(idx, E, R)
         out.update(send_counts=S, rank_offsets=rank_offsets)
-    Z = expert_outputs(x, perm, offsets, w13, w2)
+    Z = expert_outputs(x, perm, offsets, w13, w2, ffn)
     out["z"] = Z
     out["y"] = combine(Z, row_of, w)
     return out

@@ -1,6 +1,6 @@
 // Small-batch expert GEMMs with FP8 (E4M3) expert weights.
 //
-// "Serving mixture-of-experts models: expert parallelism on H200", section
+// "Serving MoE models with expert parallelism on 8xH200", section
 // "Memory math for 8xH200": DeepSeek-V3 and the Qwen3 FP8 variants ship their
 // weights at one byte per parameter; section "Quantization choices": native FP8
 // checkpoints are the default; and its FAQ: each expert sees a small slice of
