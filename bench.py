@@ -8,7 +8,7 @@ tokens, d=2048, E=128 experts, top-8, f=768, Zipf(1.0) expert skew), the
 configuration the HBM-roofline metric is quoted on.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--T T] [--fp8]
+                  [--workload NAME] [--T T] [--fp8] [--w8a8]
 
 Device timing: W untimed steps, then K steps each bracketed by CUDA events on
 the launch stream (stage boundaries come from moe_forward_staged); L2 is
@@ -65,14 +65,16 @@ def router_launches(cfg):
     return 2 if parts == 1 else 3
 
 
-def launches_per_forward(cfg, eplb_redundant=0, fp8=False):
+def launches_per_forward(cfg, eplb_redundant=0, fp8=False, w8a8=False):
     """Kernels one moe_forward (moe_forward_eplb with eplb_redundant > 0,
-    moe_forward_fp8 with fp8) launches: the router (router_launches), routing
-    (one fused kernel for T <= 1024, else top-k + histogram + scan + scatter;
-    with replicas top-k + remap + histogram + scan + scatter), the row gather,
-    the two expert GEMMs (the bf16 ones each followed by the lone-tile kernel
-    when they run on CTA pairs; the FP8 ones always run the 128-row-tile form),
-    combine."""
+    moe_forward_fp8 with fp8, moe_forward_w8a8 with w8a8) launches: the router
+    (router_launches), routing (one fused kernel for T <= 1024, else top-k +
+    histogram + scan + scatter; with replicas top-k + remap + histogram + scan
+    + scatter), the row gather (with w8a8 the gather-and-quantise kernel), the
+    two expert GEMMs (the bf16 ones each followed by the lone-tile kernel when
+    they run on CTA pairs; the FP8 ones always run the 128-row-tile form; with
+    w8a8 the SwiGLU output's quantisation between them), combine."""
+    fp8 = fp8 or w8a8
     T = cfg.T
     routing = 1 if T <= 1024 else 4
     if eplb_redundant:
@@ -81,7 +83,7 @@ def launches_per_forward(cfg, eplb_redundant=0, fp8=False):
     gemms = 2
     if T > 256 and T * cfg.k >= 128 * (cfg.E + eplb_redundant) and not fp8:
         gemms = 4
-    return router_launches(cfg) + routing + gather + gemms + 1
+    return router_launches(cfg) + routing + gather + gemms + (1 if w8a8 else 0) + 1
 
 
 def parse_args(argv=None):
@@ -98,6 +100,9 @@ def parse_args(argv=None):
                         "single-GPU run appends to its line")
     p.add_argument("--fp8", action="store_true",
                    help="E4M3 expert weights with fp32 row scales")
+    p.add_argument("--w8a8", action="store_true",
+                   help="E4M3 expert weights and E4M3 activations (one power-of-two scale per "
+                        "row; both GEMM operands one byte); implies --fp8")
     p.add_argument("--ep", action="store_true",
                    help="expert parallelism over the launched ranks: each rank holds E/N whole "
                         "experts and its own batch; tokens are exchanged with NCCL all-to-all-v "
@@ -106,7 +111,10 @@ def parse_args(argv=None):
     p.add_argument("--eplb-redundant", type=int, default=0,
                    help="time the layer with this many redundant expert copies placed by "
                         "the EPLB-style plan (built from the counts of one warm-up call)")
-    return p.parse_args(argv)
+    args = p.parse_args(argv)
+    if args.w8a8:
+        args.fp8 = True
+    return args
 
 
 def load_peaks():
@@ -288,8 +296,13 @@ def cpu_threads():
 
 def oracle_sample_run(cfg, host, tokens):
     """One oracle pass over the given tokens of the batch (fp64, CPU); FP8
-    experts are dequantised by the oracle inside the pass."""
+    experts are dequantised by the oracle inside the pass (and with FP8
+    activations the rows quantised)."""
     import oracle
+    if host.get("w8a8"):
+        return oracle.moe_forward_w8a8(host["x"][tokens], host["w_g"], host["bias"],
+                                       host["w13"], host["w13_scale"], host["w2"],
+                                       host["w2_scale"], cfg.k)
     if "w13_scale" in host:
         return oracle.moe_forward_fp8(host["x"][tokens], host["w_g"], host["bias"], host["w13"],
                                       host["w13_scale"], host["w2"], host["w2_scale"], cfg.k)
@@ -316,7 +329,7 @@ def host_inputs_for_oracle(cfg, dev_inputs, tokens):
     fp8 = "w13_scale" in dev_inputs
     raw = (lambda t: t.cpu().numpy()) if fp8 else f32  # FP8: codes and scales as stored
     names = ("w13", "w2", "w13_scale", "w2_scale") if fp8 else ("w13", "w2")
-    host = {"x": x, "w_g": w_g, "bias": bias}
+    host = {"x": x, "w_g": w_g, "bias": bias, "w8a8": bool(dev_inputs.get("w8a8"))}
     for name in names:
         host[name] = Experts()
         for e in touched.tolist():
@@ -360,7 +373,7 @@ def run_reference(args):
     inputs = {"x": wl.make_hidden(cfg, dev, 0), "w_g": w_g, "bias": bias}
     if args.fp8:
         w13, s13, w2, s2 = wl.make_experts_fp8(cfg, dev, 0)
-        inputs.update(w13=w13, w13_scale=s13, w2=w2, w2_scale=s2)
+        inputs.update(w13=w13, w13_scale=s13, w2=w2, w2_scale=s2, w8a8=args.w8a8)
     else:
         inputs["w13"], inputs["w2"] = wl.make_experts(cfg, dev, 0)
     n = min(cfg.T, 8)
@@ -390,6 +403,8 @@ def run_reference(args):
     }
     if args.fp8:
         line["config"]["weights"] = "e4m3 codes, one fp32 scale per weight row"
+    if args.w8a8:
+        line["config"]["activations"] = "e4m3 codes, one power-of-two scale per row"
     print(json.dumps(line), flush=True)
     return 0
 
@@ -625,7 +640,8 @@ def run_ours(args):
     else:
         w13, w2 = wl.make_experts(cfg, dev, 0)
         s13 = s2 = None
-    layer = moe.MoELayer(w_g, bias, w13, w2, cfg.k, cfg.R, w13_scale=s13, w2_scale=s2)
+    layer = moe.MoELayer(w_g, bias, w13, w2, cfg.k, cfg.R, w13_scale=s13, w2_scale=s2,
+                         fp8_activations=args.w8a8)
     shape = layer.shape(cfg.T)
     ws = moe.workspace(shape, dev)
     y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
@@ -642,13 +658,17 @@ def run_ours(args):
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
     def fwd(out, **kw):  # the layer through the C ABI (bf16 or FP8 experts)
-        if args.fp8:
+        if args.w8a8:
+            moe.moe_forward_w8a8(x, w_g, bias, w13, s13, w2, s2, out, shape, ws, **kw)
+        elif args.fp8:
             moe.moe_forward_fp8(x, w_g, bias, w13, s13, w2, s2, out, shape, ws, **kw)
         else:
             moe.moe_forward(x, w_g, bias, w13, w2, out, shape, ws, **kw)
 
     def fwd_staged(events):
-        if args.fp8:
+        if args.w8a8:
+            moe.moe_forward_w8a8_staged(x, w_g, bias, w13, s13, w2, s2, y, shape, ws, events)
+        elif args.fp8:
             moe.moe_forward_fp8_staged(x, w_g, bias, w13, s13, w2, s2, y, shape, ws, events)
         else:
             moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, events)
@@ -780,7 +800,8 @@ def run_ours(args):
     alg = algorithmic(cfg, touched, args.fp8)
     mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
     roof = kernel_roofline(cfg, alg, mean_stage, peaks, peak_src,
-                           f"{cfg.name}@T{cfg.T}" + ("/fp8" if args.fp8 else ""))
+                           f"{cfg.name}@T{cfg.T}" +
+                           ("/w8a8" if args.w8a8 else "/fp8" if args.fp8 else ""))
     layer_roof = layer_roofline(cfg, alg, touched, ms_per_step, peaks)
 
     line = {
@@ -802,12 +823,16 @@ def run_ours(args):
                          "(each adds a few us); the headline uses plain graph replays",
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * cfg.d * 2,
                 "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-        "gpu_launches": 2 * launches_per_forward(cfg, fp8=args.fp8) * args.steps,
+        "gpu_launches": 2 * launches_per_forward(cfg, fp8=args.fp8,
+                                                 w8a8=args.w8a8) * args.steps,
         "clocks": clk,
     }
     if args.fp8:
         line["config"]["weights"] = "e4m3 codes, one fp32 scale per weight row"
         line["dtype"] = "bf16 (tensor-core operands; expert weights stored e4m3)"
+    if args.w8a8:
+        line["config"]["activations"] = "e4m3 codes, one power-of-two scale per row"
+        line["dtype"] = "e4m3 (both tensor-core operands; fp32 accumulation)"
     if dedup_info is not None:
         line["dispatch_volume"] = dedup_info
     if eplb_info is not None:
@@ -819,7 +844,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base_inputs = {"x": x, "w_g": w_g, "bias": bias, "w13": w13, "w2": w2}
         if args.fp8:
-            base_inputs.update(w13_scale=s13, w2_scale=s2)
+            base_inputs.update(w13_scale=s13, w2_scale=s2, w8a8=args.w8a8)
         line["cpu_baseline"] = cpu_baseline(cfg, base_inputs)
     default_run = (args.workload == DEFAULT_WORKLOAD and args.T is None and not args.fp8
                    and not args.eplb_redundant)

@@ -78,7 +78,8 @@ MOE_API const char* moe_error_string(int status);
 
 /* Library ABI version (major * 100 + minor): 101 adds the EPLB calls and
  * moe_dispatch_dedup; 102 the FP8-weight calls; 103 moe_ep_recv_experts and
- * FP8 weights at every batch size. */
+ * FP8 weights at every batch size; 104 the FP8-activation (W8A8) calls and
+ * moe_quantise_rows_e4m3 (the workspace grows by their buffers). */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -379,6 +380,51 @@ MOE_API int moe_forward_fp8_staged(const moe_bf16* x, const float* w_g, const fl
                                    const uint8_t* w2, const float* w2_scale,
                                    const moe_shape* s, moe_bf16* y, void* ws,
                                    void* const* events, void* stream);
+
+/* FP8 activations too (the W8A8 layer): both operands of both expert GEMMs
+ * are E4M3, so the tensor cores multiply one-byte codes (tcgen05 kind::f8f6f4)
+ * and the bytes streamed per weight are those of the codes alone.  The pages
+ * fix no activation format; this library's reading: each activation row gets
+ * one power-of-two scale and round-to-nearest-even codes, as
+ * moe_quantise_rows_e4m3 defines.  The token rows are quantised as they are
+ * gathered; GEMM1's SwiGLU output is rounded to bf16 (as in moe_ffn), then
+ * quantised row by row; each fp32 accumulator is multiplied by its weight
+ * row's scale and its token row's scale before SwiGLU / the bf16 store.
+ * Weights, scales, alignment and outputs as moe_ffn_fp8 / moe_forward_fp8;
+ * d and f multiples of 64 as everywhere (a K block of 128 codes past the
+ * end reads zeros).  Every batch size runs the swap-AB form (touched-expert
+ * items up to 64 tokens, 128-row token tiles above).
+ * moe_ffn_w8a8 quantises x_perm's P = T*k rows itself. */
+MOE_API int moe_ffn_w8a8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w13,
+                         const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                         const moe_shape* s, moe_bf16* z, void* ws, void* stream);
+
+MOE_API int moe_forward_w8a8(const moe_bf16* x, const float* w_g, const float* bias,
+                             const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
+                             const float* w2_scale, const moe_shape* s, moe_bf16* y,
+                             int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
+                             void* stream);
+
+/* moe_forward_w8a8 with the stage events of moe_forward_staged (the SwiGLU
+ * output's quantisation falls in the GEMM2 stage). */
+MOE_API int moe_forward_w8a8_staged(const moe_bf16* x, const float* w_g, const float* bias,
+                                    const uint8_t* w13, const float* w13_scale,
+                                    const uint8_t* w2, const float* w2_scale,
+                                    const moe_shape* s, moe_bf16* y, void* ws,
+                                    void* const* events, void* stream);
+
+/* Row quantisation of bf16 activations to E4M3 with power-of-two scales:
+ *   a      [rows, cols] bf16 in (finite values; non-finite rows unspecified)
+ *   codes  [rows, cols] uint8 out   E4M3 codes
+ *   scales [rows] fp32 out          2^e_r
+ * e_r is the smallest integer with max_c |a[r,c]| <= 448 * 2^e_r (0 for a
+ * row of zeros), and codes[r,c] the E4M3 value nearest to a[r,c] * 2^-e_r,
+ * ties to the even code; the sign bit is a's, also for values that round to
+ * zero.  a * 2^-e_r is exact, so the codes depend on a alone.  cols a
+ * multiple of 16 (16 to 2^20); a and codes 16-byte aligned, scales 4-byte.
+ * One warp per row; asynchronous on `stream`. */
+MOE_API int moe_quantise_rows_e4m3(const moe_bf16* a, int64_t rows, int32_t cols,
+                                   uint8_t* codes, float* scales, void* stream);
 
 /* Self-test of the failure path every device-side wait uses: launches one
  * kernel that waits on a barrier nothing will ever complete, through the same

@@ -36,7 +36,7 @@ from . import moe_oracle as _m
 
 __all__ = ["e4m3_decode", "dequantise_rows", "moe_forward_fp8", "LazyDequant",
            "e4m3_encode", "pow2_row_exponent", "quantise_rows_pow2", "bf16_round",
-           "moe_forward_w8a8"]
+           "moe_forward_w8a8", "w8a8_ffn"]
 
 E4M3_MAX = 448.0
 
@@ -152,7 +152,7 @@ def bf16_round(a):
     return np.ldexp(q, x - 8)
 
 
-def _w8a8_ffn(X, w13_e, w2_e):
+def w8a8_ffn(X, w13_e, w2_e):
     """One expert's SwiGLU FFN with both GEMM inputs quantised per row
     (fp64 arithmetic on the dequantised codes)."""
     cx, sx = quantise_rows_pow2(X)
@@ -171,7 +171,7 @@ def moe_forward_w8a8(x, w_g, bias, w13_codes, w13_scale, w2_codes, w2_scale, k, 
                      select_dtype=np.float32, idx=None):
     """The layer with FP8 expert weights and FP8 activations: routing, gates,
     dispatch and combine as in the bf16 layer; each expert row's FFN by
-    _w8a8_ffn on the dequantised weights."""
+    w8a8_ffn on the dequantised weights."""
     return _m.moe_forward(x, w_g, bias, LazyDequant(w13_codes, w13_scale),
                           LazyDequant(w2_codes, w2_scale), k, R=R,
-                          select_dtype=select_dtype, idx=idx, ffn=_w8a8_ffn)
+                          select_dtype=select_dtype, idx=idx, ffn=w8a8_ffn)

@@ -15,5 +15,6 @@ from .binding import (EXPORTS, MOE_STAGE_EVENTS, STAGE_NAMES, MOE_ERR_CUDA, MOE_
                       moe_workspace_size, workspace, moe_eplb_plan, moe_eplb_remap,
                       moe_workspace_size_eplb, workspace_eplb, moe_forward_eplb,
                       moe_dispatch_dedup, moe_ffn_fp8, moe_forward_fp8,
-                      moe_forward_fp8_staged, moe_ep_recv_experts)
+                      moe_forward_fp8_staged, moe_ep_recv_experts, moe_ffn_w8a8,
+                      moe_forward_w8a8, moe_forward_w8a8_staged, moe_quantise_rows_e4m3)
 from .layer import MoELayer  # noqa: F401

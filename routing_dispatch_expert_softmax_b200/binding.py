@@ -31,7 +31,9 @@ EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router"
            "moe_forward_staged", "moe_selftest_bounded_wait", "moe_check",
            "moe_dispatch_noalloc", "moe_eplb_plan", "moe_eplb_remap",
            "moe_workspace_size_eplb", "moe_forward_eplb", "moe_dispatch_dedup",
-           "moe_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_staged", "moe_ep_recv_experts")
+           "moe_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_staged", "moe_ep_recv_experts",
+           "moe_ffn_w8a8", "moe_forward_w8a8", "moe_forward_w8a8_staged",
+           "moe_quantise_rows_e4m3")
 
 
 class MoEError(RuntimeError):
@@ -114,6 +116,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_forward_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P]
     lib.moe_forward_fp8_staged.restype = ctypes.c_int
     lib.moe_forward_fp8_staged.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]
+    lib.moe_ffn_w8a8.restype = ctypes.c_int
+    lib.moe_ffn_w8a8.argtypes = [_P, _P, _P, _P, _P, _P, _S, _P, _P, _P]
+    lib.moe_forward_w8a8.restype = ctypes.c_int
+    lib.moe_forward_w8a8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P]
+    lib.moe_forward_w8a8_staged.restype = ctypes.c_int
+    lib.moe_forward_w8a8_staged.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]
+    lib.moe_quantise_rows_e4m3.restype = ctypes.c_int
+    lib.moe_quantise_rows_e4m3.argtypes = [_P, ctypes.c_int64, ctypes.c_int32, _P, _P, _P]
     _lib = lib
     return lib
 
@@ -362,6 +372,54 @@ def moe_forward_fp8(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoESha
         _ptr(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
         _ptr(w_out, torch.float32, "w_out"), _ptr(counts_out, torch.int32, "counts_out"),
         _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_forward_fp8")
+
+
+def moe_ffn_w8a8(x_perm, offsets, w13, w13_scale, w2, w2_scale, z, shape: MoEShape, ws,
+                 stream=None):
+    """Expert FFNs with E4M3 weights and E4M3 activations (the rows of x_perm
+    and the SwiGLU output quantised with power-of-two row scales)."""
+    _check(load_library().moe_ffn_w8a8(
+        _ptr(x_perm, torch.bfloat16, "x_perm"), _ptr(offsets, torch.int32, "offsets"),
+        _ptr(w13, torch.uint8, "w13"), _ptr(w13_scale, torch.float32, "w13_scale"),
+        _ptr(w2, torch.uint8, "w2"), _ptr(w2_scale, torch.float32, "w2_scale"),
+        ctypes.byref(shape), _ptr(z, torch.bfloat16, "z"), _ptr(ws, torch.uint8, "ws"),
+        _stream(stream)), "moe_ffn_w8a8")
+
+
+def moe_forward_w8a8(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoEShape, ws,
+                     idx_out=None, w_out=None, counts_out=None, stream=None):
+    """The whole layer with E4M3 expert weights and E4M3 activations."""
+    _check(load_library().moe_forward_w8a8(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.uint8, "w13"),
+        _ptr(w13_scale, torch.float32, "w13_scale"), _ptr(w2, torch.uint8, "w2"),
+        _ptr(w2_scale, torch.float32, "w2_scale"), ctypes.byref(shape),
+        _ptr(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
+        _ptr(w_out, torch.float32, "w_out"), _ptr(counts_out, torch.int32, "counts_out"),
+        _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_forward_w8a8")
+
+
+def moe_forward_w8a8_staged(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoEShape,
+                            ws, events, stream=None):
+    """moe_forward_w8a8 with the stage events of moe_forward_staged."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    arr = _event_array(events, st)
+    _check(load_library().moe_forward_w8a8_staged(
+        _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
+        _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.uint8, "w13"),
+        _ptr(w13_scale, torch.float32, "w13_scale"), _ptr(w2, torch.uint8, "w2"),
+        _ptr(w2_scale, torch.float32, "w2_scale"), ctypes.byref(shape),
+        _ptr(y, torch.bfloat16, "y"), _ptr(ws, torch.uint8, "ws"), arr, _stream(st)),
+        "moe_forward_w8a8_staged")
+
+
+def moe_quantise_rows_e4m3(a, codes, scales, stream=None):
+    """E4M3 codes (uint8, a's shape) and power-of-two row scales (fp32) of a
+    2-D bf16 tensor."""
+    rows, cols = int(a.shape[0]), int(a.shape[1])
+    _check(load_library().moe_quantise_rows_e4m3(
+        _ptr(a, torch.bfloat16, "a"), rows, cols, _ptr(codes, torch.uint8, "codes"),
+        _ptr(scales, torch.float32, "scales"), _stream(stream)), "moe_quantise_rows_e4m3")
 
 
 def moe_forward_fp8_staged(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoEShape, ws,

@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libmoe_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_gemm_sm100.cu", "moe_noalloc.cu",
+SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_gemm_sm100.cu", "moe_noalloc.cu", "moe_w8a8.cu",
            "moe_eplb.cu", "moe_dedup.cu", "moe_gemm_fp8.cu", "moe_ep.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

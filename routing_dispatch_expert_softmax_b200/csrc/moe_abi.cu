@@ -9,7 +9,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int kVersion = 103;
+constexpr int kVersion = 104;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
@@ -183,9 +183,13 @@ int moe_combine(const moe_bf16* z, const int32_t* row_of, const float* w, const 
                                     static_cast<cudaStream_t>(stream)));
 }
 
-// The whole layer: bf16 expert weights, or (fp8) E4M3 expert weights with one
-// fp32 scale per weight row (small batches only).
-static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const float* bias,
+// Expert weight / activation formats of the whole layer.
+enum : int { kBf16 = 0, kFp8Weights = 1, kW8A8 = 2 };
+
+// The whole layer: bf16 expert weights; E4M3 expert weights with one fp32
+// scale per weight row (kFp8Weights, bf16 tokens); or those weights with the
+// tokens and the SwiGLU output quantised to E4M3 too (kW8A8).
+static int forward_impl(int mode, const moe_bf16* x, const float* w_g, const float* bias,
                         const void* w13, const float* w13_scale, const void* w2,
                         const float* w2_scale, const moe_shape* s, moe_bf16* y,
                         int32_t* idx_out, float* w_out, int32_t* counts_out, void* ws,
@@ -195,8 +199,10 @@ static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const flo
   if (s->T == 0) return MOE_OK;
   if (!ok16(x) || !ok4(w_g) || (bias && !aligned(bias, 4)) || !ok16(w13) || !ok16(w2) ||
       !ok16(y) || (idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4)) ||
-      (counts_out && !aligned(counts_out, 4)) || (fp8 && (!ok4(w13_scale) || !ok4(w2_scale))))
+      (counts_out && !aligned(counts_out, 4)) ||
+      (mode != kBf16 && (!ok4(w13_scale) || !ok4(w2_scale))))
     return MOE_ERR_INVALID_ARG;
+  const bool fp8 = mode != kBf16;  // the plain 128-row tile list
   int sms = 0;
   int st = device_check(&sms);
   if (st != MOE_OK) return st;
@@ -235,16 +241,28 @@ static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const flo
                                 fp8 ? 0 : -1);
     }
   }
+  uint8_t* xq = at<uint8_t>(ws, L.x_perm);  // W8A8: token codes in the x_perm region
+  float* xs = at<float>(ws, L.xs);
   if (e == cudaSuccess)
-    e = launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
+    e = mode == kW8A8
+            ? launch_quant_rows(xb, perm, L.P, s->T, s->d, xq, xs, at<int>(ws, L.err), cs)
+            : launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
   if (e == cudaSuccess) e = mark(2);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  int r = fp8 ? launch_expert_ffn_fp8(x_perm, L.Ppad, static_cast<const uint8_t*>(w13),
-                                       w13_scale, static_cast<const uint8_t*>(w2), w2_scale,
-                                       *s, L, wsb, z, sms, cs, events ? events + 3 : nullptr)
-              : launch_expert_ffn(x_perm, L.Ppad, static_cast<const __nv_bfloat16*>(w13),
-                                  static_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms,
-                                  cs, events ? events + 3 : nullptr);
+  void* const* ev = events ? events + 3 : nullptr;
+  int r;
+  if (mode == kW8A8)
+    r = launch_expert_ffn_w8a8(xq, xs, L.Ppad, static_cast<const uint8_t*>(w13), w13_scale,
+                               static_cast<const uint8_t*>(w2), w2_scale, *s, L, wsb, z, sms, cs,
+                               ev, true);
+  else if (mode == kFp8Weights)
+    r = launch_expert_ffn_fp8(x_perm, L.Ppad, static_cast<const uint8_t*>(w13), w13_scale,
+                              static_cast<const uint8_t*>(w2), w2_scale, *s, L, wsb, z, sms, cs,
+                              ev);
+  else
+    r = launch_expert_ffn(x_perm, L.Ppad, static_cast<const __nv_bfloat16*>(w13),
+                          static_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms, cs, ev,
+                          true);
   if (r != MOE_OK) return r;
   e = launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs);
   if (e == cudaSuccess) e = mark(5);
@@ -254,14 +272,14 @@ static int forward_impl(bool fp8, const moe_bf16* x, const float* w_g, const flo
 int moe_forward(const moe_bf16* x, const float* w_g, const float* bias, const moe_bf16* w13,
                 const moe_bf16* w2, const moe_shape* s, moe_bf16* y, int32_t* idx_out,
                 float* w_out, int32_t* counts_out, void* ws, void* stream) {
-  return forward_impl(false, x, w_g, bias, w13, nullptr, w2, nullptr, s, y, idx_out, w_out,
+  return forward_impl(kBf16, x, w_g, bias, w13, nullptr, w2, nullptr, s, y, idx_out, w_out,
                       counts_out, ws, stream, nullptr);
 }
 
 int moe_forward_staged(const moe_bf16* x, const float* w_g, const float* bias,
                        const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
                        moe_bf16* y, void* ws, void* const* events, void* stream) {
-  return forward_impl(false, x, w_g, bias, w13, nullptr, w2, nullptr, s, y, nullptr, nullptr,
+  return forward_impl(kBf16, x, w_g, bias, w13, nullptr, w2, nullptr, s, y, nullptr, nullptr,
                       nullptr, ws, stream, events);
 }
 
@@ -290,15 +308,71 @@ int moe_forward_fp8(const moe_bf16* x, const float* w_g, const float* bias, cons
                     const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                     const moe_shape* s, moe_bf16* y, int32_t* idx_out, float* w_out,
                     int32_t* counts_out, void* ws, void* stream) {
-  return forward_impl(true, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, idx_out, w_out,
-                      counts_out, ws, stream, nullptr);
+  return forward_impl(kFp8Weights, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, idx_out,
+                      w_out, counts_out, ws, stream, nullptr);
 }
 
 int moe_forward_fp8_staged(const moe_bf16* x, const float* w_g, const float* bias,
                            const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
                            const float* w2_scale, const moe_shape* s, moe_bf16* y, void* ws,
                            void* const* events, void* stream) {
-  return forward_impl(true, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, nullptr, nullptr,
+  return forward_impl(kFp8Weights, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, nullptr,
+                      nullptr, nullptr, ws, stream, events);
+}
+
+int moe_quantise_rows_e4m3(const moe_bf16* a, int64_t rows, int32_t cols, uint8_t* codes,
+                           float* scales, void* stream) {
+  if (rows < 0 || cols < 16 || cols % 16 || cols > (1 << 20)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!ok16(a) || !ok16(codes) || !ok4(scales)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_quant_rows(reinterpret_cast<const __nv_bfloat16*>(a), nullptr, rows,
+                                       0, cols, codes, scales, nullptr,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ffn_w8a8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* w13,
+                 const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                 const moe_shape* s, moe_bf16* z, void* ws, void* stream) {
+  if (!shape_ok(s)) return MOE_ERR_INVALID_ARG;
+  if (s->T == 0) return MOE_OK;
+  if (!ok16(x_perm) || !ok4(offsets) || !ok16(w13) || !ok4(w13_scale) || !ok16(w2) ||
+      !ok4(w2_scale) || !ok16(z) || !ws || !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*s, sms);
+  uint8_t* xq = at<uint8_t>(ws, L.x_perm);
+  float* xs = at<float>(ws, L.xs);
+  // the work list first, so GEMM1 may read it before the quantisation completes
+  cudaError_t e = launch_tiles_from_offsets(offsets, *s, at<int>(ws, L.tiles),
+                                            at<int>(ws, L.err), cs, 0);
+  if (e == cudaSuccess)
+    e = launch_quant_rows(reinterpret_cast<const __nv_bfloat16*>(x_perm), nullptr, L.P, 0, s->d,
+                          xq, xs, at<int>(ws, L.err), cs);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_expert_ffn_w8a8(xq, xs, L.Ppad, w13, w13_scale, w2, w2_scale, *s, L,
+                                static_cast<char*>(ws), reinterpret_cast<__nv_bfloat16*>(z), sms,
+                                cs, nullptr, true);
+}
+
+int moe_forward_w8a8(const moe_bf16* x, const float* w_g, const float* bias, const uint8_t* w13,
+                     const float* w13_scale, const uint8_t* w2, const float* w2_scale,
+                     const moe_shape* s, moe_bf16* y, int32_t* idx_out, float* w_out,
+                     int32_t* counts_out, void* ws, void* stream) {
+  return forward_impl(kW8A8, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, idx_out, w_out,
+                      counts_out, ws, stream, nullptr);
+}
+
+int moe_forward_w8a8_staged(const moe_bf16* x, const float* w_g, const float* bias,
+                            const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
+                            const float* w2_scale, const moe_shape* s, moe_bf16* y, void* ws,
+                            void* const* events, void* stream) {
+  return forward_impl(kW8A8, x, w_g, bias, w13, w13_scale, w2, w2_scale, s, y, nullptr, nullptr,
                       nullptr, ws, stream, events);
 }
 
@@ -370,7 +444,7 @@ int moe_forward_eplb(const moe_bf16* x, const float* w_g, const float* bias,
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   int r = launch_expert_ffn(x_perm, L.Ppad, reinterpret_cast<const __nv_bfloat16*>(w13_phys),
                             reinterpret_cast<const __nv_bfloat16*>(w2_phys), sp, L, wsb, z, sms,
-                            cs, nullptr);
+                            cs, nullptr, true);
   if (r != MOE_OK) return r;
   return cuda_status(
       launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs));

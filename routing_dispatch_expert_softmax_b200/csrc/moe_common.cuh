@@ -84,7 +84,7 @@ inline bool shape_valid(const moe_shape* s) {
 // ----------------------------------------------------------------- workspace
 struct WsLayout {
   size_t err, w3, logit_part, logits, idx, idx_phys, w, counts, offsets, blockhist, blockbase,
-      blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, total;
+      blocksend, send, rank_off, perm, row_of, tiles, x_perm, h, z, xs, hq, hs, total;
   int nblocks;      // token blocks of kTokensPerRouteBlock
   int max_mtiles;   // upper bound of 128-row expert tiles
   long long P;      // T * k
@@ -158,6 +158,12 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms, int E_tab = -1) {
   L.x_perm = take(2 * (size_t)L.Ppad * d);
   L.h = take(2 * (size_t)L.Ppad * f);
   L.z = take(2 * (size_t)L.P * d);
+  // FP8 activations: the token codes take the x_perm region (one byte per
+  // element instead of two); their row scales, the SwiGLU output's codes and
+  // its row scales have their own.
+  L.xs = take(sizeof(float) * (size_t)L.Ppad);
+  L.hq = take((size_t)L.Ppad * f);
+  L.hs = take(sizeof(float) * (size_t)L.Ppad);
   L.total = o;
   return L;
 }
@@ -205,6 +211,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
           smem_u32(bar)),
       "r"(bytes)
       : "memory");
+}
+
+// Raises the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -321,6 +334,19 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t tmem_d, uint64_t adesc,
       : "memory");
 }
 
+// D (+)= A * B^T with E4M3 A and B from shared memory (K = 32 per instruction).
+__device__ __forceinline__ void umma_e4m3_ss(uint32_t tmem_d, uint64_t adesc,
+                                             uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05.mma issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -374,6 +400,11 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// The same for kind::f8f6f4 with E4M3 A and B (format code 0 in both fields).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // ----------------------------------------------------------------- bf16

@@ -783,18 +783,35 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 }
 
 // Work items come from a list of (row0, row_end, expert) entries: the
-// touched-expert list (every item holds all of an expert's rows, at most
-// NMAX), or with row_tiles the 128-row tile list, whose entry i covers rows
-// [row0, min(row_end, row0 + 128)) so an expert with more than NMAX = 128
-// rows becomes several items.
-template <int NMAX, bool SWIGLU>
+// touched-expert list (every item holds all of an expert's rows), or with
+// row_tiles the 128-row tile list, whose entry i covers rows
+// [row0, min(row_end, row0 + 128)).  An item with more than NMAX rows (only
+// caller offsets that give one expert more rows than the batch has tokens
+// make one) runs as several passes of at most NMAX rows, each streaming the
+// item's weights again.
+//
+// early_w != 0 (an early launch): the producer issues the weight half of its
+// first S stages before waiting for the previous kernel, and the token half
+// after.  The caller guarantees that the work list is complete once this
+// kernel may launch: the previous kernel lets its dependents launch only
+// after its own wait, and the list comes from a kernel before it.  Every
+// thread of this kernel likewise lets the next kernel launch only after its
+// own wait, so the next expert GEMM may be an early launch.
+//
+// F8: both operands are E4M3 codes (kind::f8f6f4 MMAs; a stage's 128-byte
+// rows then hold 128 K elements), w_scale holds one fp32 scale per weight row
+// (the TMA row index) and x_scale one per token row, and the epilogue
+// multiplies each accumulator by its two scales.
+template <int NMAX, bool SWIGLU, bool F8>
 __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
     const int* __restrict__ list_count, const int* __restrict__ list, int row_tiles,
     int n_tiles, int K, int w_rows_per_expert,
     int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
-    int* __restrict__ err) {
+    int* __restrict__ err, int early_w, const float* __restrict__ w_scale,
+    const float* __restrict__ x_scale) {
   using C = SwapCfg<NMAX, SWIGLU>;
+  constexpr int kKb = F8 ? 128 : kGemmBK;  // K elements per stage (128-byte rows)
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -834,14 +851,18 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();  // the work lists and operands come from the previous kernels
-  const int total = list_count[0] * n_tiles;
-  const int nk = K / kGemmBK;
+  const bool early = early_w != 0 && threadIdx.x == 0;  // the producer thread
+  if (!early) {
+    pdl_wait();  // the operands come from the previous kernels
+    pdl_trigger();
+  }
+  // The work list is read around L1: an early producer reads it before its wait.
+  const int total = __ldcg(list_count) * n_tiles;
+  const int nk = (K + kKb - 1) / kKb;  // a partial last block reads zeros past K
   const int* et = list;
   // rows of item i (row_end is the expert's end; a row tile holds at most 128)
   auto item_rows = [&](int i) {
-    const int r = et[3 * i + 1] - et[3 * i + 0];
+    const int r = __ldcg(et + 3 * i + 1) - __ldcg(et + 3 * i + 0);
     return row_tiles ? min(r, kGemmBM) : r;
   };
 
@@ -856,40 +877,74 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // token tiles of stage s: expect their bytes, arrive, load them
+      auto load_tokens = [&](int s2, int kb, int row0, int nb) {
+        uint8_t* b_dst = smem + s2 * C::kStageBytes + C::kABytes;
+        mbar_arrive_expect_tx(&full[s2], (uint32_t)(nb * 16 * 128));
+        for (int b = 0; b < nb; ++b)
+          tma_load_2d(b_dst + b * 16 * 128, &tmX, &full[s2], kb * kKb, row0 + 16 * b, pol_x);
+      };
+      // An early launch defers the token half of its first S stages until the
+      // previous kernel has completed; the stage's barrier cannot complete
+      // before that arrival.
+      int deferred = 0;
+      bool waited = !early;
+      int d_kb[S], d_row0[S], d_nb[S];
+      auto release_deferred = [&]() {
+        pdl_wait();
+        pdl_trigger();
+        waited = true;
+        for (int j = 0; j < deferred; ++j) load_tokens(j, d_kb[j], d_row0[j], d_nb[j]);
+      };
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
-        const int row0 = et[3 * i + 0];
         const int n = item_rows(i);
-        const int e = et[3 * i + 2];
-        if (n < 1 || n > NMAX) continue;  // not a small-batch item (recorded by the epilogue)
-        const int nb = (n + 15) >> 4;
+        const int e = __ldcg(et + 3 * i + 2);
         const int wrow = e * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
-        const uint32_t bytes = (uint32_t)(C::kABytes + nb * 16 * 128);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* a_dst = smem + stage * C::kStageBytes;
-          uint8_t* b_dst = a_dst + C::kABytes;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          if (SWIGLU) {
-            tma_load_2d(a_dst, &tmW, &full[stage], kb * kGemmBK, wrow, pol_w);
-            tma_load_2d(a_dst + 64 * 128, &tmW, &full[stage], kb * kGemmBK, wrow + up_offset,
-                        pol_w);
-          } else {
-            tma_load_2d(a_dst, &tmW, &full[stage], kb * kGemmBK, wrow, pol_w);
-          }
-          for (int b = 0; b < nb; ++b)
-            tma_load_2d(b_dst + b * 16 * 128, &tmX, &full[stage], kb * kGemmBK, row0 + 16 * b,
-                        pol_x);
-          ++fills[stage];
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+        for (int p0 = 0; p0 < n && ok; p0 += NMAX) {  // n < 1: recorded by the epilogue
+          const int row0 = __ldcg(et + 3 * i + 0) + p0;
+          const int nb = (min(n - p0, NMAX) + 15) >> 4;
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t* a_dst = smem + stage * C::kStageBytes;
+            // One arrival per stage, with every byte of the stage expected by
+            // then: the whole stage at once, or (deferred) the weights now and
+            // the tokens with the arrival.
+            if (waited) {
+              mbar_arrive_expect_tx(&full[stage], (uint32_t)(C::kABytes + nb * 16 * 128));
+            } else {
+              mbar_expect_tx(&full[stage], (uint32_t)C::kABytes);
+            }
+            if (SWIGLU) {
+              tma_load_2d(a_dst, &tmW, &full[stage], kb * kKb, wrow, pol_w);
+              tma_load_2d(a_dst + 64 * 128, &tmW, &full[stage], kb * kKb, wrow + up_offset,
+                          pol_w);
+            } else {
+              tma_load_2d(a_dst, &tmW, &full[stage], kb * kKb, wrow, pol_w);
+            }
+            if (waited) {
+              for (int b = 0; b < nb; ++b)
+                tma_load_2d(a_dst + C::kABytes + b * 16 * 128, &tmX, &full[stage], kb * kKb,
+                            row0 + 16 * b, pol_x);
+            } else {
+              // stages 0..S-1 of this CTA's sequence, in order
+              d_kb[deferred] = kb;
+              d_row0[deferred] = row0;
+              d_nb[deferred] = nb;
+              if (++deferred == S) release_deferred();
+            }
+            ++fills[stage];
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
+      if (!waited) release_deferred();  // fewer than S stages, or none
       if (*abort_flag) {
 #pragma unroll
         for (int s2 = 0; s2 < S; ++s2)
@@ -904,38 +959,47 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int i = w / n_tiles;
         const int n = item_rows(i);
-        if (n < 1 || n > NMAX) {
-          --it;  // skipped items use no accumulator buffer (same in the epilogue)
-          continue;
-        }
-        const uint32_t idesc = idesc_bf16_f32(128, ((n + 15) >> 4) * 16);
-        const int ab = it & 1;
-        const uint32_t aph = (uint32_t)((it >> 1) & 1);
-        if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(ab * NMAX);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+        // one accumulator buffer per pass (an empty item has none; the same in the epilogue)
+        for (int p0 = 0; p0 < n && ok; p0 += NMAX, ++it) {
+          const int ncol = ((min(n - p0, NMAX) + 15) >> 4) * 16;
+          const uint32_t idesc = F8 ? idesc_e4m3_f32(128, ncol) : idesc_bf16_f32(128, ncol);
+          const int ab = it & 1;
+          const uint32_t aph = (uint32_t)((it >> 1) & 1);
+          if (!mbar_wait_bounded(&tempty[ab], aph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b_addr = a_addr + C::kABytes;
+          const uint32_t d_tmem = tmem_base + (uint32_t)(ab * NMAX);
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
+            const uint32_t b_addr = a_addr + C::kABytes;
+            // four MMAs per stage: K = 16 bf16 or 32 E4M3 elements, 32 bytes each
 #pragma unroll
-          for (int kk = 0; kk < kGemmBK / 16; ++kk)
-            umma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
-                         sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
-          umma_commit(&empty[stage]);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+            for (int kk = 0; kk < 4; ++kk) {
+              if (F8)
+                umma_e4m3_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                             sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+              else
+                umma_bf16_ss(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                             sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
+          if (ok) umma_commit(&tfull[ab]);
         }
-        if (ok) umma_commit(&tfull[ab]);
       }
       if (*abort_flag) {
         umma_commit(drain);
@@ -947,70 +1011,83 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     const int q = warp & 3;  // TMEM lanes q*32 .. q*32+31 = weight rows
     int it = 0;
     int chunk_parity = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+    bool stop = false;
+    for (int w = blockIdx.x; w < total && !stop; w += gridDim.x) {
       const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
-      const int row0 = et[3 * i + 0];
-      const int n = item_rows(i);
-      if (n < 1 || n > NMAX) {
-        if (threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
-        --it;  // the MMA warp skipped it too: no accumulator was used
-        continue;
-      }
-      const int ncols = ((n + 15) >> 4) * 16;
-      const int ab = it & 1;
-      const uint32_t aph = (uint32_t)((it >> 1) & 1);
-      mbar_wait_bounded(&tfull[ab], aph, abort_flag);
-      // The four epilogue warps decide together whether to go on, so none is
-      // left waiting at the exchange barrier below.
-      named_bar_sync(2, 128);
-      if (*abort_flag) break;
-      tc_fence_after();
-      const uint32_t t_addr = tmem_base + (uint32_t)(ab * NMAX) + ((uint32_t)(q * 32) << 16);
-      if (SWIGLU) {
-        // lanes 0..63: gate rows j, lanes 64..127: up rows j (j = lane & 63)
-        const int j = (q & 1) * 32 + lane;
-        const int col = nt * 64 + j;
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
-          float* x = xch + chunk_parity * (64 * 16);
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_addr + c0, v);
-          tmem_ld_wait();
-          if (q >= 2) {
+      const int n_item = item_rows(i);
+      if (n_item < 1 && threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
+      for (int p0 = 0; p0 < n_item; p0 += NMAX, ++it) {
+        const int row0 = et[3 * i + 0] + p0;
+        const int n = min(n_item - p0, NMAX);
+        const int ncols = ((n + 15) >> 4) * 16;
+        const int ab = it & 1;
+        const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        mbar_wait_bounded(&tfull[ab], aph, abort_flag);
+        // The four epilogue warps decide together whether to go on, so none is
+        // left waiting at the exchange barrier below.
+        named_bar_sync(2, 128);
+        if (*abort_flag) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t t_addr = tmem_base + (uint32_t)(ab * NMAX) + ((uint32_t)(q * 32) << 16);
+        // first weight row of the item (the TMA row index; the F8 scales' index)
+        const int wrow0 = __ldcg(et + 3 * i + 2) * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
+        // accumulator of token column c times its scales (F8), else as is
+        auto scaled = [&](uint32_t bits, float sw, int c) {
+          const float a = __uint_as_float(bits);
+          if (!F8) return a;
+          return c < n ? a * sw * __ldg(x_scale + row0 + c) : 0.0f;
+        };
+        if (SWIGLU) {
+          // lanes 0..63: gate rows j, lanes 64..127: up rows j (j = lane & 63)
+          const int j = (q & 1) * 32 + lane;
+          const int col = nt * 64 + j;
+          const float sw = F8 ? __ldg(w_scale + wrow0 + (q >= 2 ? up_offset : 0) + j) : 1.0f;
+          for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float* x = xch + chunk_parity * (64 * 16);
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_addr + c0, v);
+            tmem_ld_wait();
+            if (q >= 2) {
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) x[cc * 64 + j] = __uint_as_float(v[cc]);
+              for (int cc = 0; cc < 16; ++cc) x[cc * 64 + j] = scaled(v[cc], sw, c0 + cc);
+            }
+            named_bar_sync(1, 128);
+            if (q < 2 && col < n_out) {
+#pragma unroll
+              for (int cc = 0; cc < 16; ++cc) {
+                const int c = c0 + cc;
+                if (c < n) {
+                  const float g = scaled(v[cc], sw, c);
+                  const float u = x[cc * 64 + j];
+                  out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(silu_f(g) * u);
+                }
+              }
+            }
+            chunk_parity ^= 1;
           }
-          named_bar_sync(1, 128);
-          if (q < 2 && col < n_out) {
+        } else {
+          const int col = nt * 128 + q * 32 + lane;
+          const float sw = (F8 && col < n_out) ? __ldg(w_scale + wrow0 + q * 32 + lane) : 1.0f;
+          for (int c0 = 0; c0 < ncols; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(t_addr + c0, v);
+            tmem_ld_wait();
+            if (col < n_out) {
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const int c = c0 + cc;
-              if (c < n) {
-                const float g = __uint_as_float(v[cc]);
-                const float u = x[cc * 64 + j];
-                out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(silu_f(g) * u);
+              for (int cc = 0; cc < 16; ++cc) {
+                const int c = c0 + cc;
+                if (c < n)
+                  out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(scaled(v[cc], sw, c));
               }
             }
           }
-          chunk_parity ^= 1;
         }
-      } else {
-        const int col = nt * 128 + q * 32 + lane;
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_addr + c0, v);
-          tmem_ld_wait();
-          if (col < n_out) {
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const int c = c0 + cc;
-              if (c < n)
-                out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(__uint_as_float(v[cc]));
-            }
-          }
-        }
+        tc_fence_before();
+        mbar_arrive(&tempty[ab]);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[ab]);
     }
   }
 
@@ -1058,6 +1135,22 @@ static bool make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// 2-D uint8 tensor map (E4M3 codes) over a row-major [rows, cols] byte
+// matrix; box = 128 columns (128 bytes, the swizzle span) x box_rows rows.
+static bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int BN, int EPI>
 static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
                                  const GemmArgs& args, int max_work, int num_sms,
@@ -1077,16 +1170,18 @@ static cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb,
                        1, ta, tb, args);
 }
 
-template <int NMAX, bool SWIGLU>
+template <int NMAX, bool SWIGLU, bool F8 = false>
 static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
                                  const int* list_count, const int* list, int row_tiles,
                                  int max_work, int n_tiles, int K,
                                  int w_rows, int up_off, int n_out, __nv_bfloat16* out,
-                                 int ld_out, int* err, int num_sms, cudaStream_t st) {
+                                 int ld_out, int* err, int early, int num_sms,
+                                 cudaStream_t st, const float* w_scale = nullptr,
+                                 const float* x_scale = nullptr) {
   using C = SwapCfg<NMAX, SWIGLU>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_swap<NMAX, SWIGLU>,
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_swap<NMAX, SWIGLU, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -1094,17 +1189,20 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
   }
   int grid = max_work < num_sms ? max_work : num_sms;
   if (grid < 1) grid = 1;
-  return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU>, dim3(grid), dim3(192), C::kSmemBytes, st,
-                       1, tw, tx, list_count, list, row_tiles, n_tiles, K, w_rows, up_off,
-                       n_out, out, ld_out, err);
+  return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU, F8>, dim3(grid), dim3(192),
+                       C::kSmemBytes, st, 1, tw, tx, list_count, list, row_tiles, n_tiles, K,
+                       w_rows, up_off, n_out, out, ld_out, err, early, w_scale, x_scale);
 }
 
-// Small batches (every expert has at most 256 rows): both GEMMs in swap-AB form.
+// Small batches (T <= 256): both GEMMs in swap-AB form.  GEMM2 is always an
+// early launch (GEMM1 lets it launch only after GEMM1's own wait, and the
+// work list precedes GEMM1); GEMM1 is one when the caller says so.
 static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
                                   const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                   const moe_shape& s, const WsLayout& L, char* ws,
                                   __nv_bfloat16* z, int num_sms, cudaStream_t st,
-                                  void* const* events) {
+                                  void* const* events, bool early1) {
+  const int e1 = early1 ? 1 : 0;
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
     return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,
@@ -1128,22 +1226,81 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
     const int* cnt = tiles + 1;
     const int* ents = expert_entries(const_cast<int*>(tiles));
     e = launch_swap_t<64, true>(tW1, tX1, cnt, ents, 0, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h,
-                                s.f, err, num_sms, st);
+                                s.f, err, e1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_swap_t<64, false>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d, z,
-                                   s.d, err, num_sms, st);
+                                   s.d, err, 1, num_sms, st);
   } else {
-    // one item per 128-row tile: 6 K-stages of weights in flight instead of
+    // one item per 128-row tile: 5 K-stages of weights in flight instead of
     // the 4 that 256-row items leave room for
     const int* cnt = tiles;
     const int* ents = row_tile_entries(const_cast<int*>(tiles), E);
     e = launch_swap_t<128, true>(tW1, tX1, cnt, ents, 1, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
-                                 s.f, s.f, h, s.f, err, num_sms, st);
+                                 s.f, s.f, h, s.f, err, e1, num_sms, st);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_swap_t<128, false>(tW2, tX2, cnt, ents, 1, L.max_mtiles * nt2, nt2, s.f, s.d,
-                                    0, s.d, z, s.d, err, num_sms, st);
+                                    0, s.d, z, s.d, err, 1, num_sms, st);
+  }
+  if (e == cudaSuccess) e = mark(1);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Both GEMMs with E4M3 operands on both sides, at every batch size: the
+// swap-AB kernels over the touched-expert list (T <= 64) or the plain 128-row
+// tile list, and between them the SwiGLU output quantised row by row.  GEMM2
+// is an early launch (the quantisation kernel lets it launch after its own
+// wait; the work list precedes GEMM1).
+int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
+                           const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
+                           const float* w2_scale, const moe_shape& s, const WsLayout& L,
+                           char* ws, __nv_bfloat16* z, int num_sms, cudaStream_t st,
+                           void* const* events, bool early_gemm1) {
+  auto mark = [&](int i) -> cudaError_t {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), st,
+                                    cudaEventRecordExternal);
+  };
+  int* err = reinterpret_cast<int*>(ws + L.err);
+  const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+  uint8_t* hq = reinterpret_cast<uint8_t*>(ws + L.hq);
+  float* hs = reinterpret_cast<float*>(ws + L.hs);
+  CUtensorMap tW1, tX1, tW2, tX2;
+  if (!make_tmap_u8(&tW1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, 64) ||
+      !make_tmap_u8(&tX1, xq, (uint64_t)x_rows, (uint64_t)s.d, 16) ||
+      !make_tmap_u8(&tW2, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, 128) ||
+      !make_tmap_u8(&tX2, hq, (uint64_t)L.Ppad, (uint64_t)s.f, 16))
+    return MOE_ERR_CUDA;
+  const int nt1 = s.f / 64, nt2 = (s.d + 127) / 128, E = s.E;
+  const int e1 = early_gemm1 ? 1 : 0;
+  auto quant_h = [&]() {
+    return launch_quant_rows(h, nullptr, L.P, 0, s.f, hq, hs, err, st);
+  };
+  cudaError_t e;
+  if (s.T <= 64) {
+    const int* cnt = tiles + 1;
+    const int* ents = expert_entries(const_cast<int*>(tiles));
+    e = launch_swap_t<64, true, true>(tW1, tX1, cnt, ents, 0, E * nt1, nt1, s.d, 2 * s.f, s.f,
+                                      s.f, h, s.f, err, e1, num_sms, st, w13_scale, xs);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess) e = quant_h();
+    if (e == cudaSuccess)
+      e = launch_swap_t<64, false, true>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d,
+                                         z, s.d, err, 1, num_sms, st, w2_scale, hs);
+  } else {
+    const int* cnt = tiles;
+    const int* ents = row_tile_entries(const_cast<int*>(tiles), E);
+    e = launch_swap_t<128, true, true>(tW1, tX1, cnt, ents, 1, L.max_mtiles * nt1, nt1, s.d,
+                                       2 * s.f, s.f, s.f, h, s.f, err, e1, num_sms, st,
+                                       w13_scale, xs);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess) e = quant_h();
+    if (e == cudaSuccess)
+      e = launch_swap_t<128, false, true>(tW2, tX2, cnt, ents, 1, L.max_mtiles * nt2, nt2, s.f,
+                                          s.d, 0, s.d, z, s.d, err, 1, num_sms, st, w2_scale,
+                                          hs);
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -1175,7 +1332,7 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                       const moe_shape& s, const WsLayout& L, char* ws,
                       __nv_bfloat16* z, int num_sms, cudaStream_t st,
-                      void* const* events) {
+                      void* const* events, bool early_gemm1) {
   // events (optional): [0] recorded after GEMM1, [1] after GEMM2.
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
@@ -1183,7 +1340,8 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                                     cudaEventRecordExternal);
   };
   if (s.T <= kSwapMaxT)
-    return launch_expert_ffn_swap(x_perm, x_rows, w13, w2, s, L, ws, z, num_sms, st, events);
+    return launch_expert_ffn_swap(x_perm, x_rows, w13, w2, s, L, ws, z, num_sms, st, events,
+                                  early_gemm1);
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);

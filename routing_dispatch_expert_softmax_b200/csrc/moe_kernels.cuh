@@ -36,11 +36,14 @@ cudaError_t launch_selftest_bounded_wait(unsigned long long limit_ns, int* err,
                                          cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const float* w,
                            const moe_shape& s, __nv_bfloat16* y, cudaStream_t st);
+// early_gemm1: the kernel just before (the row gather) lets GEMM1 launch only
+// after its own wait, and the work list comes from a kernel before it, so
+// GEMM1 may start streaming weights before the gather completes.
 int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                       const moe_shape& s, const WsLayout& L, char* ws,
                       __nv_bfloat16* z, int num_sms, cudaStream_t st,
-                      void* const* events = nullptr);
+                      void* const* events = nullptr, bool early_gemm1 = false);
 
 // The same two GEMMs with E4M3 expert weights and one fp32 scale per weight
 // row (moe_gemm_fp8.cu): swap-AB form at every batch size, over the plain
@@ -49,6 +52,22 @@ int launch_expert_ffn_fp8(const __nv_bfloat16* x_perm, long long x_rows, const u
                           const float* w13_scale, const uint8_t* w2, const float* w2_scale,
                           const moe_shape& s, const WsLayout& L, char* ws, __nv_bfloat16* z,
                           int num_sms, cudaStream_t st, void* const* events = nullptr);
+
+// Row quantisation to E4M3 with power-of-two row scales (moe_w8a8.cu):
+// output row r from input row perm[r] (perm != nullptr; ids outside
+// [0, n_src) are recorded in err) or row r.
+cudaError_t launch_quant_rows(const __nv_bfloat16* a, const int* perm, long long rows, int n_src,
+                              int cols, uint8_t* codes, float* scales, int* err,
+                              cudaStream_t st);
+
+// Both expert GEMMs with E4M3 weights (one fp32 scale per weight row) and
+// E4M3 tokens (xq, one scale per row in xs): GEMM1 with the SwiGLU epilogue
+// into h (bf16), h quantised into the workspace, GEMM2 (moe_gemm_sm100.cu).
+int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
+                           const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
+                           const float* w2_scale, const moe_shape& s, const WsLayout& L,
+                           char* ws, __nv_bfloat16* z, int num_sms, cudaStream_t st,
+                           void* const* events = nullptr, bool early_gemm1 = false);
 
 // Logical -> physical expert ids of a replica plan (moe_eplb.cu).
 cudaError_t launch_eplb_remap(const int* idx, int T, int k, int E, const int* rep_offsets,

@@ -742,8 +742,10 @@ __global__ void __launch_bounds__(kTokensPerRouteBlock) k_scatter(
 __global__ void __launch_bounds__(256) k_gather_rows(
     const __nv_bfloat16* __restrict__ x, const int* __restrict__ perm, long long P,
     int T, int d, __nv_bfloat16* __restrict__ x_perm, int* err) {
-  pdl_trigger();
+  // Lets the expert GEMMs launch only after this wait: they may then read the
+  // work lists (written before this kernel) before their own wait.
   pdl_wait();
+  pdl_trigger();
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= P) return;
   const int lane = threadIdx.x & 31;

@@ -104,18 +104,24 @@ class MoELayer:
 
     FP8 experts: pass w13 / w2 as uint8 E4M3 codes of the same shapes with
     ``w13_scale`` (E, 2f) and ``w2_scale`` (E, d) fp32 row scales; the layer
-    then runs moe_forward_fp8."""
+    then runs moe_forward_fp8 (bf16 activations), or with
+    ``fp8_activations=True`` moe_forward_w8a8 (activations quantised to E4M3
+    too, both GEMM operands one byte)."""
 
     def __init__(self, w_g: torch.Tensor, bias: Optional[torch.Tensor],
                  w13: torch.Tensor, w2: torch.Tensor, k: int, R: int = 0,
                  w13_scale: Optional[torch.Tensor] = None,
-                 w2_scale: Optional[torch.Tensor] = None):
+                 w2_scale: Optional[torch.Tensor] = None,
+                 fp8_activations: bool = False):
         B.load_library()
         if (w13_scale is None) != (w2_scale is None):
             raise ValueError("FP8 experts need both w13_scale and w2_scale")
+        if fp8_activations and w13_scale is None:
+            raise ValueError("FP8 activations need FP8 experts (w13_scale, w2_scale)")
         self.w_g, self.bias, self.w13, self.w2 = w_g, bias, w13, w2
         self.w13_scale, self.w2_scale = w13_scale, w2_scale
         self.fp8 = w13_scale is not None
+        self.w8a8 = bool(fp8_activations)
         self.d, self.E = int(w_g.shape[0]), int(w_g.shape[1])
         self.f = int(w2.shape[2])
         self.k, self.R = int(k), int(R)
@@ -141,9 +147,9 @@ class MoELayer:
     def _call(self, x, y, ws, idx_out=None, w_out=None, counts_out=None, stream=None):
         shape = self.shape(int(x.shape[0]))
         if self.fp8:
-            B.moe_forward_fp8(x, self.w_g, self.bias, self.w13, self.w13_scale, self.w2,
-                              self.w2_scale, y, shape, ws, idx_out=idx_out, w_out=w_out,
-                              counts_out=counts_out, stream=stream)
+            fwd = B.moe_forward_w8a8 if self.w8a8 else B.moe_forward_fp8
+            fwd(x, self.w_g, self.bias, self.w13, self.w13_scale, self.w2, self.w2_scale, y,
+                shape, ws, idx_out=idx_out, w_out=w_out, counts_out=counts_out, stream=stream)
         elif self._eplb is None:
             B.moe_forward(x, self.w_g, self.bias, self.w13, self.w2, y, shape, ws,
                           idx_out=idx_out, w_out=w_out, counts_out=counts_out, stream=stream)

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_error_strings(lib):
-    assert moe.moe_version() == 103
+    assert moe.moe_version() == 104
     for code in range(6):
         assert moe.moe_error_string(code).startswith("MOE_")
     assert "unknown" in moe.moe_error_string(99)
@@ -151,6 +151,33 @@ def test_fp8_calls_reject_before_launch(lib):
                 None) == B.MOE_OK
 
 
+def test_w8a8_calls_reject_before_launch(lib):
+    s = ctypes.byref(B.MoEShape.of(**VALID))
+    INV = B.MOE_ERR_INVALID_ARG
+    ws = _P(A16)
+    # moe_ffn_w8a8(x_perm, offsets, w13, w13_scale, w2, w2_scale, s, z, ws, stream)
+    assert _raw(lib, "moe_ffn_w8a8", _P(A16), _P(A16), _P(A16), None, _P(A16), _P(A16), s,
+                _P(A16), ws, None) == INV                       # null w13 scales
+    assert _raw(lib, "moe_ffn_w8a8", _P(A16), _P(A16), _P(A16 + 8), _P(A16), _P(A16),
+                _P(A16), s, _P(A16), ws, None) == INV           # codes not 16-byte aligned
+    fwd = [_P(A16), _P(A16), None, _P(A16), _P(A16), _P(A16), _P(A16)]
+    assert _raw(lib, "moe_forward_w8a8", *fwd[:6], None, s, _P(A16), None, None, None, ws,
+                None) == INV                                    # null w2 scales
+    assert _raw(lib, "moe_forward_w8a8", *fwd, s, _P(A16), None, None, None, None,
+                None) == INV                                    # null workspace
+    s0 = ctypes.byref(B.MoEShape.of(**dict(VALID, T=0)))
+    assert _raw(lib, "moe_forward_w8a8", *[None] * 7, s0, None, None, None, None, ws,
+                None) == B.MOE_OK
+    # moe_quantise_rows_e4m3(a, rows, cols, codes, scales, stream)
+    assert _raw(lib, "moe_quantise_rows_e4m3", _P(A16), 4, 24, _P(A16), _P(A16),
+                None) == INV                                    # cols not a multiple of 16
+    assert _raw(lib, "moe_quantise_rows_e4m3", _P(A16), -1, 32, _P(A16), _P(A16),
+                None) == INV                                    # negative rows
+    assert _raw(lib, "moe_quantise_rows_e4m3", _P(A16), 4, 32, _P(A16 + 4), _P(A16),
+                None) == INV                                    # misaligned codes
+    assert _raw(lib, "moe_quantise_rows_e4m3", None, 0, 32, None, None, None) == B.MOE_OK
+
+
 def test_empty_batch_is_a_no_op(lib):
     s0 = ctypes.byref(B.MoEShape.of(**dict(VALID, T=0)))
     # T = 0 launches nothing, so even null activation pointers are accepted.
@@ -170,6 +197,10 @@ def test_no_cpu_fallback_without_a_gpu(lib):
                 None) == B.MOE_ERR_CUDA
     assert _raw(lib, "moe_forward_fp8", *[_P(A16)] * 7, s, _P(A16), None, None, None,
                 _P(A16), None) == B.MOE_ERR_CUDA
+    assert _raw(lib, "moe_forward_w8a8", *[_P(A16)] * 7, s, _P(A16), None, None, None,
+                _P(A16), None) == B.MOE_ERR_CUDA
+    assert _raw(lib, "moe_quantise_rows_e4m3", _P(A16), 4, 32, _P(A16), _P(A16),
+                None) == B.MOE_ERR_CUDA
 
 
 def test_binding_refuses_cpu_tensors(lib):

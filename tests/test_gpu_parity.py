@@ -331,6 +331,41 @@ def test_ffn_pair_regime_tile_kinds(counts):
     assert_layer_close(z, ref, "moe_ffn tile kinds")
 
 
+@pytest.mark.parametrize("T,counts", [
+    # T <= 64: one item per expert of at most 64 rows; 100 rows -> 2 passes
+    (16, [100, 0, 20, 8, 0, 0, 0, 0]),
+    # T <= 64: items of at most 64 rows; 300 rows -> 5 passes, 65 -> 2
+    (64, [300, 1, 64, 65, 0, 82, 0, 0]),
+    # 64 < T <= 256: 128-row tiles
+    (200, [1000, 300, 0, 300, 0, 0, 0, 0]),
+], ids=["T16", "T64", "T200"])
+def test_ffn_small_batch_expert_with_more_rows_than_tokens(T, counts):
+    """moe_ffn at decode batch sizes on caller offsets that give one expert
+    more rows than the batch has tokens (the header allows any monotone
+    offsets ending at T*k): every row still matches the oracle and no error
+    is recorded."""
+    counts = np.array(counts, dtype=np.int64)
+    E, k = counts.size, 8
+    P = int(counts.sum())
+    assert P == T * k
+    cfg = wl.MoEConfig("swap-passes", T=T, d=256, E=E, k=k, f=384)
+    x_perm = wl.make_hidden(cfg.with_T(P), DEV, 11)
+    w13, w2 = wl.make_experts(cfg, DEV, 11)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    shape = MoEShape.from_config(cfg)
+    ws = moe.workspace(shape)
+    z = torch.empty(P, cfg.d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn(x_perm, torch.from_numpy(offsets).to(DEV), w13, w2, z, shape, ws)
+    _check_clean(ws)
+    xp = np64(x_perm)
+    ref = np.zeros((P, cfg.d))
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if b > a:
+            ref[a:b] = oracle.swiglu_ffn(xp[a:b], np64(w13[e]), np64(w2[e]))
+    assert_layer_close(z, ref, f"moe_ffn T={T} oversized expert")
+
+
 def test_ffn_qwen_prefill_sampled():
     _ffn_case(wl.QWEN3_30B_A3B_PREFILL, sample_rows=_sample_rows())
 

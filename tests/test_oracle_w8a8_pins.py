@@ -139,7 +139,7 @@ def test_w8a8_ffn_equals_its_recomposition_from_library_casts():
     ulp = np.ldexp(1.0, np.frexp(hb)[1] - 8)
     assert not np.any(np.abs(np.abs(h32 - hb) - ulp / 2) == 0), "double-rounding tie in seed"
     want = q(hb) @ w2.T
-    got = F._w8a8_ffn(X, w13, w2)
+    got = F.w8a8_ffn(X, w13, w2)
     np.testing.assert_array_equal(got, want)
 
 
