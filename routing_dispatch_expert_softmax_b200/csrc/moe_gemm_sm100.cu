@@ -765,7 +765,12 @@ struct SwapCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * NMAX;
   static constexpr int kXchBytes = SWIGLU ? 2 * 64 * 16 * 4 : 0;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kXchBytes + 1024 + 256;
+  // This CTA's first kMaxItems work items (row0, rows, expert, column tile),
+  // read from the list once: a per-item L2 read in the producer and the MMA
+  // loop stalls both at every item boundary.
+  static constexpr int kMaxItems = 128;
+  static constexpr int kItemBytes = 16 * kMaxItems;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kXchBytes + 1024 + 256 + kItemBytes;
 };
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
@@ -824,6 +829,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* n_items_s = const_cast<int*>(abort_flag) + 1;
+  int4* items_s = reinterpret_cast<int4*>(smem + S * C::kStageBytes + C::kXchBytes + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -851,20 +858,44 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Warp 0 (the producer's) of an early launch reads the work list before its
+  // wait; every other thread waits here.
   const bool early = early_w != 0 && threadIdx.x == 0;  // the producer thread
-  if (!early) {
+  if (!(early_w != 0 && warp == 0)) {
     pdl_wait();  // the operands come from the previous kernels
     pdl_trigger();
   }
-  // The work list is read around L1: an early producer reads it before its wait.
-  const int total = __ldcg(list_count) * n_tiles;
   const int nk = (K + kKb - 1) / kKb;  // a partial last block reads zeros past K
-  const int* et = list;
-  // rows of item i (row_end is the expert's end; a row tile holds at most 128)
-  auto item_rows = [&](int i) {
-    const int r = __ldcg(et + 3 * i + 1) - __ldcg(et + 3 * i + 0);
-    return row_tiles ? min(r, kGemmBM) : r;
+  // This CTA's j-th work item is w = blockIdx.x + j * gridDim.x: (row0, rows,
+  // expert, column tile); a row tile holds at most 128 rows of its expert.
+  // The list is read around L1 (an early producer reads it before its wait).
+  auto load_item = [&](int j) -> int4 {
+    const int w = blockIdx.x + j * gridDim.x;
+    const int i = w / n_tiles;
+    const int row0 = __ldcg(list + 3 * i + 0);
+    const int r = __ldcg(list + 3 * i + 1) - row0;
+    return make_int4(row0, row_tiles ? min(r, kGemmBM) : r, __ldcg(list + 3 * i + 2),
+                     w - i * n_tiles);
   };
+  // Warp 0 fills the table, then arrives (without waiting) on named barrier 3,
+  // which the other warps wait on.
+  if (warp == 0) {
+    const int total = __ldcg(list_count) * n_tiles;
+    const int my = total > (int)blockIdx.x ? (total - (int)blockIdx.x - 1) / (int)gridDim.x + 1
+                                           : 0;
+    for (int j = lane; j < min(my, C::kMaxItems); j += 32) items_s[j] = load_item(j);
+    if (lane == 0) *n_items_s = my;
+    __syncwarp();
+    asm volatile("bar.arrive 3, 192;" ::: "memory");
+    if (early_w != 0 && lane != 0) {
+      pdl_wait();
+      pdl_trigger();
+    }
+  } else {
+    named_bar_sync(3, 192);
+  }
+  const int my_items = *n_items_s;
+  auto item = [&](int j) -> int4 { return j < C::kMaxItems ? items_s[j] : load_item(j); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -896,13 +927,12 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         waited = true;
         for (int j = 0; j < deferred; ++j) load_tokens(j, d_kb[j], d_row0[j], d_nb[j]);
       };
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
-        const int n = item_rows(i);
-        const int e = __ldcg(et + 3 * i + 2);
-        const int wrow = e * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
+      for (int j = 0; j < my_items && ok; ++j) {
+        const int4 itm = item(j);
+        const int n = itm.y;
+        const int wrow = itm.z * w_rows_per_expert + itm.w * (SWIGLU ? 64 : 128);
         for (int p0 = 0; p0 < n && ok; p0 += NMAX) {  // n < 1: recorded by the epilogue
-          const int row0 = __ldcg(et + 3 * i + 0) + p0;
+          const int row0 = itm.x + p0;
           const int nb = (min(n - p0, NMAX) + 15) >> 4;
           for (int kb = 0; kb < nk; ++kb) {
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -959,9 +989,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int i = w / n_tiles;
-        const int n = item_rows(i);
+      for (int j = 0; j < my_items && ok; ++j) {
+        const int n = item(j).y;
         // one accumulator buffer per pass (an empty item has none; the same in the epilogue)
         for (int p0 = 0; p0 < n && ok; p0 += NMAX, ++it) {
           const int ncol = ((min(n - p0, NMAX) + 15) >> 4) * 16;
@@ -1012,12 +1041,12 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     int it = 0;
     int chunk_parity = 0;
     bool stop = false;
-    for (int w = blockIdx.x; w < total && !stop; w += gridDim.x) {
-      const int i = w / n_tiles, nt = w - (w / n_tiles) * n_tiles;
-      const int n_item = item_rows(i);
+    for (int j = 0; j < my_items && !stop; ++j) {
+      const int4 itm = item(j);
+      const int n_item = itm.y, nt = itm.w;
       if (n_item < 1 && threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
       for (int p0 = 0; p0 < n_item; p0 += NMAX, ++it) {
-        const int row0 = et[3 * i + 0] + p0;
+        const int row0 = itm.x + p0;
         const int n = min(n_item - p0, NMAX);
         const int ncols = ((n + 15) >> 4) * 16;
         const int ab = it & 1;
@@ -1033,7 +1062,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         tc_fence_after();
         const uint32_t t_addr = tmem_base + (uint32_t)(ab * NMAX) + ((uint32_t)(q * 32) << 16);
         // first weight row of the item (the TMA row index; the F8 scales' index)
-        const int wrow0 = __ldcg(et + 3 * i + 2) * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
+        const int wrow0 = itm.z * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
         // accumulator of token column c times its scales (F8), else as is
         auto scaled = [&](uint32_t bits, float sw, int c) {
           const float a = __uint_as_float(bits);
