@@ -71,10 +71,11 @@ def launches_per_forward(cfg, eplb_redundant=0, fp8=False, w8a8=False):
     (router_launches), routing (one fused kernel for T <= 1024, else top-k +
     histogram + scan + scatter; with replicas top-k + remap + histogram + scan
     + scatter), the row gather (with w8a8 the gather-and-quantise kernel), the
-    two expert GEMMs (the bf16 ones each followed by the lone-tile kernel when
-    they run on CTA pairs; the FP8 ones always run the 128-row-tile form; with
-    w8a8 the SwiGLU output's quantisation between them), combine."""
-    fp8 = fp8 or w8a8
+    two expert GEMMs (the bf16 and W8A8 ones each followed by the lone-tile
+    kernel when they run on CTA pairs; the FP8-weight ones always run the
+    128-row-tile form; with w8a8 the SwiGLU output's quantisation between
+    them), combine."""
+    fp8 = fp8 and not w8a8
     T = cfg.T
     routing = 1 if T <= 1024 else 4
     if eplb_redundant:

@@ -202,7 +202,9 @@ static int forward_impl(int mode, const moe_bf16* x, const float* w_g, const flo
       (counts_out && !aligned(counts_out, 4)) ||
       (mode != kBf16 && (!ok4(w13_scale) || !ok4(w2_scale))))
     return MOE_ERR_INVALID_ARG;
-  const bool fp8 = mode != kBf16;  // the plain 128-row tile list
+  // The FP8-weight GEMMs run on the plain 128-row tile list; the bf16 and
+  // W8A8 ones on the CTA-pair layout when pair_tiles(s).
+  const int pair = mode == kFp8Weights ? 0 : -1;
   int sms = 0;
   int st = device_check(&sms);
   if (st != MOE_OK) return st;
@@ -232,13 +234,12 @@ static int forward_impl(int mode, const moe_bf16* x, const float* w_g, const flo
     if (s->T <= kFusedRouteMaxT) {
       e = launch_route_fused(logits, *s, idx, gw, counts, offsets, at<int>(ws, L.tiles),
                              at<int>(ws, L.send), at<int>(ws, L.rank_off), row_of, perm,
-                             at<int>(ws, L.err), cs, fp8 ? 0 : -1);
+                             at<int>(ws, L.err), cs, pair);
     } else {
       e = launch_topk(logits, *s, idx, gw, cs);
       if (e == cudaSuccess)
         e = launch_route_tables(idx, *s, L, wsb, counts, offsets, row_of, perm,
-                                at<int>(ws, L.send), at<int>(ws, L.rank_off), cs,
-                                fp8 ? 0 : -1);
+                                at<int>(ws, L.send), at<int>(ws, L.rank_off), cs, pair);
     }
   }
   uint8_t* xq = at<uint8_t>(ws, L.x_perm);  // W8A8: token codes in the x_perm region
@@ -350,7 +351,7 @@ int moe_ffn_w8a8(const moe_bf16* x_perm, const int32_t* offsets, const uint8_t* 
   float* xs = at<float>(ws, L.xs);
   // the work list first, so GEMM1 may read it before the quantisation completes
   cudaError_t e = launch_tiles_from_offsets(offsets, *s, at<int>(ws, L.tiles),
-                                            at<int>(ws, L.err), cs, 0);
+                                            at<int>(ws, L.err), cs);
   if (e == cudaSuccess)
     e = launch_quant_rows(reinterpret_cast<const __nv_bfloat16*>(x_perm), nullptr, L.P, 0, s->d,
                           xq, xs, at<int>(ws, L.err), cs);

@@ -65,6 +65,8 @@ struct GemmArgs {
   int kparts;             // K partitions per output tile (kEpiLogits; 1 otherwise)
   long long part_stride;  // elements between the partial outputs of two partitions
   int pdl;                // kPdlStart / kPdlAfterWait / kPdlTail
+  const float* a_scale;   // E4M3 operands (the CTA-pair kernel's F8 form): one scale per A row
+  const float* b_scale;   // and one per B row (weight row)
 };
 
 __device__ __forceinline__ void pdl_enter(int mode) {
@@ -456,6 +458,17 @@ __device__ __forceinline__ void umma_bf16_ss_pair(uint32_t tmem_d, uint64_t ades
       : "memory");
 }
 
+// The same with E4M3 A and B (K = 32 per instruction).
+__device__ __forceinline__ void umma_e4m3_ss_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on the barrier at this offset in every CTA of `mask` when all
 // tcgen05.mma issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t mask) {
@@ -497,12 +510,16 @@ struct PairCfg {
   static constexpr int kSmemBytes = kStages * kStageBytes + kOutStageBytes + 1024 + 256;
 };
 
-template <int EPI>
+// F8: A (token rows) and B (weight rows) are E4M3 codes; a stage's 128-byte
+// rows then hold 128 K elements (kind::f8f6f4 MMAs), and the epilogue
+// multiplies each accumulator by args.a_scale[row] * args.b_scale[weight row].
+template <int EPI, bool F8 = false>
 __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const GemmArgs args) {
   using C = PairCfg<EPI>;
   constexpr int S = C::kStages;
+  constexpr int kKb = F8 ? 128 : kGemmBK;  // K elements per stage
   constexpr int BN = 256;
   constexpr bool SWIGLU = (EPI == kEpiSwiGLU);
   extern __shared__ uint8_t smem_raw[];
@@ -554,7 +571,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
   const int num_pairs = tile_ld(args.tile_count) / 2;
   const int n_tiles = args.n_tiles;
   const int total = num_pairs * n_tiles;
-  const int nk = args.K / kGemmBK;
+  const int nk = (args.K + kKb - 1) / kKb;  // F8: a partial last block reads zeros past K
   const int* tl = args.tile_rows;
   const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
 
@@ -585,8 +602,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
           uint8_t* b_dst = a_dst + C::kABytes;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
           const uint32_t lbar = smem_u32(&full[stage]) & 0xFEFFFFFFu;  // the leader's barrier
-          tma_load_2d_pair(a_dst, &tmA, lbar, kb * kGemmBK, a_row, pol);
-          tma_load_2d_pair(b_dst, &tmB, lbar, kb * kGemmBK, b_row, pol);
+          tma_load_2d_pair(a_dst, &tmA, lbar, kb * kKb, a_row, pol);
+          tma_load_2d_pair(b_dst, &tmB, lbar, kb * kKb, b_row, pol);
           ++fills[stage];
           if (++stage == S) {
             stage = 0;
@@ -603,7 +620,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------ MMA issuer (leader)
-      constexpr uint32_t idesc = idesc_bf16_f32(256, BN);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(256, BN) : idesc_bf16_f32(256, BN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -622,10 +639,18 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t b_addr = a_addr + C::kABytes;
+          // four MMAs per stage: K = 16 bf16 or 32 E4M3 elements, 32 bytes each
 #pragma unroll
-          for (int kk = 0; kk < kGemmBK / 16; ++kk)
-            umma_bf16_ss_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
-                              sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            if (F8)
+              umma_e4m3_ss_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                                sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                                (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16_ss_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                                sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                                (kb | kk) != 0 ? 1u : 0u);
+          }
           umma_commit_pair_mc(&empty[stage], 0x3);  // frees this stage in both CTAs
           if (++stage == S) {
             stage = 0;
@@ -655,6 +680,10 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
       raster(w, n_tiles, num_pairs, mp, nt);
       const int row0 = tile_ld(tl + 3 * (2 * mp) + 0);
       const int rowend = tile_ld(tl + 3 * (2 * mp) + 1);
+      // F8: first weight row of the tile (SwiGLU: of its gate half)
+      const int wrow0 = F8 ? tile_ld(tl + 3 * (2 * mp) + 2) * args.b_rows_per_expert +
+                                 nt * (SWIGLU ? BN / 2 : BN)
+                           : 0;
       const int ab = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       const bool got = mbar_wait_bounded(&tfull[ab], aph, abort_flag);
@@ -684,6 +713,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
         constexpr int H = BN / 2;
         const int row = row_base + lane;
         const bool row_ok = row < rowend;
+        const float sa = (F8 && row_ok) ? __ldg(args.a_scale + row) : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < H; c += 32) {
           uint32_t g[32], u[32];
@@ -692,6 +722,15 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
           tmem_ld_wait();
           const int col = nt * H + c;
           if (row_ok && col < args.n_out) {
+            if (F8) {  // gate rows wrow0 + c + i, up rows up_offset further
+              const float* sg = args.b_scale + wrow0 + c;
+              const float* su = sg + args.up_offset;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                g[i] = __float_as_uint(__uint_as_float(g[i]) * sa * __ldg(sg + i));
+                u[i] = __float_as_uint(__uint_as_float(u[i]) * sa * __ldg(su + i));
+              }
+            }
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -706,6 +745,8 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
           }
         }
       } else {
+        const int row = row_base + lane;
+        const float sa = (F8 && row < rowend) ? __ldg(args.a_scale + row) : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 64) {
 #pragma unroll
@@ -713,6 +754,12 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
             uint32_t a[32];
             tmem_ld_32x32b_x32(t_addr + c + 32 * half, a);
             tmem_ld_wait();
+            if (F8 && nt * BN + c + 32 * half < args.n_out) {
+              const float* sb = args.b_scale + wrow0 + c + 32 * half;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                a[i] = __float_as_uint(__uint_as_float(a[i]) * sa * __ldg(sb + i));
+            }
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -1276,11 +1323,33 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// Both GEMMs with E4M3 operands on both sides, at every batch size: the
-// swap-AB kernels over the touched-expert list (T <= 64) or the plain 128-row
-// tile list, and between them the SwiGLU output quantised row by row.  GEMM2
-// is an early launch (the quantisation kernel lets it launch after its own
-// wait; the work list precedes GEMM1).
+template <int EPI, bool F8 = false>
+static cudaError_t launch_gemm_2sm(const CUtensorMap& ta, const CUtensorMap& tb,
+                                   const GemmArgs& args, int max_pairs_work, int num_sms,
+                                   cudaStream_t st) {
+  using C = PairCfg<EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_2sm<EPI, F8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int clusters = max_pairs_work < num_sms / 2 ? max_pairs_work : num_sms / 2;
+  if (clusters < 1) clusters = 1;
+  return launch_kernel(k_grouped_gemm_2sm<EPI, F8>, dim3(2 * clusters), dim3(192), C::kSmemBytes,
+                       st, 2, ta, tb, args);
+}
+
+// Both GEMMs with E4M3 operands on both sides, at every batch size, and
+// between them the SwiGLU output quantised row by row: the swap-AB kernels
+// over the touched-expert list (T <= 64) or the 128-row tile list; for large
+// dense batches (the CTA-pair tile layout, pair_tiles) the CTA-pair kernels
+// over the tile pairs, with the lone-tile experts' leftover list on the
+// swap-AB kernels (their tokens fit one 128-row item).  The swap-AB GEMM2 of
+// the small-batch forms is an early launch (the quantisation kernel lets it
+// launch after its own wait; the work list precedes GEMM1).
 int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
                            const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
                            const float* w2_scale, const moe_shape& s, const WsLayout& L,
@@ -1318,6 +1387,34 @@ int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
     if (e == cudaSuccess)
       e = launch_swap_t<64, false, true>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d,
                                          z, s.d, err, 1, num_sms, st, w2_scale, hs);
+  } else if (pair_tiles(s)) {
+    CUtensorMap pA1, pB1, pA2, pB2;  // 128-row boxes: each CTA of a pair loads 128 rows
+    if (!make_tmap_u8(&pA1, xq, (uint64_t)x_rows, (uint64_t)s.d, 128) ||
+        !make_tmap_u8(&pB1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, 128) ||
+        !make_tmap_u8(&pA2, hq, (uint64_t)L.Ppad, (uint64_t)s.f, 128) ||
+        !make_tmap_u8(&pB2, w2, (uint64_t)s.E * s.d, (uint64_t)s.f, 128))
+      return MOE_ERR_CUDA;
+    const int* count = tiles;
+    const int* rows = row_tile_entries(const_cast<int*>(tiles), E);
+    const int* lcount = tiles + 2;
+    const int* lrows = leftover_entries(const_cast<int*>(tiles), E);
+    const int pnt1 = (s.f + 127) / 128, pnt2 = (s.d + 255) / 256;  // 256-wide output tiles
+    GemmArgs g1{count, rows, E, 0, pnt1, s.d, 0, 2 * s.f, s.f, s.f, h, s.f, nullptr, err, 0, 1,
+                0, kPdlStart, xs, w13_scale};
+    GemmArgs g2{count, rows, E, 0, pnt2, s.f, 0, s.d, 0, s.d, z, s.d, nullptr, err, 0, 1, 0,
+                kPdlStart, hs, w2_scale};
+    const int max_pairs = (L.max_mtiles + 1) / 2;
+    e = launch_gemm_2sm<kEpiSwiGLU, true>(pA1, pB1, g1, max_pairs * pnt1, num_sms, st);
+    if (e == cudaSuccess)
+      e = launch_swap_t<128, true, true>(tW1, tX1, lcount, lrows, 1, E * nt1, nt1, s.d, 2 * s.f,
+                                         s.f, s.f, h, s.f, err, 0, num_sms, st, w13_scale, xs);
+    if (e == cudaSuccess) e = mark(0);
+    if (e == cudaSuccess) e = quant_h();
+    if (e == cudaSuccess)
+      e = launch_gemm_2sm<kEpiStore, true>(pA2, pB2, g2, max_pairs * pnt2, num_sms, st);
+    if (e == cudaSuccess)
+      e = launch_swap_t<128, false, true>(tW2, tX2, lcount, lrows, 1, E * nt2, nt2, s.f, s.d, 0,
+                                          s.d, z, s.d, err, 0, num_sms, st, w2_scale, hs);
   } else {
     const int* cnt = tiles;
     const int* ents = row_tile_entries(const_cast<int*>(tiles), E);
@@ -1333,25 +1430,6 @@ int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
-template <int EPI>
-static cudaError_t launch_gemm_2sm(const CUtensorMap& ta, const CUtensorMap& tb,
-                                   const GemmArgs& args, int max_pairs_work, int num_sms,
-                                   cudaStream_t st) {
-  using C = PairCfg<EPI>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_2sm<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  int clusters = max_pairs_work < num_sms / 2 ? max_pairs_work : num_sms / 2;
-  if (clusters < 1) clusters = 1;
-  return launch_kernel(k_grouped_gemm_2sm<EPI>, dim3(2 * clusters), dim3(192), C::kSmemBytes, st,
-                       2, ta, tb, args);
 }
 
 // Both expert GEMMs over the rows described by the device tile list.

@@ -149,6 +149,34 @@ def test_ffn_w8a8_caller_offsets(T, counts):
     _ffn_case(cfg, 3, offsets=offsets, x_perm=x_perm)
 
 
+@pytest.mark.parametrize("counts", [
+    # CTA-pair regime (T*k >= 128*E): lone-tile experts (<= 128 rows) go to the
+    # leftover list (swap-AB kernels), odd tile counts to padded pairs, empty
+    # experts to nothing
+    [600, 100, 300, 50, 0, 50, 0, 1],
+    [0, 128, 1, 127, 64, 8, 9, 1024 + 129],
+], ids=["mixed", "lone"])
+def test_ffn_w8a8_pair_regime_tile_kinds(counts):
+    counts = np.array(counts, dtype=np.int64)
+    E, P = counts.size, int(counts.sum())
+    cfg = wl.MoEConfig("w8a8-pairs", T=P, d=256, E=E, k=1, f=384)
+    assert P > 256 and P >= 128 * E
+    x_perm = wl.make_hidden(cfg, DEV, 7)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    _ffn_case(cfg, 7, offsets=offsets, x_perm=x_perm)
+
+
+def test_ffn_w8a8_pair_regime_ragged_widths():
+    # f = 192: a partial 128-column gate tile; d = 320: a partial 256-column
+    # output tile and partial last K blocks on both GEMMs
+    counts = np.array([300, 129, 0, 700], dtype=np.int64)
+    E, P = counts.size, int(counts.sum())
+    cfg = wl.MoEConfig("w8a8-pairs-ragged", T=P, d=320, E=E, k=1, f=192)
+    x_perm = wl.make_hidden(cfg, DEV, 8)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    _ffn_case(cfg, 8, offsets=offsets, x_perm=x_perm)
+
+
 # ------------------------------------------------------------ whole layer
 def _forward_case(cfg, sample=None, seed=0):
     x = wl.make_hidden(cfg, DEV, seed)
@@ -202,8 +230,12 @@ def test_forward_w8a8_deepseek(T):
 
 
 @pytest.mark.parametrize("cfg", [wl.QWEN3_30B_A3B_DECODE.with_T(257),
-                                 wl.QWEN3_30B_A3B_PREFILL], ids=lambda c: c.name)
+                                 wl.QWEN3_30B_A3B_PREFILL,
+                                 wl.DEEPSEEK_V3_ROUTED.with_T(512)], ids=lambda c: c.name)
 def test_forward_w8a8_large_batches(cfg):
+    # above 256 tokens: the CTA-pair kernels once experts average 128 rows (the
+    # prefill), the swap-AB kernels on 128-row tiles below that (T = 257,
+    # DeepSeek-V3 at T = 512)
     _forward_case(cfg, sample=None if cfg.T <= 257 else token_sample())
 
 
