@@ -512,9 +512,16 @@ def timed_passes(plain_fn, staged_fn, steps, warmup, flush_l2, stream, dist, dev
 STAGE_EVENTS = 6
 
 
-def kernel_roofline(cfg, alg, mean_stage, peaks, peak_src, traffic_key):
+# Dense E4M3 tensor-core throughput is twice bf16's (4.5 vs 2.25 PFLOP/s
+# nominal); the e4m3 peak is the measured bf16 figure times that ratio.
+E4M3_OVER_BF16 = 2.0
+
+
+def kernel_roofline(cfg, alg, mean_stage, peaks, peak_src, traffic_key, e4m3=False):
     """Roofline of the dominant stage: its algorithmic bytes (or flops, for
-    an expert GEMM at a tensor-bound batch) over its mean event time."""
+    an expert GEMM at a tensor-bound batch) over its mean event time.  With
+    e4m3 (both GEMM operands E4M3) a tensor-bound stage is measured against
+    the e4m3 peak."""
     decode = cfg.P / cfg.E < 64
     dom = max(range(len(mean_stage)), key=lambda j: mean_stage[j])
     kern = STAGES[dom]
@@ -522,8 +529,11 @@ def kernel_roofline(cfg, alg, mean_stage, peaks, peak_src, traffic_key):
     if kern in ("gemm1_swiglu", "gemm2") and not decode:
         fl = alg["gemm1_flops"] if kern == "gemm1_swiglu" else alg["gemm2_flops"]
         achieved = fl / t_kern / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+        peak = peaks["bf16_tflops"] * (E4M3_OVER_BF16 if e4m3 else 1.0)
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak}
+        if e4m3:
+            roof["peak_dtype"] = "e4m3 (the bf16 peak x 2, the nominal dense ratio)"
     else:
         by = {"gemm1_swiglu": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(
             kern, cfg.T * cfg.d * 2 * 2)
@@ -537,17 +547,19 @@ def kernel_roofline(cfg, alg, mean_stage, peaks, peak_src, traffic_key):
     return roof
 
 
-def layer_roofline(cfg, alg, touched, ms_per_step, peaks):
+def layer_roofline(cfg, alg, touched, ms_per_step, peaks, e4m3=False):
     """The whole layer's algorithmic bytes and flops against the measured
-    peaks and the spec denominators (~8 TB/s HBM, 2.25 PF/s dense bf16)."""
+    peaks and the spec denominators (~8 TB/s HBM, 2.25 PF/s dense bf16;
+    with e4m3 GEMM operands twice those tensor peaks)."""
     t_layer = ms_per_step / 1e3
     decode = cfg.P / cfg.E < 64
+    r = E4M3_OVER_BF16 if e4m3 else 1.0
     return {
         "bytes": alg["bytes"], "flops": alg["flops"], "touched_experts": touched,
         "hbm_frac_measured": alg["bytes"] / t_layer / (peaks["hbm_gbs"] * 1e9),
         "hbm_frac_spec_8TBs": alg["bytes"] / t_layer / 8e12,
-        "tensor_frac_measured": alg["flops"] / t_layer / (peaks["bf16_tflops"] * 1e12),
-        "tensor_frac_spec_2250TF": alg["flops"] / t_layer / 2.25e15,
+        "tensor_frac_measured": alg["flops"] / t_layer / (r * peaks["bf16_tflops"] * 1e12),
+        "tensor_frac_spec": alg["flops"] / t_layer / (r * 2.25e15),
         "bound": "hbm" if decode else "tensor",
     }
 
@@ -564,55 +576,73 @@ def run_sweep(args, dev, local, peaks, peak_src, flush_l2, stream):
     points = []
     clocks = ClockSampler(local).start()
     steps, warmup = max(args.steps, 1), max(args.warmup, 3)
-    for name, Ts in SWEEP:
-        base = wl.CONFIGS[name]
-        w_g, bias = wl.make_router(base, dev, 0)
-        w13, w2 = wl.make_experts(base, dev, 0)
-        for T in Ts:
-            cfg = base.with_T(T)
-            x = wl.make_hidden(cfg, dev, 0)
-            shape = moe.MoEShape.from_config(cfg)
-            ws = moe.workspace(shape, dev)
-            y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
-            counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
-            moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, counts_out=counts)
-            torch.cuda.synchronize(dev)
+    for w8a8 in (False, True):
+        for name, Ts in SWEEP:
+            base = wl.CONFIGS[name]
+            w_g, bias = wl.make_router(base, dev, 0)
+            if w8a8:
+                w13, s13, w2, s2 = wl.make_experts_fp8(base, dev, 0)
+            else:
+                w13, w2 = wl.make_experts(base, dev, 0)
+            for T in Ts:
+                cfg = base.with_T(T)
+                x = wl.make_hidden(cfg, dev, 0)
+                shape = moe.MoEShape.from_config(cfg)
+                ws = moe.workspace(shape, dev)
+                y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=dev)
+                counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+                if w8a8:
+                    plain = lambda: moe.moe_forward_w8a8(x, w_g, bias, w13, s13, w2, s2, y,
+                                                         shape, ws)
+                    staged = lambda e: moe.moe_forward_w8a8_staged(x, w_g, bias, w13, s13, w2,
+                                                                   s2, y, shape, ws, e)
+                    moe.moe_forward_w8a8(x, w_g, bias, w13, s13, w2, s2, y, shape, ws,
+                                         counts_out=counts)
+                else:
+                    plain = lambda: moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws)
+                    staged = lambda e: moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape,
+                                                              ws, e)
+                    moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, counts_out=counts)
+                torch.cuda.synchronize(dev)
 
-            def check():
-                st = moe.moe_check(ws)
-                if st != moe.MOE_OK:
-                    raise RuntimeError(f"{cfg.name}: {moe.moe_error_string(st)}")
+                def check():
+                    st = moe.moe_check(ws)
+                    if st != moe.MOE_OK:
+                        raise RuntimeError(f"{cfg.name}: {moe.moe_error_string(st)}")
 
-            step_ms, stage_ms, win = timed_passes(
-                lambda: moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws),
-                lambda e: moe.moe_forward_staged(x, w_g, bias, w13, w2, y, shape, ws, e),
-                steps, warmup, flush_l2, stream, None, dev, check)
-            counts_h = counts.cpu().tolist()
-            touched = sum(1 for v in counts_h if v > 0)
-            alg = algorithmic(cfg, touched)
-            ms = statistics.fmean(step_ms)
-            mean_stage = [statistics.fmean(s[j] for s in stage_ms)
-                          for j in range(len(stage_ms[0]))]
-            points.append({
-                "workload": base.name, "T": cfg.T, "us_per_layer": ms * 1e3,
-                "tokens_per_s": cfg.T / (ms / 1e3),
-                "layer_roofline": layer_roofline(cfg, alg, touched, ms, peaks),
-                "roofline": kernel_roofline(cfg, alg, mean_stage, peaks, peak_src,
-                                            f"{base.name}@T{cfg.T}"),
-                "stage_us": {k: v * 1e3 for k, v in zip(STAGES, mean_stage)},
-                "routing": routing_stats(counts_h, cfg.R), "window": win})
-            del x, ws, y, counts
-        del w_g, bias, w13, w2
-        torch.cuda.empty_cache()
+                step_ms, stage_ms, win = timed_passes(plain, staged, steps, warmup, flush_l2,
+                                                      stream, None, dev, check)
+                counts_h = counts.cpu().tolist()
+                touched = sum(1 for v in counts_h if v > 0)
+                alg = algorithmic(cfg, touched, fp8=w8a8)
+                ms = statistics.fmean(step_ms)
+                mean_stage = [statistics.fmean(s[j] for s in stage_ms)
+                              for j in range(len(stage_ms[0]))]
+                points.append({
+                    "workload": base.name, "T": cfg.T,
+                    "precision": "w8a8 (e4m3 weights and activations)" if w8a8 else "bf16",
+                    "us_per_layer": ms * 1e3, "tokens_per_s": cfg.T / (ms / 1e3),
+                    "layer_roofline": layer_roofline(cfg, alg, touched, ms, peaks, w8a8),
+                    "roofline": kernel_roofline(cfg, alg, mean_stage, peaks, peak_src,
+                                                f"{base.name}@T{cfg.T}" +
+                                                ("/w8a8" if w8a8 else ""), e4m3=w8a8),
+                    "stage_us": {k: v * 1e3 for k, v in zip(STAGES, mean_stage)},
+                    "routing": routing_stats(counts_h, cfg.R), "window": win})
+                del x, ws, y, counts
+            del w_g, bias, w13, w2
+            if w8a8:
+                del s13, s2
+            torch.cuda.empty_cache()
     overall = clocks.stop()
     for p in points:
         t0, t1 = p.pop("window")
         p["clocks"] = clocks.summary(t0, t1)
     return {"points": points, "clocks": overall, "steps": steps, "warmup": warmup,
-            "note": "each point: mean of K plain CUDA-graph replays of moe_forward, L2 flushed "
-                    "before every step; stage_us from the staged pass (event nodes add a few "
-                    "us each); roofline = dominant stage vs MEASURED_PEAKS.json; clocks = "
-                    "samples inside the point's timed region, else the nearest sample"}
+            "note": "each point: mean of K plain CUDA-graph replays of moe_forward (bf16) or "
+                    "moe_forward_w8a8 (e4m3 weights and activations, the second half), L2 "
+                    "flushed before every step; stage_us from the staged pass (event nodes add "
+                    "a few us each); roofline = dominant stage vs MEASURED_PEAKS.json; clocks "
+                    "= samples inside the point's timed region, else the nearest sample"}
 
 
 def run_ours(args):
@@ -802,8 +832,9 @@ def run_ours(args):
     mean_stage = [statistics.fmean(s[j] for s in stage_ms) for j in range(len(stage_ms[0]))]
     roof = kernel_roofline(cfg, alg, mean_stage, peaks, peak_src,
                            f"{cfg.name}@T{cfg.T}" +
-                           ("/w8a8" if args.w8a8 else "/fp8" if args.fp8 else ""))
-    layer_roof = layer_roofline(cfg, alg, touched, ms_per_step, peaks)
+                           ("/w8a8" if args.w8a8 else "/fp8" if args.fp8 else ""),
+                           e4m3=args.w8a8)
+    layer_roof = layer_roofline(cfg, alg, touched, ms_per_step, peaks, args.w8a8)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
