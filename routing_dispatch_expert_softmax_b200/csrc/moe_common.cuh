@@ -109,8 +109,20 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // would be half empty, so it runs as a single-CTA leftover tile instead.
 __host__ __device__ inline int pair_row_tiles(int nt) { return nt == 1 ? 0 : (nt + 1) & ~1; }
 
+// Upper bound of the row-tile list: each expert one partial tile and, in the
+// CTA-pair layout, one padding tile.
+__host__ __device__ inline int max_mtiles_of(long long P, int E) {
+  return (int)((P + kGemmBM - 1) / kGemmBM + 2 * E);
+}
+// After the lists: one ready counter per list entry (max_mtiles + E of them),
+// zeroed by every kernel that writes the lists.  The small-batch GEMM1 adds 1
+// to entry i's counter when one of its column tiles of that entry's rows is
+// stored; GEMM2 starts an entry's work once the count is complete.
 __host__ __device__ inline size_t tile_list_ints(int max_mtiles, int E) {
-  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E);
+  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E) + (size_t)max_mtiles + E;
+}
+__host__ __device__ inline int* ready_counters(int* tiles, int max_mtiles, int E) {
+  return tiles + 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E);
 }
 __host__ __device__ inline int* expert_entries(int* tiles) { return tiles + 4; }
 __host__ __device__ inline int* leftover_entries(int* tiles, int E) { return tiles + 4 + 3 * E; }
@@ -129,7 +141,7 @@ inline WsLayout ws_layout(const moe_shape& s, int num_sms, int E_tab = -1) {
   L.Ppad = L.P + kGemmBM;
   L.nblocks = (int)((T + kTokensPerRouteBlock - 1) / kTokensPerRouteBlock);
   // each expert: one partial tile and, in the CTA-pair layout, one padding tile
-  L.max_mtiles = (int)((L.P + kGemmBM - 1) / kGemmBM + 2 * E);
+  L.max_mtiles = max_mtiles_of(L.P, (int)E);
   (void)num_sms;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -252,6 +264,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(
       *abort = 1;
       return false;
     }
+  }
+}
+
+// Orders this thread's generic-proxy global accesses with later async-proxy
+// (TMA) accesses, in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Spins until *counter >= target (acquire, GPU scope), with the bounded-wait
+// limit; on timeout sets *abort_flag and returns false.
+__device__ __forceinline__ bool wait_count_bounded(const int* counter, int target,
+                                                   volatile int* abort_flag) {
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
   }
 }
 

@@ -850,6 +850,14 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 // thread of this kernel likewise lets the next kernel launch only after its
 // own wait, so the next expert GEMM may be an early launch.
 //
+// ready != nullptr: the GEMM1 / GEMM2 pair synchronises per work-list entry
+// instead of per kernel.  GEMM1 (SWIGLU) adds 1 to ready[i] once it has
+// stored an item's columns of entry i's rows; GEMM2 never waits for GEMM1 as
+// a whole: before streaming an item of entry i it waits (bounded) until
+// ready[i] == ready_target (GEMM1's column tiles), so GEMM2 CTAs on SMs that
+// GEMM1's tail frees start at once.  GEMM2 waits for the previous kernel only
+// at its end, so its completion still implies GEMM1's.
+//
 // F8: both operands are E4M3 codes (kind::f8f6f4 MMAs; a stage's 128-byte
 // rows then hold 128 K elements), w_scale holds one fp32 scale per weight row
 // (the TMA row index) and x_scale one per token row, and the epilogue
@@ -861,7 +869,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     int n_tiles, int K, int w_rows_per_expert,
     int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
     int* __restrict__ err, int early_w, const float* __restrict__ w_scale,
-    const float* __restrict__ x_scale) {
+    const float* __restrict__ x_scale, int* __restrict__ ready, int ready_target) {
   using C = SwapCfg<NMAX, SWIGLU>;
   constexpr int kKb = F8 ? 128 : kGemmBK;  // K elements per stage (128-byte rows)
   constexpr int S = C::kStages;
@@ -908,7 +916,10 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   // Warp 0 (the producer's) of an early launch reads the work list before its
   // wait; every other thread waits here.
   const bool early = early_w != 0 && threadIdx.x == 0;  // the producer thread
-  if (!(early_w != 0 && warp == 0)) {
+  const bool counted = !SWIGLU && ready != nullptr;      // GEMM2 of a counted pair
+  if (counted) {
+    pdl_trigger();
+  } else if (!(early_w != 0 && warp == 0)) {
     pdl_wait();  // the operands come from the previous kernels
     pdl_trigger();
   }
@@ -962,22 +973,44 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         for (int b = 0; b < nb; ++b)
           tma_load_2d(b_dst + b * 16 * 128, &tmX, &full[s2], kb * kKb, row0 + 16 * b, pol_x);
       };
-      // An early launch defers the token half of its first S stages until the
-      // previous kernel has completed; the stage's barrier cannot complete
-      // before that arrival.
+      // Token tiles that cannot be read yet are deferred: an early launch's
+      // first S stages (until the previous kernel completes) and, in a
+      // counted GEMM2, the stages of an item whose entry GEMM1 has not
+      // finished.  A deferred stage gets its weights at once and its tokens
+      // (with the stage's single arrival) when released, so its barrier
+      // cannot complete before; at most S stages, of one item, are deferred.
       int deferred = 0;
-      bool waited = !early;
-      int d_kb[S], d_row0[S], d_nb[S];
-      auto release_deferred = [&]() {
-        pdl_wait();
-        pdl_trigger();
-        waited = true;
-        for (int j = 0; j < deferred; ++j) load_tokens(j, d_kb[j], d_row0[j], d_nb[j]);
+      bool waited = !early;  // the previous kernel is complete (or need not be)
+      int d_stage[S], d_kb[S], d_row0[S], d_nb[S];
+      auto release_deferred = [&](const int* counter) -> bool {
+        if (!waited) {
+          pdl_wait();
+          pdl_trigger();
+          waited = true;
+        }
+        if (counter != nullptr) {  // entry's rows of h complete, then read by TMA
+          if (!wait_count_bounded(counter, ready_target, abort_flag)) return false;
+          fence_proxy_async_global();
+        }
+        for (int q = 0; q < deferred; ++q) load_tokens(d_stage[q], d_kb[q], d_row0[q], d_nb[q]);
+        deferred = 0;
+        return true;
       };
       for (int j = 0; j < my_items && ok; ++j) {
         const int4 itm = item(j);
         const int n = itm.y;
         const int wrow = itm.z * w_rows_per_expert + itm.w * (SWIGLU ? 64 : 128);
+        // counted GEMM2: this item's entry counter, or nullptr once it is complete
+        const int* pending = nullptr;
+        if (counted && n > 0) {
+          const int* c = ready + (int)(blockIdx.x + j * gridDim.x) / n_tiles;
+          int v;
+          asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+          if (v >= ready_target)
+            fence_proxy_async_global();
+          else
+            pending = c;
+        }
         for (int p0 = 0; p0 < n && ok; p0 += NMAX) {  // n < 1: recorded by the epilogue
           const int row0 = itm.x + p0;
           const int nb = (min(n - p0, NMAX) + 15) >> 4;
@@ -987,10 +1020,11 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
               break;
             }
             uint8_t* a_dst = smem + stage * C::kStageBytes;
+            const bool now = waited && pending == nullptr;
             // One arrival per stage, with every byte of the stage expected by
             // then: the whole stage at once, or (deferred) the weights now and
             // the tokens with the arrival.
-            if (waited) {
+            if (now) {
               mbar_arrive_expect_tx(&full[stage], (uint32_t)(C::kABytes + nb * 16 * 128));
             } else {
               mbar_expect_tx(&full[stage], (uint32_t)C::kABytes);
@@ -1002,26 +1036,32 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
             } else {
               tma_load_2d(a_dst, &tmW, &full[stage], kb * kKb, wrow, pol_w);
             }
-            if (waited) {
+            if (now) {
               for (int b = 0; b < nb; ++b)
                 tma_load_2d(a_dst + C::kABytes + b * 16 * 128, &tmX, &full[stage], kb * kKb,
                             row0 + 16 * b, pol_x);
             } else {
-              // stages 0..S-1 of this CTA's sequence, in order
+              d_stage[deferred] = stage;
               d_kb[deferred] = kb;
               d_row0[deferred] = row0;
               d_nb[deferred] = nb;
-              if (++deferred == S) release_deferred();
+              if (++deferred == S) {  // the ring is full of deferred stages
+                ok = release_deferred(pending);
+                pending = nullptr;
+              }
             }
             ++fills[stage];
             if (++stage == S) {
               stage = 0;
               phase ^= 1u;
             }
+            if (!ok) break;
           }
         }
+        // an item's deferred stages are released before the next item begins
+        if (ok && pending != nullptr) ok = release_deferred(pending);
       }
-      if (!waited) release_deferred();  // fewer than S stages, or none
+      if (ok && (!waited || deferred > 0)) ok = release_deferred(nullptr);  // few stages, or none
       if (*abort_flag) {
 #pragma unroll
         for (int s2 = 0; s2 < S; ++s2)
@@ -1164,6 +1204,15 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         tc_fence_before();
         mbar_arrive(&tempty[ab]);
       }
+      if (SWIGLU && ready != nullptr && !stop) {
+        // every epilogue thread's stores of this item, then one release add
+        fence_proxy_async_global();
+        named_bar_sync(4, 128);
+        if (threadIdx.x == 64) {
+          __threadfence();
+          atomicAdd(ready + (int)(blockIdx.x + j * gridDim.x) / n_tiles, 1);
+        }
+      }
     }
   }
 
@@ -1172,6 +1221,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   tc_fence_after();
   if (threadIdx.x == 0 && *abort_flag) record_error(err, MOE_ERR_TIMEOUT, 11);
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  if (counted) pdl_wait();  // completion implies the previous kernel's
 }
 
 // ============================================================== host side
@@ -1253,7 +1303,8 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
                                  int w_rows, int up_off, int n_out, __nv_bfloat16* out,
                                  int ld_out, int* err, int early, int num_sms,
                                  cudaStream_t st, const float* w_scale = nullptr,
-                                 const float* x_scale = nullptr) {
+                                 const float* x_scale = nullptr, int* ready = nullptr,
+                                 int ready_target = 0) {
   using C = SwapCfg<NMAX, SWIGLU>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1267,12 +1318,13 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
   if (grid < 1) grid = 1;
   return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU, F8>, dim3(grid), dim3(192),
                        C::kSmemBytes, st, 1, tw, tx, list_count, list, row_tiles, n_tiles, K,
-                       w_rows, up_off, n_out, out, ld_out, err, early, w_scale, x_scale);
+                       w_rows, up_off, n_out, out, ld_out, err, early, w_scale, x_scale, ready,
+                       ready_target);
 }
 
-// Small batches (T <= 256): both GEMMs in swap-AB form.  GEMM2 is always an
-// early launch (GEMM1 lets it launch only after GEMM1's own wait, and the
-// work list precedes GEMM1); GEMM1 is one when the caller says so.
+// Small batches (T <= 256): both GEMMs in swap-AB form.  GEMM2 waits for
+// GEMM1 per work-list entry (ready counters), so its CTAs start as GEMM1's
+// tail frees SMs; GEMM1 is an early launch when the caller says so.
 static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
                                   const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                   const moe_shape& s, const WsLayout& L, char* ws,
@@ -1296,28 +1348,31 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
   const int nt1 = s.f / 64;               // 64 gate + 64 up rows per item
   const int nt2 = (s.d + 127) / 128;      // 128 output columns per item
   const int E = s.E;
+  // GEMM2 starts each list entry once GEMM1 has stored all nt1 column tiles of it
+  int* ready = ready_counters(const_cast<int*>(tiles), L.max_mtiles, E);
   cudaError_t e;
   if (s.T <= 64) {
     // one item per touched expert (at most 64 rows)
     const int* cnt = tiles + 1;
     const int* ents = expert_entries(const_cast<int*>(tiles));
     e = launch_swap_t<64, true>(tW1, tX1, cnt, ents, 0, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h,
-                                s.f, err, e1, num_sms, st);
+                                s.f, err, e1, num_sms, st, nullptr, nullptr, ready);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_swap_t<64, false>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d, z,
-                                   s.d, err, 1, num_sms, st);
+                                   s.d, err, 0, num_sms, st, nullptr, nullptr, ready, nt1);
   } else {
     // one item per 128-row tile: 5 K-stages of weights in flight instead of
     // the 4 that 256-row items leave room for
     const int* cnt = tiles;
     const int* ents = row_tile_entries(const_cast<int*>(tiles), E);
     e = launch_swap_t<128, true>(tW1, tX1, cnt, ents, 1, L.max_mtiles * nt1, nt1, s.d, 2 * s.f,
-                                 s.f, s.f, h, s.f, err, e1, num_sms, st);
+                                 s.f, s.f, h, s.f, err, e1, num_sms, st, nullptr, nullptr, ready);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_swap_t<128, false>(tW2, tX2, cnt, ents, 1, L.max_mtiles * nt2, nt2, s.f, s.d,
-                                    0, s.d, z, s.d, err, 1, num_sms, st);
+                                    0, s.d, z, s.d, err, 0, num_sms, st, nullptr, nullptr, ready,
+                                    nt1);
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -31,7 +31,7 @@ bool scratch_layout(const moe_shape& s, WsLayout* L) {
   L->P = T * k;
   L->Ppad = L->P + kGemmBM;
   L->nblocks = (int)((T + kTokensPerRouteBlock - 1) / kTokensPerRouteBlock);
-  L->max_mtiles = (int)((L->P + kGemmBM - 1) / kGemmBM + 2 * E);
+  L->max_mtiles = max_mtiles_of(L->P, (int)E);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t at = o;

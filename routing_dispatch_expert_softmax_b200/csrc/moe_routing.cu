@@ -418,7 +418,9 @@ __device__ int block_exclusive_scan_1024(int v, int* scratch /*[32]*/, int* tota
 // and first row off.  pair: tile pairs for CTA-pair GEMMs (see
 // pair_row_tiles).
 __device__ void write_work_lists(int e, int E, int c, int off, int* tiles, int* scratch,
-                                 int* total, bool pair) {
+                                 int* total, bool pair, int max_mtiles) {
+  int* ready = ready_counters(tiles, max_mtiles, E);
+  for (int i = threadIdx.x; i < max_mtiles + E; i += blockDim.x) ready[i] = 0;
   const int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
   const int nrow = pair ? pair_row_tiles(nt) : nt;  // tiles in the row-tile list
   const int left = (pair && nt == 1) ? 1 : 0;       // a lone tile: leftover list
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(1024) k_scan(
     const int* __restrict__ blockhist, int nblocks, int E, int R,
     const int* __restrict__ blocksend, int* __restrict__ blockbase,
     int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ tiles,
-    int* __restrict__ send, int* __restrict__ rank_off, int pair) {
+    int* __restrict__ send, int* __restrict__ rank_off, int pair, int max_mtiles) {
   pdl_trigger();
   pdl_wait();
   __shared__ int scratch[32];
@@ -478,7 +480,7 @@ __global__ void __launch_bounds__(1024) k_scan(
     for (int b = 0; b < nblocks; ++b) blockbase[(size_t)b * E + e] += off;
   }
   if (e == 0) offsets[E] = P;
-  write_work_lists(e, E, c, off, tiles, scratch, &total, pair != 0);
+  write_work_lists(e, E, c, off, tiles, scratch, &total, pair != 0, max_mtiles);
   if (R > 1) {
     for (int i = threadIdx.x; i < R * R; i += blockDim.x) {
       int s = 0;
@@ -511,7 +513,7 @@ __global__ void __launch_bounds__(1024) k_tiles_from_offsets(
       c = 0;
     }
   }
-  write_work_lists(e, E, c, a, tiles, scratch, &total, pair != 0);
+  write_work_lists(e, E, c, a, tiles, scratch, &total, pair != 0, max_mtiles_of(P, E));
 }
 
 // ============================================================== fused routing, T <= 1024
@@ -577,7 +579,7 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     int* __restrict__ idx, float* __restrict__ w, int* __restrict__ counts,
     int* __restrict__ offsets, int* __restrict__ tiles, int* __restrict__ send_out,
     int* __restrict__ rank_off, int* __restrict__ row_of, int* __restrict__ perm, int* err,
-    int* ticket, int pair) {
+    int* ticket, int pair, int max_mtiles) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int sm[];
@@ -619,6 +621,10 @@ __global__ void __launch_bounds__(1024) k_route_fused(
     __syncthreads();
   }
   const int* ids = ids_in_smem ? idx_s : idx;
+  {
+    int* ready = ready_counters(tiles, max_mtiles, E);
+    for (int i = threadIdx.x; i < max_mtiles + E; i += 1024) ready[i] = 0;
+  }
   const int t = threadIdx.x;
   const bool valid = t < T;
   // The ids come from this kernel's own selection: distinct per token by
@@ -955,7 +961,8 @@ static cudaError_t route_fused_t(const float* logits, const moe_shape& s, int R,
   const unsigned blocks = (unsigned)((s.T + kFusedSelTokens - 1) / kFusedSelTokens);
   return launch_kernel(k_route_fused<VPL>, dim3(blocks), dim3(1024), smem, st, 1, logits, s.T,
                        s.E, s.k, R, chunk, idx, w, counts, offsets, tiles, send, rank_off, row_of,
-                       perm, err, err + kRouteTicket, pair);
+                       perm, err, err + kRouteTicket, pair,
+                       max_mtiles_of((long long)s.T * s.k, s.E));
 }
 
 cudaError_t launch_route_fused(const float* logits, const moe_shape& s, int* idx, float* w,
@@ -993,7 +1000,8 @@ cudaError_t launch_route_tables(const int* idx, const moe_shape& s, const WsLayo
                                 st, 1, idx, s.T, s.E, s.k, R, chunk, blockhist, blocksend, err);
   if (e != cudaSuccess) return e;
   e = launch_kernel(k_scan, dim3(1), dim3(1024), 0, st, 1, blockhist, L.nblocks, s.E, R,
-                    blocksend, blockbase, counts, offsets, tiles, send, rank_off, pair);
+                    blocksend, blockbase, counts, offsets, tiles, send, rank_off, pair,
+                    L.max_mtiles);
   if (e != cudaSuccess) return e;
   const size_t scat_smem = sizeof(uint32_t) * (kTokensPerRouteBlock / 32) * s.E;
   return launch_kernel(k_scatter, dim3(L.nblocks), dim3(kTokensPerRouteBlock), scat_smem, st, 1,
