@@ -118,8 +118,9 @@ __host__ __device__ inline int max_mtiles_of(long long P, int E) {
 // zeroed by every kernel that writes the lists.  The small-batch GEMM1 adds 1
 // to entry i's counter when one of its column tiles of that entry's rows is
 // stored; GEMM2 starts an entry's work once the count is complete.
+// One more int after them: the small-batch GEMM2's item queue.
 __host__ __device__ inline size_t tile_list_ints(int max_mtiles, int E) {
-  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E) + (size_t)max_mtiles + E;
+  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E) + (size_t)max_mtiles + E + 1;
 }
 __host__ __device__ inline int* ready_counters(int* tiles, int max_mtiles, int E) {
   return tiles + 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E);

@@ -858,6 +858,14 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 // GEMM1's tail frees start at once.  GEMM2 waits for the previous kernel only
 // at its end, so its completion still implies GEMM1's.
 //
+// A counted GEMM2 with ready_count > 0 takes its items from a queue
+// (ready[ready_count], an int after the counters, zeroed with them) instead
+// of every gridDim.x-th item:
+// the producer claims item w with atomicAdd, in order, and passes (row0,
+// rows, expert, w) to the MMA and epilogue warps through a ring of 8
+// records with full / empty barriers; a record with rows < 0 ends the work.
+// Its CTAs start as GEMM1's tail frees SMs, so the early ones take more items.
+//
 // F8: both operands are E4M3 codes (kind::f8f6f4 MMAs; a stage's 128-byte
 // rows then hold 128 K elements), w_scale holds one fp32 scale per weight row
 // (the TMA row index) and x_scale one per token row, and the epilogue
@@ -869,7 +877,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     int n_tiles, int K, int w_rows_per_expert,
     int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
     int* __restrict__ err, int early_w, const float* __restrict__ w_scale,
-    const float* __restrict__ x_scale, int* __restrict__ ready, int ready_target) {
+    const float* __restrict__ x_scale, int* __restrict__ ready, int ready_target,
+    int ready_count) {
   using C = SwapCfg<NMAX, SWIGLU>;
   constexpr int kKb = F8 ? 128 : kGemmBK;  // K elements per stage (128-byte rows)
   constexpr int S = C::kStages;
@@ -886,6 +895,12 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* n_items_s = const_cast<int*>(abort_flag) + 1;
   int4* items_s = reinterpret_cast<int4*>(smem + S * C::kStageBytes + C::kXchBytes + 256);
+  // dynamic items: the first 8 table slots are the ring, its barriers follow
+  constexpr int kRing = 8;
+  uint64_t* ifull = reinterpret_cast<uint64_t*>(items_s + kRing);
+  uint64_t* iempty = ifull + kRing;
+  const bool counted = !SWIGLU && ready != nullptr;  // GEMM2 of a counted pair
+  const bool dyn = counted && ready_count > 0;       // ... taking items from the queue
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -898,6 +913,12 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    if (dyn) {
+      for (int r = 0; r < kRing; ++r) {
+        mbar_init(&ifull[r], 1);
+        mbar_init(&iempty[r], 1);
+      }
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -916,7 +937,6 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   // Warp 0 (the producer's) of an early launch reads the work list before its
   // wait; every other thread waits here.
   const bool early = early_w != 0 && threadIdx.x == 0;  // the producer thread
-  const bool counted = !SWIGLU && ready != nullptr;      // GEMM2 of a counted pair
   if (counted) {
     pdl_trigger();
   } else if (!(early_w != 0 && warp == 0)) {
@@ -924,20 +944,23 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     pdl_trigger();
   }
   const int nk = (K + kKb - 1) / kKb;  // a partial last block reads zeros past K
-  // This CTA's j-th work item is w = blockIdx.x + j * gridDim.x: (row0, rows,
-  // expert, column tile); a row tile holds at most 128 rows of its expert.
-  // The list is read around L1 (an early producer reads it before its wait).
-  auto load_item = [&](int j) -> int4 {
-    const int w = blockIdx.x + j * gridDim.x;
+  // Work item w: (row0, rows, expert, w) of list entry w / n_tiles, column
+  // tile w % n_tiles; a row tile holds at most 128 rows of its expert.  The
+  // list is read around L1 (an early producer reads it before its wait).
+  auto load_w = [&](int w) -> int4 {
     const int i = w / n_tiles;
     const int row0 = __ldcg(list + 3 * i + 0);
     const int r = __ldcg(list + 3 * i + 1) - row0;
-    return make_int4(row0, row_tiles ? min(r, kGemmBM) : r, __ldcg(list + 3 * i + 2),
-                     w - i * n_tiles);
+    return make_int4(row0, row_tiles ? min(r, kGemmBM) : r, __ldcg(list + 3 * i + 2), w);
   };
+  // Static items: this CTA's j-th is w = blockIdx.x + j * gridDim.x.
+  auto load_item = [&](int j) -> int4 { return load_w(blockIdx.x + j * gridDim.x); };
   // Warp 0 fills the table, then arrives (without waiting) on named barrier 3,
   // which the other warps wait on.
-  if (warp == 0) {
+  if (dyn) {
+    if (warp != 0) named_bar_sync(3, 192);
+    else asm volatile("bar.arrive 3, 192;" ::: "memory");
+  } else if (warp == 0) {
     const int total = __ldcg(list_count) * n_tiles;
     const int my = total > (int)blockIdx.x ? (total - (int)blockIdx.x - 1) / (int)gridDim.x + 1
                                            : 0;
@@ -952,8 +975,21 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   } else {
     named_bar_sync(3, 192);
   }
-  const int my_items = *n_items_s;
+  const int my_items = dyn ? 0 : *n_items_s;
   auto item = [&](int j) -> int4 { return j < C::kMaxItems ? items_s[j] : load_item(j); };
+  // Item j of the MMA and epilogue warps: the table's, or (counted) the ring's
+  // record; false at the end of the work.
+  auto fetch = [&](int j, int4& itm) -> bool {
+    if (!dyn) {
+      if (j >= my_items) return false;
+      itm = item(j);
+      return true;
+    }
+    if (!mbar_wait_bounded(&ifull[j & (kRing - 1)], (uint32_t)((j / kRing) & 1), abort_flag))
+      return false;
+    itm = items_s[j & (kRing - 1)];
+    return itm.y >= 0;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -996,14 +1032,33 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         deferred = 0;
         return true;
       };
-      for (int j = 0; j < my_items && ok; ++j) {
-        const int4 itm = item(j);
+      // counted GEMM2: claim the next item, publish it to the ring
+      const int total = dyn ? __ldcg(list_count) * n_tiles : 0;
+      auto claim = [&](int j, int4& itm) -> bool {
+        const int slot = j & (kRing - 1);
+        if (j >= kRing &&
+            !mbar_wait_bounded(&iempty[slot], (uint32_t)(((j / kRing) - 1) & 1), abort_flag))
+          return false;
+        const int w = atomicAdd(ready + ready_count, 1);
+        itm = w < total ? load_w(w) : make_int4(0, -1, 0, 0);
+        items_s[slot] = itm;
+        mbar_arrive(&ifull[slot]);
+        return itm.y >= 0;
+      };
+      for (int j = 0; ok; ++j) {
+        int4 itm;
+        if (dyn) {
+          if (!claim(j, itm)) break;
+        } else {
+          if (j >= my_items) break;
+          itm = item(j);
+        }
         const int n = itm.y;
-        const int wrow = itm.z * w_rows_per_expert + itm.w * (SWIGLU ? 64 : 128);
+        const int wrow = itm.z * w_rows_per_expert + (itm.w % n_tiles) * (SWIGLU ? 64 : 128);
         // counted GEMM2: this item's entry counter, or nullptr once it is complete
         const int* pending = nullptr;
         if (counted && n > 0) {
-          const int* c = ready + (int)(blockIdx.x + j * gridDim.x) / n_tiles;
+          const int* c = ready + itm.w / n_tiles;
           int v;
           asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
           if (v >= ready_target)
@@ -1076,8 +1131,10 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int j = 0; j < my_items && ok; ++j) {
-        const int n = item(j).y;
+      for (int j = 0; ok; ++j) {
+        int4 itm;
+        if (!fetch(j, itm)) break;
+        const int n = itm.y;
         // one accumulator buffer per pass (an empty item has none; the same in the epilogue)
         for (int p0 = 0; p0 < n && ok; p0 += NMAX, ++it) {
           const int ncol = ((min(n - p0, NMAX) + 15) >> 4) * 16;
@@ -1128,9 +1185,10 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     int it = 0;
     int chunk_parity = 0;
     bool stop = false;
-    for (int j = 0; j < my_items && !stop; ++j) {
-      const int4 itm = item(j);
-      const int n_item = itm.y, nt = itm.w;
+    for (int j = 0; !stop; ++j) {
+      int4 itm;
+      if (!fetch(j, itm)) break;
+      const int n_item = itm.y, nt = itm.w % n_tiles;
       if (n_item < 1 && threadIdx.x == 64) record_error(err, MOE_ERR_DEVICE_CHECK, 12);
       for (int p0 = 0; p0 < n_item; p0 += NMAX, ++it) {
         const int row0 = itm.x + p0;
@@ -1210,9 +1268,10 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         named_bar_sync(4, 128);
         if (threadIdx.x == 64) {
           __threadfence();
-          atomicAdd(ready + (int)(blockIdx.x + j * gridDim.x) / n_tiles, 1);
+          atomicAdd(ready + itm.w / n_tiles, 1);
         }
       }
+      if (dyn && threadIdx.x == 64) mbar_arrive(&iempty[j & (kRing - 1)]);
     }
   }
 
@@ -1304,7 +1363,7 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
                                  int ld_out, int* err, int early, int num_sms,
                                  cudaStream_t st, const float* w_scale = nullptr,
                                  const float* x_scale = nullptr, int* ready = nullptr,
-                                 int ready_target = 0) {
+                                 int ready_target = 0, int ready_count = 0) {
   using C = SwapCfg<NMAX, SWIGLU>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1319,7 +1378,7 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
   return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU, F8>, dim3(grid), dim3(192),
                        C::kSmemBytes, st, 1, tw, tx, list_count, list, row_tiles, n_tiles, K,
                        w_rows, up_off, n_out, out, ld_out, err, early, w_scale, x_scale, ready,
-                       ready_target);
+                       ready_target, ready_count);
 }
 
 // Small batches (T <= 256): both GEMMs in swap-AB form.  GEMM2 waits for
@@ -1348,8 +1407,14 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
   const int nt1 = s.f / 64;               // 64 gate + 64 up rows per item
   const int nt2 = (s.d + 127) / 128;      // 128 output columns per item
   const int E = s.E;
-  // GEMM2 starts each list entry once GEMM1 has stored all nt1 column tiles of it
+  // GEMM2 starts each list entry once GEMM1 has stored all nt1 column tiles of
+  // it, taking its items from the queue after the counters unless at most one
+  // wave of items can exist (then every CTA has one item at most anyway)
   int* ready = ready_counters(const_cast<int*>(tiles), L.max_mtiles, E);
+  const long long max_items2 =
+      s.T <= 64 ? (long long)std::min<long long>(E, (long long)s.T * s.k) * nt2
+                : (long long)L.max_mtiles * nt2;
+  const int rq = max_items2 <= num_sms ? 0 : L.max_mtiles + E;
   cudaError_t e;
   if (s.T <= 64) {
     // one item per touched expert (at most 64 rows)
@@ -1360,7 +1425,7 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_swap_t<64, false>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d, z,
-                                   s.d, err, 0, num_sms, st, nullptr, nullptr, ready, nt1);
+                                   s.d, err, 0, num_sms, st, nullptr, nullptr, ready, nt1, rq);
   } else {
     // one item per 128-row tile: 5 K-stages of weights in flight instead of
     // the 4 that 256-row items leave room for
@@ -1372,7 +1437,7 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
     if (e == cudaSuccess)
       e = launch_swap_t<128, false>(tW2, tX2, cnt, ents, 1, L.max_mtiles * nt2, nt2, s.f, s.d,
                                     0, s.d, z, s.d, err, 0, num_sms, st, nullptr, nullptr, ready,
-                                    nt1);
+                                    nt1, rq);
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
