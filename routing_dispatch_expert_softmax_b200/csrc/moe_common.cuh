@@ -118,12 +118,18 @@ __host__ __device__ inline int max_mtiles_of(long long P, int E) {
 // zeroed by every kernel that writes the lists.  The small-batch GEMM1 adds 1
 // to entry i's counter when one of its column tiles of that entry's rows is
 // stored; GEMM2 starts an entry's work once the count is complete.
-// One more int after them: the small-batch GEMM2's item queue.
+// One more int after them: the small-batch GEMM2's item queue; then a second
+// array of counters and its queue, laid out the same way (the W8A8 layer's
+// quantised entries, which its GEMM2 waits on).
 __host__ __device__ inline size_t tile_list_ints(int max_mtiles, int E) {
-  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E) + (size_t)max_mtiles + E + 1;
+  return 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E) + 2 * ((size_t)max_mtiles + E + 1);
 }
 __host__ __device__ inline int* ready_counters(int* tiles, int max_mtiles, int E) {
   return tiles + 4 + 3 * ((size_t)max_mtiles + 2 * (size_t)E);
+}
+// ints after ready_counters() that the list writers zero: both arrays and their queues
+__host__ __device__ inline int ready_ints(int max_mtiles, int E) {
+  return 2 * (max_mtiles + E + 1);
 }
 __host__ __device__ inline int* expert_entries(int* tiles) { return tiles + 4; }
 __host__ __device__ inline int* leftover_entries(int* tiles, int E) { return tiles + 4 + 3 * E; }

@@ -1196,6 +1196,20 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         const int ncols = ((n + 15) >> 4) * 16;
         const int ab = it & 1;
         const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        // F8: the item's token scales, lane l holding those of columns l,
+        // l + 32, ... (one parallel load per lane instead of one dependent load
+        // per column).  A counted GEMM2's scales come from a kernel that may
+        // still run: read through L2 once the item's accumulator is complete
+        // (its producer waited for the entry); otherwise before the wait.
+        float xsr[F8 ? (NMAX + 31) / 32 : 1];
+        auto load_scales = [&]() {
+#pragma unroll
+          for (int i = 0; i < (F8 ? (NMAX + 31) / 32 : 1); ++i) {
+            const float* p = x_scale + row0 + lane + 32 * i;
+            xsr[i] = (F8 && lane + 32 * i < n) ? (counted ? __ldcg(p) : __ldg(p)) : 0.0f;
+          }
+        };
+        if (!counted) load_scales();
         mbar_wait_bounded(&tfull[ab], aph, abort_flag);
         // The four epilogue warps decide together whether to go on, so none is
         // left waiting at the exchange barrier below.
@@ -1208,11 +1222,22 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         const uint32_t t_addr = tmem_base + (uint32_t)(ab * NMAX) + ((uint32_t)(q * 32) << 16);
         // first weight row of the item (the TMA row index; the F8 scales' index)
         const int wrow0 = itm.z * w_rows_per_expert + nt * (SWIGLU ? 64 : 128);
+        if (counted) load_scales();
+        // token c0 + cc's scale for the 16 columns from c0 (warp-wide shuffles)
+        auto chunk_scales = [&](int c0, float* xv) {
+          if (!F8) return;
+          float xsel = xsr[0];
+#pragma unroll
+          for (int i = 1; i < (F8 ? (NMAX + 31) / 32 : 1); ++i)
+            if ((c0 >> 5) == i) xsel = xsr[i];
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) xv[cc] = __shfl_sync(0xffffffffu, xsel, (c0 + cc) & 31);
+        };
         // accumulator of token column c times its scales (F8), else as is
-        auto scaled = [&](uint32_t bits, float sw, int c) {
+        auto scaled = [&](uint32_t bits, float sw, int c, float xc) {
           const float a = __uint_as_float(bits);
           if (!F8) return a;
-          return c < n ? a * sw * __ldg(x_scale + row0 + c) : 0.0f;
+          return c < n ? a * sw * xc : 0.0f;
         };
         if (SWIGLU) {
           // lanes 0..63: gate rows j, lanes 64..127: up rows j (j = lane & 63)
@@ -1222,11 +1247,13 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
           for (int c0 = 0; c0 < ncols; c0 += 16) {
             float* x = xch + chunk_parity * (64 * 16);
             uint32_t v[16];
+            float xv[16];
+            chunk_scales(c0, xv);
             tmem_ld_32x32b_x16(t_addr + c0, v);
             tmem_ld_wait();
             if (q >= 2) {
 #pragma unroll
-              for (int cc = 0; cc < 16; ++cc) x[cc * 64 + j] = scaled(v[cc], sw, c0 + cc);
+              for (int cc = 0; cc < 16; ++cc) x[cc * 64 + j] = scaled(v[cc], sw, c0 + cc, xv[cc]);
             }
             named_bar_sync(1, 128);
             if (q < 2 && col < n_out) {
@@ -1234,7 +1261,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
               for (int cc = 0; cc < 16; ++cc) {
                 const int c = c0 + cc;
                 if (c < n) {
-                  const float g = scaled(v[cc], sw, c);
+                  const float g = scaled(v[cc], sw, c, xv[cc]);
                   const float u = x[cc * 64 + j];
                   out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(silu_f(g) * u);
                 }
@@ -1247,6 +1274,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
           const float sw = (F8 && col < n_out) ? __ldg(w_scale + wrow0 + q * 32 + lane) : 1.0f;
           for (int c0 = 0; c0 < ncols; c0 += 16) {
             uint32_t v[16];
+            float xv[16];
+            chunk_scales(c0, xv);
             tmem_ld_32x32b_x16(t_addr + c0, v);
             tmem_ld_wait();
             if (col < n_out) {
@@ -1254,7 +1283,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
               for (int cc = 0; cc < 16; ++cc) {
                 const int c = c0 + cc;
                 if (c < n)
-                  out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(scaled(v[cc], sw, c));
+                  out[(size_t)(row0 + c) * ld_out + col] =
+                      __float2bfloat16_rn(scaled(v[cc], sw, c, xv[cc]));
               }
             }
           }
@@ -1462,6 +1492,55 @@ static cudaError_t launch_gemm_2sm(const CUtensorMap& ta, const CUtensorMap& tb,
                        st, 2, ta, tb, args);
 }
 
+// The W8A8 expert GEMMs in the swap-AB form over the touched-expert list
+// (NMAX = 64: T <= 64) or the 128-row tile list (NMAX = 128).  overlap: GEMM1
+// counts each entry's stored column tiles (first counter array), the entry
+// quantiser waits for complete entries and counts them (second array), and
+// GEMM2 waits per entry, taking its items from the second array's queue when
+// they can exceed one wave.  Otherwise the row quantiser runs between the
+// GEMMs and GEMM2 is an early launch.  mark(0) after GEMM1.
+template <int NMAX, typename Mark>
+static cudaError_t swap_ffn_w8a8(const CUtensorMap& tW1, const CUtensorMap& tX1,
+                                 const CUtensorMap& tW2, const CUtensorMap& tX2,
+                                 const moe_shape& s, const WsLayout& L, const int* tiles,
+                                 __nv_bfloat16* h, uint8_t* hq, float* hs, const float* xs,
+                                 const float* w13_scale, const float* w2_scale,
+                                 __nv_bfloat16* z, int* err, int e1, bool overlap, int num_sms,
+                                 cudaStream_t st, Mark&& mark) {
+  const int nt1 = s.f / 64, nt2 = (s.d + 127) / 128, E = s.E;
+  const bool experts = NMAX == 64;  // one entry per touched expert
+  const int* cnt = experts ? tiles + 1 : tiles;
+  const int* ents = experts ? expert_entries(const_cast<int*>(tiles))
+                            : row_tile_entries(const_cast<int*>(tiles), E);
+  const int row_tiles = experts ? 0 : 1;
+  const int max_entries = experts ? E : L.max_mtiles;
+  int* ready1 = overlap ? ready_counters(const_cast<int*>(tiles), L.max_mtiles, E) : nullptr;
+  const int rq_at = L.max_mtiles + E;  // each counter array's queue, after its counters
+  int* ready2 = overlap ? ready1 + rq_at + 1 : nullptr;
+  cudaError_t e = launch_swap_t<NMAX, true, true>(
+      tW1, tX1, cnt, ents, row_tiles, max_entries * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h, s.f,
+      err, e1, num_sms, st, w13_scale, xs, ready1);
+  if (e == cudaSuccess) e = mark(0);
+  if (!overlap) {
+    if (e == cudaSuccess) e = launch_quant_rows(h, nullptr, L.P, 0, s.f, hq, hs, err, st);
+    if (e == cudaSuccess)
+      e = launch_swap_t<NMAX, false, true>(tW2, tX2, cnt, ents, row_tiles, max_entries * nt2,
+                                           nt2, s.f, s.d, 0, s.d, z, s.d, err, 1, num_sms, st,
+                                           w2_scale, hs);
+    return e;
+  }
+  if (e == cudaSuccess)
+    e = launch_quant_entries(h, s.f, cnt, ents, row_tiles, max_entries, ready1, nt1, ready2, hq,
+                             hs, err, st);
+  const long long max_items2 =
+      (experts ? std::min<long long>(E, (long long)s.T * s.k) : (long long)L.max_mtiles) * nt2;
+  if (e == cudaSuccess)
+    e = launch_swap_t<NMAX, false, true>(tW2, tX2, cnt, ents, row_tiles, max_entries * nt2, nt2,
+                                         s.f, s.d, 0, s.d, z, s.d, err, 0, num_sms, st, w2_scale,
+                                         hs, ready2, 1, max_items2 <= num_sms ? 0 : rq_at);
+  return e;
+}
+
 // Both GEMMs with E4M3 operands on both sides, at every batch size, and
 // between them the SwiGLU output quantised row by row: the swap-AB kernels
 // over the touched-expert list (T <= 64) or the 128-row tile list; for large
@@ -1469,7 +1548,9 @@ static cudaError_t launch_gemm_2sm(const CUtensorMap& ta, const CUtensorMap& tb,
 // over the tile pairs, with the lone-tile experts' leftover list on the
 // swap-AB kernels (their tokens fit one 128-row item).  The swap-AB GEMM2 of
 // the small-batch forms is an early launch (the quantisation kernel lets it
-// launch after its own wait; the work list precedes GEMM1).
+// launch after its own wait; the work list precedes GEMM1); with at most 64
+// (token, expert) rows the quantisation runs per list entry beside GEMM1
+// instead, and GEMM2 waits per entry.
 int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
                            const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
                            const float* w2_scale, const moe_shape& s, const WsLayout& L,
@@ -1497,17 +1578,22 @@ int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
     return launch_quant_rows(h, nullptr, L.P, 0, s.f, hq, hs, err, st);
   };
   cudaError_t e;
-  if (s.T <= 64) {
-    const int* cnt = tiles + 1;
-    const int* ents = expert_entries(const_cast<int*>(tiles));
-    e = launch_swap_t<64, true, true>(tW1, tX1, cnt, ents, 0, E * nt1, nt1, s.d, 2 * s.f, s.f,
-                                      s.f, h, s.f, err, e1, num_sms, st, w13_scale, xs);
-    if (e == cudaSuccess) e = mark(0);
-    if (e == cudaSuccess) e = quant_h();
-    if (e == cudaSuccess)
-      e = launch_swap_t<64, false, true>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d,
-                                         z, s.d, err, 1, num_sms, st, w2_scale, hs);
-  } else if (pair_tiles(s)) {
+  if (!pair_tiles(s)) {
+    // The swap-AB forms: one item per touched expert (T <= 64) or per 128-row
+    // tile.  They overlap the three kernels (GEMM1 counting each list entry's
+    // stored column tiles, the entry quantiser turning complete entries into
+    // codes and counting them, GEMM2 waiting per entry) when an entry is
+    // small or there are enough entries for them to complete while GEMM1
+    // runs; a few large entries complete only near GEMM1's end, and then the
+    // row quantiser between the kernels is cheaper.
+    const bool small = s.T <= 64;
+    const long long entries = std::min<long long>(E, (long long)s.T * s.k);
+    const bool overlap = (long long)s.T * s.k <= 64 || entries >= 16;
+    e = small ? swap_ffn_w8a8<64>(tW1, tX1, tW2, tX2, s, L, tiles, h, hq, hs, xs, w13_scale,
+                                  w2_scale, z, err, e1, overlap, num_sms, st, mark)
+              : swap_ffn_w8a8<128>(tW1, tX1, tW2, tX2, s, L, tiles, h, hq, hs, xs, w13_scale,
+                                   w2_scale, z, err, e1, overlap, num_sms, st, mark);
+  } else {
     CUtensorMap pA1, pB1, pA2, pB2;  // 128-row boxes: each CTA of a pair loads 128 rows
     if (!make_tmap_u8(&pA1, xq, (uint64_t)x_rows, (uint64_t)s.d, 128) ||
         !make_tmap_u8(&pB1, w13, (uint64_t)s.E * 2 * s.f, (uint64_t)s.d, 128) ||
@@ -1535,18 +1621,6 @@ int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
     if (e == cudaSuccess)
       e = launch_swap_t<128, false, true>(tW2, tX2, lcount, lrows, 1, E * nt2, nt2, s.f, s.d, 0,
                                           s.d, z, s.d, err, 0, num_sms, st, w2_scale, hs);
-  } else {
-    const int* cnt = tiles;
-    const int* ents = row_tile_entries(const_cast<int*>(tiles), E);
-    e = launch_swap_t<128, true, true>(tW1, tX1, cnt, ents, 1, L.max_mtiles * nt1, nt1, s.d,
-                                       2 * s.f, s.f, s.f, h, s.f, err, e1, num_sms, st,
-                                       w13_scale, xs);
-    if (e == cudaSuccess) e = mark(0);
-    if (e == cudaSuccess) e = quant_h();
-    if (e == cudaSuccess)
-      e = launch_swap_t<128, false, true>(tW2, tX2, cnt, ents, 1, L.max_mtiles * nt2, nt2, s.f,
-                                          s.d, 0, s.d, z, s.d, err, 1, num_sms, st, w2_scale,
-                                          hs);
   }
   if (e == cudaSuccess) e = mark(1);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

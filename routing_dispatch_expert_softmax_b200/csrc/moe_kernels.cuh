@@ -60,6 +60,15 @@ cudaError_t launch_quant_rows(const __nv_bfloat16* a, const int* perm, long long
                               int cols, uint8_t* codes, float* scales, int* err,
                               cudaStream_t st);
 
+// The small-batch W8A8 SwiGLU output quantised per work-list entry while
+// GEMM1 runs (moe_w8a8.cu): one block per entry (max_entries blocks; the
+// count is list_count[0]), waiting on ready1[i] >= target1 and setting
+// ready2[i].
+cudaError_t launch_quant_entries(const __nv_bfloat16* h, int cols, const int* list_count,
+                                 const int* list, int row_tiles, int max_entries,
+                                 const int* ready1, int target1, int* ready2, uint8_t* codes,
+                                 float* scales, int* err, cudaStream_t st);
+
 // Both expert GEMMs with E4M3 weights (one fp32 scale per weight row) and
 // E4M3 tokens (xq, one scale per row in xs): GEMM1 with the SwiGLU epilogue
 // into h (bf16), h quantised into the workspace, GEMM2 (moe_gemm_sm100.cu).

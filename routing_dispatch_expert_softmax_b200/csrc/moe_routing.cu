@@ -420,7 +420,7 @@ __device__ int block_exclusive_scan_1024(int v, int* scratch /*[32]*/, int* tota
 __device__ void write_work_lists(int e, int E, int c, int off, int* tiles, int* scratch,
                                  int* total, bool pair, int max_mtiles) {
   int* ready = ready_counters(tiles, max_mtiles, E);
-  for (int i = threadIdx.x; i <= max_mtiles + E; i += blockDim.x) ready[i] = 0;  // + queue
+  for (int i = threadIdx.x; i < ready_ints(max_mtiles, E); i += blockDim.x) ready[i] = 0;
   const int nt = (e < E) ? (c + kGemmBM - 1) / kGemmBM : 0;
   const int nrow = pair ? pair_row_tiles(nt) : nt;  // tiles in the row-tile list
   const int left = (pair && nt == 1) ? 1 : 0;       // a lone tile: leftover list
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(1024) k_route_fused(
   const int* ids = ids_in_smem ? idx_s : idx;
   {
     int* ready = ready_counters(tiles, max_mtiles, E);
-    for (int i = threadIdx.x; i <= max_mtiles + E; i += 1024) ready[i] = 0;  // + queue
+    for (int i = threadIdx.x; i < ready_ints(max_mtiles, E); i += 1024) ready[i] = 0;
   }
   const int t = threadIdx.x;
   const bool valid = t < T;

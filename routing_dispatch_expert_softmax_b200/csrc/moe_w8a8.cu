@@ -31,6 +31,49 @@ __device__ __forceinline__ int pow2_exponent_of_bf16_mag(uint32_t m) {
   return p - 141 + (4 * f > (7 << p) ? 1 : 0);
 }
 
+// One row of cols elements (a multiple of 8) to codes and (lane 0) its
+// scale, one warp cooperating.  L2: read around L1 (rows another CTA of a
+// running kernel wrote); else through the read-only path.
+template <bool L2>
+__device__ __forceinline__ void quant_row(const __nv_bfloat16* src, int cols, uint8_t* codes,
+                                          float* scale, int lane) {
+  const uint4* in = reinterpret_cast<const uint4*>(src);
+  auto ld = [&](int c) { return L2 ? __ldcg(in + c) : __ldg(in + c); };
+  const int nv = cols / 8;
+  // the largest magnitude: bf16 magnitude bits order like the magnitudes
+  uint32_t m = 0;
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = ld(c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  const int e = pow2_exponent_of_bf16_mag(m);
+  // multiply by 2^-e in two exact steps (each factor a normal fp32)
+  const int k1 = (-e) >> 1, k2 = -e - k1;
+  const float s1 = pow2f(k1), s2 = pow2f(k2);
+  uint2* out = reinterpret_cast<uint2*>(codes);
+  for (int c = lane; c < nv; c += 32) {
+    const uint4 v = ld(c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t q[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(w[i] << 16) * s1 * s2;
+      const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * s1 * s2;
+      const uint32_t pair =
+          __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+      if (i & 1)
+        q[i >> 1] |= pair << 16;
+      else
+        q[i >> 1] = pair;
+    }
+    out[c] = make_uint2(q[0], q[1]);
+  }
+  if (lane == 0) *scale = pow2f(e >> 1) * pow2f(e - (e >> 1));
+}
+
 // One warp per row.  GATHER: output row r quantises input row perm[r] (the
 // dispatch gather fused in), else input row r.
 template <bool GATHER>
@@ -54,40 +97,60 @@ __global__ void __launch_bounds__(256) k_quant_rows_e4m3(
     }
     src = t;
   }
-  const uint4* in = reinterpret_cast<const uint4*>(a + src * cols);
-  const int nv = cols / 8;
-  // the largest magnitude: bf16 magnitude bits order like the magnitudes
-  uint32_t m = 0;
-  for (int c = lane; c < nv; c += 32) {
-    const uint4 v = __ldg(in + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
-  }
-  m = __reduce_max_sync(0xffffffffu, m);
-  const int e = pow2_exponent_of_bf16_mag(m);
-  // multiply by 2^-e in two exact steps (each factor a normal fp32)
-  const int k1 = (-e) >> 1, k2 = -e - k1;
-  const float s1 = pow2f(k1), s2 = pow2f(k2);
-  uint2* out = reinterpret_cast<uint2*>(codes + row * cols);
-  for (int c = lane; c < nv; c += 32) {
-    const uint4 v = __ldg(in + c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t q[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float lo = __uint_as_float(w[i] << 16) * s1 * s2;
-      const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * s1 * s2;
-      const uint32_t pair =
-          __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
-      if (i & 1)
-        q[i >> 1] |= pair << 16;
-      else
-        q[i >> 1] = pair;
+  quant_row<false>(a + src * cols, cols, codes + row * cols, scales + row, lane);
+}
+
+// The SwiGLU output of the small-batch W8A8 GEMM1, quantised per work-list
+// entry while GEMM1 runs: block i takes entry i (list entries: row0, row_end,
+// expert; row_tiles caps an entry at 128 rows), waits (bounded) until GEMM1
+// has stored all `target1` column tiles of the entry's rows (ready1[i]),
+// quantises those rows as k_quant_rows_e4m3 does (the reads go through L2:
+// GEMM1 wrote them while this kernel ran), then sets ready2[i] for GEMM2.  It
+// lets GEMM2 launch at once and waits for GEMM1 only at its end, so its
+// completion still implies GEMM1's.
+__global__ void __launch_bounds__(256) k_quant_entries_e4m3(
+    const __nv_bfloat16* __restrict__ h, int cols, const int* __restrict__ list_count,
+    const int* __restrict__ list, int row_tiles, const int* __restrict__ ready1, int target1,
+    int* __restrict__ ready2, uint8_t* __restrict__ codes, float* __restrict__ scales,
+    int* __restrict__ err) {
+  pdl_trigger();
+  __shared__ int go;
+  const int i = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (i < __ldcg(list_count)) {
+    const int row0 = __ldcg(list + 3 * i + 0);
+    const int rows = __ldcg(list + 3 * i + 1) - row0;
+    const int n = row_tiles ? min(rows, kGemmBM) : rows;
+    if (threadIdx.x == 0) {
+      int flag = 0;
+      go = wait_count_bounded(ready1 + i, target1, &flag) ? 1 : 0;
+      if (!go) record_error(err, MOE_ERR_TIMEOUT, 14);
     }
-    out[c] = make_uint2(q[0], q[1]);
+    __syncthreads();
+    if (go) {
+      __threadfence();
+      for (int r = warp; r < n; r += 8)
+        quant_row<true>(h + (size_t)(row0 + r) * cols, cols, codes + (size_t)(row0 + r) * cols,
+                        scales + row0 + r, lane);
+      fence_proxy_async_global();  // the codes before GEMM2's TMA reads
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ready2 + i, 1);
+      }
+    }
   }
-  if (lane == 0) scales[row] = pow2f(e >> 1) * pow2f(e - (e >> 1));
+  pdl_wait();
+}
+
+cudaError_t launch_quant_entries(const __nv_bfloat16* h, int cols, const int* list_count,
+                                 const int* list, int row_tiles, int max_entries,
+                                 const int* ready1, int target1, int* ready2, uint8_t* codes,
+                                 float* scales, int* err, cudaStream_t st) {
+  if (max_entries < 1) return cudaSuccess;
+  return launch_kernel(k_quant_entries_e4m3, dim3((unsigned)max_entries), dim3(256), 0, st, 1,
+                       h, cols, list_count, list, row_tiles, ready1, target1, ready2, codes,
+                       scales, err);
 }
 
 cudaError_t launch_quant_rows(const __nv_bfloat16* a, const int* perm, long long rows, int n_src,

@@ -132,6 +132,14 @@ def test_ffn_w8a8_ragged_shapes():
     # 128-row W_down tile; f = 192: a partial K block of GEMM2; 37 tokens
     _ffn_case(wl.MoEConfig("ragged", T=37, d=320, E=3, k=2, f=192))
     _ffn_case(wl.MoEConfig("one-expert", T=100, d=128, E=1, k=1, f=128))
+    # at most 64 (token, expert) rows: the per-entry quantiser beside GEMM1,
+    # with the same partial K blocks and tiles
+    _ffn_case(wl.MoEConfig("ragged-entries", T=7, d=320, E=5, k=3, f=192))
+    _ffn_case(wl.MoEConfig("one-row", T=1, d=128, E=1, k=1, f=128))
+    # 128-row tiles with the per-entry quantiser (at least 16 experts): ragged
+    # widths, and experts of more than one tile (about 128 rows each)
+    _ffn_case(wl.MoEConfig("ragged-tiles", T=300, d=320, E=20, k=2, f=192))
+    _ffn_case(wl.MoEConfig("multi-tile-entries", T=256, d=256, E=16, k=8, f=384))
 
 
 @pytest.mark.parametrize("T,counts", [
