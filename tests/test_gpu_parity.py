@@ -480,6 +480,42 @@ def test_forward_large_batch_gemm_regimes(cfg):
     _check_forward(cfg)
 
 
+@pytest.mark.parametrize("cfg", [wl.QWEN3_30B_A3B_DECODE.with_T(1),
+                                 wl.QWEN3_30B_A3B_DECODE.with_T(64),
+                                 wl.QWEN3_30B_A3B_DECODE.with_T(256),
+                                 wl.MoEConfig("ragged-combine", T=37, d=320, E=6, k=3, f=128)],
+                         ids=["T1", "T64", "T256", "ragged"])
+def test_forward_equals_ffn_then_combine(cfg):
+    """moe_forward's y equals moe_combine over moe_ffn's z on the layer's own
+    dispatch bit for bit (the layer's gather, GEMMs and combine against the
+    caller-offset FFN and the standalone combine), including a partial last
+    128-column tile (d = 320), and again on a second call on the same
+    workspace."""
+    x = wl.make_hidden(cfg, DEV, 4)
+    w_g, bias = wl.make_router(cfg, DEV, 0)
+    w13, w2 = wl.make_experts(cfg, DEV, 0)
+    shape = MoEShape.from_config(cfg)
+    ws = moe.workspace(shape)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device=DEV)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=DEV)
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=DEV)
+    for _ in range(2):  # the second call runs on counters the first one used
+        y.fill_(float("nan"))
+        moe.moe_forward(x, w_g, bias, w13, w2, y, shape, ws, idx_out=idx, w_out=w)
+        _check_clean(ws)
+    idx_h = idx.cpu().numpy()
+    offsets = oracle.expert_offsets(oracle.expert_counts(idx_h, cfg.E))
+    perm, row_of = oracle.dispatch_rows(idx_h, cfg.E)
+    x_perm = x[torch.from_numpy(perm).long().to(DEV)].contiguous()
+    ws2 = moe.workspace(shape)
+    z = torch.empty(cfg.P, cfg.d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_ffn(x_perm, torch.from_numpy(offsets).to(DEV), w13, w2, z, shape, ws2)
+    _check_clean(ws2)
+    y2 = torch.empty_like(y)
+    moe.moe_combine(z, torch.from_numpy(row_of).to(DEV), w, y2, shape)
+    assert torch.equal(y, y2)
+
+
 def test_forward_k_equals_E_and_single_expert():
     _check_forward(wl.MoEConfig("dense-k=E", T=70, d=128, E=4, k=4, f=128))
     _check_forward(wl.MoEConfig("E=1", T=33, d=256, E=1, k=1, f=192))
