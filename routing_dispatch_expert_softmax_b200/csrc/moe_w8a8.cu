@@ -100,6 +100,56 @@ __global__ void __launch_bounds__(256) k_quant_rows_e4m3(
   quant_row<false>(a + src * cols, cols, codes + row * cols, scales + row, lane);
 }
 
+// One row of cols <= 32 * 8 * kRegVecs elements held in registers (loaded
+// once through L2, then the maximum and the codes as quant_row computes them).
+// Same-box A/B against the two-pass quant_row: Qwen3 W8A8 T = 256 163 -> 156
+// us with 768-column rows; 2048-column rows (DeepSeek-V3) were slower this way.
+constexpr int kRegVecs = 4;  // 16-byte vectors per lane: rows of up to 1024 bf16
+__device__ __forceinline__ void quant_row_regs(const __nv_bfloat16* src, int cols,
+                                               uint8_t* codes, float* scale, int lane) {
+  const uint4* in = reinterpret_cast<const uint4*>(src);
+  const int nv = cols / 8;
+  uint4 v[kRegVecs];
+#pragma unroll
+  for (int i = 0; i < kRegVecs; ++i) {
+    const int c = lane + 32 * i;
+    v[i] = c < nv ? __ldcg(in + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < kRegVecs; ++i) {
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  const int e = pow2_exponent_of_bf16_mag(m);
+  const int k1 = (-e) >> 1, k2 = -e - k1;
+  const float s1 = pow2f(k1), s2 = pow2f(k2);
+  uint2* out = reinterpret_cast<uint2*>(codes);
+#pragma unroll
+  for (int i = 0; i < kRegVecs; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nv) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t q[2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(w[j] << 16) * s1 * s2;
+        const float hi = __uint_as_float(w[j] & 0xFFFF0000u) * s1 * s2;
+        const uint32_t pair =
+            __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+        if (j & 1)
+          q[j >> 1] |= pair << 16;
+        else
+          q[j >> 1] = pair;
+      }
+      out[c] = make_uint2(q[0], q[1]);
+    }
+  }
+  if (lane == 0) *scale = pow2f(e >> 1) * pow2f(e - (e >> 1));
+}
+
 // The SwiGLU output of the small-batch W8A8 GEMM1, quantised per work-list
 // entry while GEMM1 runs: block i takes entry i (list entries: row0, row_end,
 // expert; row_tiles caps an entry at 128 rows), waits (bounded) until GEMM1
@@ -124,14 +174,19 @@ __global__ void __launch_bounds__(256) k_quant_entries_e4m3(
     if (threadIdx.x == 0) {
       int flag = 0;
       go = wait_count_bounded(ready1 + i, target1, &flag) ? 1 : 0;
-      if (!go) record_error(err, MOE_ERR_TIMEOUT, 14);
+      if (!go) record_error(err, MOE_ERR_TIMEOUT, 16);
     }
     __syncthreads();
     if (go) {
       __threadfence();
-      for (int r = warp; r < n; r += 8)
-        quant_row<true>(h + (size_t)(row0 + r) * cols, cols, codes + (size_t)(row0 + r) * cols,
-                        scales + row0 + r, lane);
+      const int nw = blockDim.x >> 5;
+      for (int r = warp; r < n; r += nw) {  // one row per warp
+        const size_t o = (size_t)(row0 + r) * cols;
+        if (cols <= 256 * kRegVecs)
+          quant_row_regs(h + o, cols, codes + o, scales + row0 + r, lane);
+        else
+          quant_row<true>(h + o, cols, codes + o, scales + row0 + r, lane);
+      }
       fence_proxy_async_global();  // the codes before GEMM2's TMA reads
       __syncthreads();
       if (threadIdx.x == 0) {
@@ -143,12 +198,16 @@ __global__ void __launch_bounds__(256) k_quant_entries_e4m3(
   pdl_wait();
 }
 
+// Threads per entry block: one warp per row of the entry, 8 rows at once (a
+// block of 1024 threads does not fit beside a GEMM1 CTA's registers).
+constexpr int kQuantEntryThreads = 256;
+
 cudaError_t launch_quant_entries(const __nv_bfloat16* h, int cols, const int* list_count,
                                  const int* list, int row_tiles, int max_entries,
                                  const int* ready1, int target1, int* ready2, uint8_t* codes,
                                  float* scales, int* err, cudaStream_t st) {
   if (max_entries < 1) return cudaSuccess;
-  return launch_kernel(k_quant_entries_e4m3, dim3((unsigned)max_entries), dim3(256), 0, st, 1,
+  return launch_kernel(k_quant_entries_e4m3, dim3((unsigned)max_entries), dim3(kQuantEntryThreads), 0, st, 1,
                        h, cols, list_count, list, row_tiles, ready1, target1, ready2, codes,
                        scales, err);
 }
