@@ -70,7 +70,8 @@ def launches_per_forward(cfg, eplb_redundant=0, fp8=False, w8a8=False):
     moe_forward_fp8 with fp8, moe_forward_w8a8 with w8a8) launches: the router
     (router_launches), routing (one fused kernel for T <= 1024, else top-k +
     histogram + scan + scatter; with replicas top-k + remap + histogram + scan
-    + scatter), the row gather (with w8a8 the gather-and-quantise kernel), the
+    + scatter), the row gather (with w8a8 the gather-and-quantise kernel; none
+    in bf16 up to 16 tokens, where GEMM1 reads x itself), the
     two expert GEMMs (the bf16 and W8A8 ones each followed by the lone-tile
     kernel when they run on CTA pairs; the FP8-weight ones always run the
     128-row-tile form; with w8a8 the SwiGLU output's quantisation between
@@ -80,7 +81,7 @@ def launches_per_forward(cfg, eplb_redundant=0, fp8=False, w8a8=False):
     routing = 1 if T <= 1024 else 4
     if eplb_redundant:
         routing = 5
-    gather = 1
+    gather = 0 if (T <= 16 and not fp8 and not w8a8 and not eplb_redundant) else 1
     gemms = 2
     if T > 256 and T * cfg.k >= 128 * (cfg.E + eplb_redundant) and not fp8:
         gemms = 4

@@ -244,7 +244,12 @@ static int forward_impl(int mode, const moe_bf16* x, const float* w_g, const flo
   }
   uint8_t* xq = at<uint8_t>(ws, L.x_perm);  // W8A8: token codes in the x_perm region
   float* xs = at<float>(ws, L.xs);
-  if (e == cudaSuccess)
+  // bf16 with at most 16 tokens: GEMM1 reads x itself (all tokens in one
+  // 16-row tile, the bytes a gathered tile of up to 16 rows has); with more,
+  // the whole token tile in every stage slows the weight stream (same-box A/B:
+  // T = 64 116.5 -> 133.4 us, T = 8 66.2 -> 63.8, T = 1 44.9 -> 43.1)
+  const bool direct = mode == kBf16 && s->T <= 16;
+  if (e == cudaSuccess && !direct)
     e = mode == kW8A8
             ? launch_quant_rows(xb, perm, L.P, s->T, s->d, xq, xs, at<int>(ws, L.err), cs)
             : launch_gather(xb, perm, L.P, s->T, s->d, x_perm, at<int>(ws, L.err), cs);
@@ -261,9 +266,12 @@ static int forward_impl(int mode, const moe_bf16* x, const float* w_g, const flo
                               static_cast<const uint8_t*>(w2), w2_scale, *s, L, wsb, z, sms, cs,
                               ev);
   else
-    r = launch_expert_ffn(x_perm, L.Ppad, static_cast<const __nv_bfloat16*>(w13),
-                          static_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms, cs, ev,
-                          true);
+    r = direct ? launch_expert_ffn(xb, s->T, static_cast<const __nv_bfloat16*>(w13),
+                                   static_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms, cs,
+                                   ev, false, perm)
+               : launch_expert_ffn(x_perm, L.Ppad, static_cast<const __nv_bfloat16*>(w13),
+                                   static_cast<const __nv_bfloat16*>(w2), *s, L, wsb, z, sms, cs,
+                                   ev, true);
   if (r != MOE_OK) return r;
   e = launch_combine(z, row_of, gw, *s, reinterpret_cast<__nv_bfloat16*>(y), cs);
   if (e == cudaSuccess) e = mark(5);

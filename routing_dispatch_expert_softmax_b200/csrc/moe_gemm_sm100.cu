@@ -884,7 +884,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
     int up_offset, int n_out, __nv_bfloat16* __restrict__ out, int ld_out,
     int* __restrict__ err, int early_w, const float* __restrict__ w_scale,
     const float* __restrict__ x_scale, int* __restrict__ ready, int ready_target,
-    int ready_count) {
+    int ready_count, const int* __restrict__ tok_row, int n_tok) {
   using C = SwapCfg<NMAX, SWIGLU>;
   constexpr int kKb = F8 ? 128 : kGemmBK;  // K elements per stage (128-byte rows)
   constexpr int S = C::kStages;
@@ -906,6 +906,11 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
   uint64_t* ifull = reinterpret_cast<uint64_t*>(items_s + kRing);
   uint64_t* iempty = ifull + kRing;
   const bool counted = !SWIGLU && ready != nullptr;  // GEMM2 of a counted pair
+  // Direct tokens (GEMM1, at most 64 tokens): the token operand of every item
+  // is all n_tok rows of the unpermuted x (one N <= 64 tile), and the
+  // epilogue stores column t (token t) to the h row r of the item's entry
+  // with tok_row[r] == t; the dispatch gather is not needed.
+  const bool direct = SWIGLU && NMAX == 64 && tok_row != nullptr;
   const bool dyn = counted && ready_count > 0;       // ... taking items from the queue
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1073,8 +1078,8 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
             pending = c;
         }
         for (int p0 = 0; p0 < n && ok; p0 += NMAX) {  // n < 1: recorded by the epilogue
-          const int row0 = itm.x + p0;
-          const int nb = (min(n - p0, NMAX) + 15) >> 4;
+          const int row0 = direct ? 0 : itm.x + p0;
+          const int nb = direct ? (n_tok + 15) >> 4 : (min(n - p0, NMAX) + 15) >> 4;
           for (int kb = 0; kb < nk; ++kb) {
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
               ok = false;
@@ -1143,7 +1148,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
         const int n = itm.y;
         // one accumulator buffer per pass (an empty item has none; the same in the epilogue)
         for (int p0 = 0; p0 < n && ok; p0 += NMAX, ++it) {
-          const int ncol = ((min(n - p0, NMAX) + 15) >> 4) * 16;
+          const int ncol = (((direct ? n_tok : min(n - p0, NMAX)) + 15) >> 4) * 16;
           const uint32_t idesc = F8 ? idesc_e4m3_f32(128, ncol) : idesc_bf16_f32(128, ncol);
           const int ab = it % C::kAccBufs;
           const uint32_t aph = (uint32_t)((it / C::kAccBufs) & 1);
@@ -1199,7 +1204,7 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
       for (int p0 = 0; p0 < n_item; p0 += NMAX, ++it) {
         const int row0 = itm.x + p0;
         const int n = min(n_item - p0, NMAX);
-        const int ncols = ((n + 15) >> 4) * 16;
+        const int ncols = (((direct ? n_tok : n) + 15) >> 4) * 16;
         const int ab = it % C::kAccBufs;
         const uint32_t aph = (uint32_t)((it / C::kAccBufs) & 1);
         // F8: the item's token scales, lane l holding those of columns l,
@@ -1250,10 +1255,30 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
           const int j = (q & 1) * 32 + lane;
           const int col = nt * 64 + j;
           const float sw = F8 ? __ldg(w_scale + wrow0 + (q >= 2 ? up_offset : 0) + j) : 1.0f;
+          // h row of accumulator column c: row0 + c for c < n, or (direct)
+          // the entry row holding token c (lane l keeps columns l and l + 32),
+          // -1 for a column with no row
+          int map0 = -1, map1 = -1;
+          if (direct) {
+            const int pv0 = lane < n ? __ldg(tok_row + row0 + lane) : -1;
+            const int pv1 = lane + 32 < n ? __ldg(tok_row + row0 + lane + 32) : -1;
+            for (int i = 0; i < n; ++i) {
+              const int t = __shfl_sync(0xffffffffu, i < 32 ? pv0 : pv1, i & 31);
+              if (t == lane) map0 = row0 + i;
+              if (t == lane + 32) map1 = row0 + i;
+            }
+          }
           for (int c0 = 0; c0 < ncols; c0 += 16) {
             float* x = xch + chunk_parity * (64 * 16);
             uint32_t v[16];
             float xv[16];
+            int rr[16];
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const int c = c0 + cc;
+              rr[cc] = direct ? __shfl_sync(0xffffffffu, c < 32 ? map0 : map1, c & 31)
+                              : (c < n ? row0 + c : -1);
+            }
             chunk_scales(c0, xv);
             tmem_ld_32x32b_x16(t_addr + c0, v);
             tmem_ld_wait();
@@ -1266,10 +1291,10 @@ __global__ void __launch_bounds__(192, 1) k_expert_gemm_swap(
 #pragma unroll
               for (int cc = 0; cc < 16; ++cc) {
                 const int c = c0 + cc;
-                if (c < n) {
+                if (rr[cc] >= 0) {
                   const float g = scaled(v[cc], sw, c, xv[cc]);
                   const float u = x[cc * 64 + j];
-                  out[(size_t)(row0 + c) * ld_out + col] = __float2bfloat16_rn(silu_f(g) * u);
+                  out[(size_t)rr[cc] * ld_out + col] = __float2bfloat16_rn(silu_f(g) * u);
                 }
               }
             }
@@ -1399,7 +1424,8 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
                                  int ld_out, int* err, int early, int num_sms,
                                  cudaStream_t st, const float* w_scale = nullptr,
                                  const float* x_scale = nullptr, int* ready = nullptr,
-                                 int ready_target = 0, int ready_count = 0) {
+                                 int ready_target = 0, int ready_count = 0,
+                                 const int* tok_row = nullptr, int n_tok = 0) {
   using C = SwapCfg<NMAX, SWIGLU>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1414,7 +1440,7 @@ static cudaError_t launch_swap_t(const CUtensorMap& tw, const CUtensorMap& tx,
   return launch_kernel(k_expert_gemm_swap<NMAX, SWIGLU, F8>, dim3(grid), dim3(192),
                        C::kSmemBytes, st, 1, tw, tx, list_count, list, row_tiles, n_tiles, K,
                        w_rows, up_off, n_out, out, ld_out, err, early, w_scale, x_scale, ready,
-                       ready_target, ready_count);
+                       ready_target, ready_count, tok_row, n_tok);
 }
 
 // Small batches (T <= 256): both GEMMs in swap-AB form.  GEMM2 waits for
@@ -1424,7 +1450,7 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
                                   const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                                   const moe_shape& s, const WsLayout& L, char* ws,
                                   __nv_bfloat16* z, int num_sms, cudaStream_t st,
-                                  void* const* events, bool early1) {
+                                  void* const* events, bool early1, const int* tok_row) {
   const int e1 = early1 ? 1 : 0;
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
@@ -1456,8 +1482,12 @@ static int launch_expert_ffn_swap(const __nv_bfloat16* x_perm, long long x_rows,
     // one item per touched expert (at most 64 rows)
     const int* cnt = tiles + 1;
     const int* ents = expert_entries(const_cast<int*>(tiles));
+    // tok_row: x_perm is the unpermuted x (T rows) and GEMM1 maps its rows
+    // itself; the work list then comes from the kernel just before, so no
+    // early start
     e = launch_swap_t<64, true>(tW1, tX1, cnt, ents, 0, E * nt1, nt1, s.d, 2 * s.f, s.f, s.f, h,
-                                s.f, err, e1, num_sms, st, nullptr, nullptr, ready);
+                                s.f, err, tok_row ? 0 : e1, num_sms, st, nullptr, nullptr, ready,
+                                0, 0, tok_row, s.T);
     if (e == cudaSuccess) e = mark(0);
     if (e == cudaSuccess)
       e = launch_swap_t<64, false>(tW2, tX2, cnt, ents, 0, E * nt2, nt2, s.f, s.d, 0, s.d, z,
@@ -1639,7 +1669,7 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                       const moe_shape& s, const WsLayout& L, char* ws,
                       __nv_bfloat16* z, int num_sms, cudaStream_t st,
-                      void* const* events, bool early_gemm1) {
+                      void* const* events, bool early_gemm1, const int* tok_row) {
   // events (optional): [0] recorded after GEMM1, [1] after GEMM2.
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
@@ -1648,7 +1678,7 @@ int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
   };
   if (s.T <= kSwapMaxT)
     return launch_expert_ffn_swap(x_perm, x_rows, w13, w2, s, L, ws, z, num_sms, st, events,
-                                  early_gemm1);
+                                  early_gemm1, s.T <= 64 ? tok_row : nullptr);
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int* tiles = reinterpret_cast<const int*>(ws + L.tiles);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);

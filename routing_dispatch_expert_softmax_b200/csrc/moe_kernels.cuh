@@ -39,11 +39,16 @@ cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const floa
 // early_gemm1: the kernel just before (the row gather) lets GEMM1 launch only
 // after its own wait, and the work list comes from a kernel before it, so
 // GEMM1 may start streaming weights before the gather completes.
+// tok_row (T <= 64 only; else ignored): x_perm is the unpermuted x (x_rows =
+// T) and tok_row[r] the token of dispatch row r; GEMM1 multiplies all T
+// tokens per item and stores each entry's rows itself, so no gather runs
+// (the forward uses it up to 16 tokens).
 int launch_expert_ffn(const __nv_bfloat16* x_perm, long long x_rows,
                       const __nv_bfloat16* w13, const __nv_bfloat16* w2,
                       const moe_shape& s, const WsLayout& L, char* ws,
                       __nv_bfloat16* z, int num_sms, cudaStream_t st,
-                      void* const* events = nullptr, bool early_gemm1 = false);
+                      void* const* events = nullptr, bool early_gemm1 = false,
+                      const int* tok_row = nullptr);
 
 // The same two GEMMs with E4M3 expert weights and one fp32 scale per weight
 // row (moe_gemm_fp8.cu): swap-AB form at every batch size, over the plain

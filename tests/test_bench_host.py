@@ -40,6 +40,8 @@ def test_launch_counts_match_the_profiled_launch_lists():
     # its lone-tile kernel, combine); the FP8 layer runs its two 128-row-tile
     # GEMMs at every batch size (11 at prefill).
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE) == 6
+    # up to 16 tokens GEMM1 reads x itself: no row gather
+    assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE.with_T(8)) == 5
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE, fp8=True) == 6
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_PREFILL) == 13
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_PREFILL, fp8=True) == 11
