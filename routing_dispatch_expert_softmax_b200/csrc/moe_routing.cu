@@ -16,30 +16,35 @@ namespace moe {
 
 // ============================================================== router GEMM
 // logits[t,e] = sum_i x[t,i] * w_g[i,e] (+ bias[e]), fp32.
-// A thread-block cluster of CS CTAs owns a 32-token x 32-expert tile; CTA r
-// of the cluster accumulates the K slice [r*d/CS, (r+1)*d/CS) in fp32 FMA
-// order, the partial tiles meet in distributed shared memory, and CTA r then
-// sums output slice r over the CS partials in rank order 0..CS-1.  The order
-// is fixed, so every call with the same d gives the same bits, and nothing
-// leaves the SMs but the logits.
-constexpr int kRtT = 32, kRtE = 32, kRtKC = 128;
+// A thread-block cluster of CS CTAs owns a 32-token x RE-expert tile (RE = 32
+// or 64); CTA r of the cluster accumulates the K slice [r*d/CS, (r+1)*d/CS)
+// in fp32 FMA order, the partial tiles meet in distributed shared memory,
+// and CTA r then sums output slice r over the CS partials in rank order
+// 0..CS-1.  Each logit's sequence of operations depends on d and CS only (not
+// on RE or the K chunking), so every call with the same d gives the same
+// bits, and nothing leaves the SMs but the logits.
+constexpr int kRtT = 32;
 
 // Chunk loads of the router: every thread issues all of its 16-byte loads for
-// a 128-deep K chunk before using any of them (W: 128 x 32 fp32 = 4 float4
-// per thread; x: 32 x 128 bf16 = 2 uint4 per thread), so a chunk costs one
-// memory latency, and the next chunk's loads are in flight while this one is
-// multiplied.
+// a KC-deep K chunk before using any of them (W: KC x RE fp32 = KC*RE/1024
+// float4 per thread; x: 32 x KC bf16 = KC/64 uint4 per thread), so a chunk
+// costs one memory latency, and the next chunk's loads are in flight while
+// this one is multiplied.
+template <int RE, int KC>
 struct RouterRegs {
-  float4 w[4];
-  uint4 x[2];
+  static constexpr int NW = KC * RE / 1024, NX = KC / 64;
+  float4 w[NW];
+  uint4 x[NX];
 };
 
-__device__ __forceinline__ void router_load(RouterRegs& r, const __nv_bfloat16* __restrict__ x,
+template <int RE, int KC>
+__device__ __forceinline__ void router_load(RouterRegs<RE, KC>& r,
+                                            const __nv_bfloat16* __restrict__ x,
                                             const float* __restrict__ w_g, int T, int d, int E,
                                             int t0, int e0, int kc, int chunk) {
   const int vpr = chunk / 8;  // 16-byte x vectors per token row
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
+  for (int u = 0; u < RouterRegs<RE, KC>::NX; ++u) {
     const int v = threadIdx.x + 256 * u;
     r.x[u] = make_uint4(0, 0, 0, 0);
     if (v < kRtT * vpr) {
@@ -49,9 +54,9 @@ __device__ __forceinline__ void router_load(RouterRegs& r, const __nv_bfloat16* 
     }
   }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int v = threadIdx.x + 256 * u;  // 8 float4 per K row (32 experts)
-    const int row = v >> 3, c4 = (v & 7) * 4;
+  for (int u = 0; u < RouterRegs<RE, KC>::NW; ++u) {
+    const int v = threadIdx.x + 256 * u;  // RE/4 float4 per K row
+    const int row = v / (RE / 4), c4 = (v % (RE / 4)) * 4;
     r.w[u] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (row < chunk) {
       const int e = e0 + c4;
@@ -68,11 +73,12 @@ __device__ __forceinline__ void router_load(RouterRegs& r, const __nv_bfloat16* 
   }
 }
 
-__device__ __forceinline__ void router_store(const RouterRegs& r, float (*xs)[kRtKC],
-                                             float (*ws)[kRtE], int chunk) {
+template <int RE, int KC>
+__device__ __forceinline__ void router_store(const RouterRegs<RE, KC>& r, float (*xs)[KC],
+                                             float (*ws)[RE], int chunk) {
   const int vpr = chunk / 8;
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
+  for (int u = 0; u < RouterRegs<RE, KC>::NX; ++u) {
     const int v = threadIdx.x + 256 * u;
     if (v < kRtT * vpr) {
       const int row = v / vpr, c8 = (v - row * vpr) * 8;
@@ -86,13 +92,17 @@ __device__ __forceinline__ void router_store(const RouterRegs& r, float (*xs)[kR
     }
   }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < RouterRegs<RE, KC>::NW; ++u) {
     const int v = threadIdx.x + 256 * u;
-    const int row = v >> 3, c4 = (v & 7) * 4;
+    const int row = v / (RE / 4), c4 = (v % (RE / 4)) * 4;
     if (row < chunk) *reinterpret_cast<float4*>(&ws[row][c4]) = r.w[u];
   }
 }
 
+// RE = 32 with 128-deep K chunks, or RE = 64 (half the CTAs: large grids
+// fit fewer waves) with 64-deep ones; thread (ty, tx) accumulates tokens
+// ty + 8i and experts tx + 32ee of the tile.
+template <int RE, int KC>
 __global__ void __launch_bounds__(256) k_router_cluster(
     const __nv_bfloat16* __restrict__ x, const float* __restrict__ w_g,
     const float* __restrict__ bias, int T, int d, int E, float* __restrict__ logits) {
@@ -100,45 +110,55 @@ __global__ void __launch_bounds__(256) k_router_cluster(
   pdl_wait();
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
+  constexpr int NE = RE / 32;
   const int CS = (int)cl.num_blocks();
   const int rank = (int)cl.block_rank();
-  __shared__ __align__(16) float xs[kRtT][kRtKC];
-  __shared__ __align__(16) float ws[kRtKC][kRtE];
-  __shared__ float part[kRtT * kRtE];
-  const int e0 = (blockIdx.x / CS) * kRtE;
+  __shared__ __align__(16) float xs[kRtT][KC];
+  __shared__ __align__(16) float ws[KC][RE];
+  __shared__ float part[kRtT * RE];
+  const int e0 = (blockIdx.x / CS) * RE;
   const int t0 = blockIdx.y * kRtT;
   const int kslice = d / CS;
   const int kbeg = rank * kslice, kend = kbeg + kslice;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  RouterRegs regs;
-  router_load(regs, x, w_g, T, d, E, t0, e0, kbeg, min(kRtKC, kend - kbeg));
-  for (int kc = kbeg; kc < kend; kc += kRtKC) {
-    const int chunk = min(kRtKC, kend - kc);  // 64 or 128
-    router_store(regs, xs, ws, chunk);
+  float acc[4][NE];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int ee = 0; ee < NE; ++ee) acc[i][ee] = 0.f;
+  RouterRegs<RE, KC> regs;
+  router_load<RE, KC>(regs, x, w_g, T, d, E, t0, e0, kbeg, min(KC, kend - kbeg));
+  for (int kc = kbeg; kc < kend; kc += KC) {
+    const int chunk = min(KC, kend - kc);  // a multiple of 64
+    router_store<RE, KC>(regs, xs, ws, chunk);
     __syncthreads();
-    if (kc + kRtKC < kend)
-      router_load(regs, x, w_g, T, d, E, t0, e0, kc + kRtKC, min(kRtKC, kend - kc - kRtKC));
+    if (kc + KC < kend)
+      router_load<RE, KC>(regs, x, w_g, T, d, E, t0, e0, kc + KC, min(KC, kend - kc - KC));
     for (int kk = 0; kk < chunk; kk += 4) {  // same FMA order as one kk at a time
       float4 xv[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(&xs[ty + 8 * i][kk]);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float wv = ws[kk + j][tx];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float xe = j == 0 ? xv[i].x : j == 1 ? xv[i].y : j == 2 ? xv[i].z : xv[i].w;
-          acc[i] = fmaf(xe, wv, acc[i]);
+        for (int ee = 0; ee < NE; ++ee) {
+          const float wv = ws[kk + j][tx + 32 * ee];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float xe = j == 0 ? xv[i].x : j == 1 ? xv[i].y : j == 2 ? xv[i].z : xv[i].w;
+            acc[i][ee] = fmaf(xe, wv, acc[i][ee]);
+          }
         }
       }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) part[(ty + 8 * i) * kRtE + tx] = acc[i];
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int ee = 0; ee < NE; ++ee) part[(ty + 8 * i) * RE + tx + 32 * ee] = acc[i][ee];
   cl.sync();
-  const int per = (kRtT * kRtE) / CS;
+  const int per = (kRtT * RE) / CS;
   for (int o = rank * per + threadIdx.x; o < (rank + 1) * per; o += 256) {
     // all CS remote loads in flight at once, then the sum in rank order
     float pv[16];
@@ -148,7 +168,7 @@ __global__ void __launch_bounds__(256) k_router_cluster(
 #pragma unroll
     for (int r = 0; r < 16; ++r)
       if (r < CS) v += pv[r];
-    const int t = t0 + o / kRtE, e = e0 + (o % kRtE);
+    const int t = t0 + o / RE, e = e0 + (o % RE);
     if (t < T && e < E) logits[(size_t)t * E + e] = bias ? v + bias[e] : v;
   }
   cl.sync();  // partial tiles stay alive until every CTA has read them
@@ -888,8 +908,10 @@ static int router_max_cluster() {
   static int max_cs = 0;
   if (max_cs == 0) {
     max_cs = 8;
-    if (cudaFuncSetAttribute(k_router_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                             1) == cudaSuccess) {
+    if (cudaFuncSetAttribute(k_router_cluster<32, 128>,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(k_router_cluster<64, 64>,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(16, 1, 1);
       cfg.blockDim = dim3(256, 1, 1);
@@ -901,7 +923,8 @@ static int router_max_cluster() {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k_router_cluster, &cfg) == cudaSuccess && n > 0)
+      if (cudaOccupancyMaxActiveClusters(&n, k_router_cluster<32, 128>, &cfg) == cudaSuccess &&
+          n > 0)
         max_cs = 16;
     }
     cudaGetLastError();
@@ -918,10 +941,15 @@ static int router_cluster_size(int d) {
 cudaError_t launch_router(const __nv_bfloat16* x, const float* w_g, const float* bias,
                           const moe_shape& s, float* logits, cudaStream_t st) {
   const int cs = router_cluster_size(s.d);
-  const dim3 grid((unsigned)(cs * ((s.E + kRtE - 1) / kRtE)), (unsigned)((s.T + kRtT - 1) / kRtT),
-                  1);
-  return launch_kernel(k_router_cluster, grid, dim3(256), 0, st, cs, x, w_g, bias, s.T, s.d, s.E,
-                       logits);
+  const unsigned ty = (unsigned)((s.T + kRtT - 1) / kRtT);
+  // 64-expert tiles when 32-expert ones would need more than 128 CTAs (a
+  // second wave of clusters)
+  const long long ctas32 = (long long)cs * ((s.E + 31) / 32) * ty;
+  if (ctas32 > 128 && s.E > 32)
+    return launch_kernel(k_router_cluster<64, 64>, dim3((unsigned)(cs * ((s.E + 63) / 64)), ty, 1),
+                         dim3(256), 0, st, cs, x, w_g, bias, s.T, s.d, s.E, logits);
+  return launch_kernel(k_router_cluster<32, 128>, dim3((unsigned)(cs * ((s.E + 31) / 32)), ty, 1),
+                       dim3(256), 0, st, cs, x, w_g, bias, s.T, s.d, s.E, logits);
 }
 
 #define MOE_VPL_DISPATCH(VPL_VAR, CALL) \
