@@ -126,6 +126,11 @@ __global__ void __launch_bounds__(256) k_router_cluster(
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int ee = 0; ee < NE; ++ee) acc[i][ee] = 0.f;
+  // warp ty's token rows ty + 8i hold tokens for i < ni; with one such row
+  // (at most 8 tokens in the tile) the warp multiplies only that row, and a
+  // warp with none multiplies nothing (the other rows' sums stay zero and are
+  // not stored)
+  const int ni = min(4, max(0, (min(kRtT, T - t0) - ty + 7) / 8));
   RouterRegs<RE, KC> regs;
   router_load<RE, KC>(regs, x, w_g, T, d, E, t0, e0, kbeg, min(KC, kend - kbeg));
   for (int kc = kbeg; kc < kend; kc += KC) {
@@ -134,20 +139,34 @@ __global__ void __launch_bounds__(256) k_router_cluster(
     __syncthreads();
     if (kc + KC < kend)
       router_load<RE, KC>(regs, x, w_g, T, d, E, t0, e0, kc + KC, min(KC, kend - kc - KC));
-    for (int kk = 0; kk < chunk; kk += 4) {  // same FMA order as one kk at a time
-      float4 xv[4];
+    if (ni >= 2) {
+      for (int kk = 0; kk < chunk; kk += 4) {  // same FMA order as one kk at a time
+        float4 xv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(&xs[ty + 8 * i][kk]);
+        for (int i = 0; i < 4; ++i)
+          xv[i] = *reinterpret_cast<const float4*>(&xs[ty + 8 * i][kk]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 4; ++j) {
 #pragma unroll
-        for (int ee = 0; ee < NE; ++ee) {
-          const float wv = ws[kk + j][tx + 32 * ee];
+          for (int ee = 0; ee < NE; ++ee) {
+            const float wv = ws[kk + j][tx + 32 * ee];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float xe = j == 0 ? xv[i].x : j == 1 ? xv[i].y : j == 2 ? xv[i].z : xv[i].w;
-            acc[i][ee] = fmaf(xe, wv, acc[i][ee]);
+            for (int i = 0; i < 4; ++i) {
+              const float xe = j == 0 ? xv[i].x : j == 1 ? xv[i].y : j == 2 ? xv[i].z : xv[i].w;
+              acc[i][ee] = fmaf(xe, wv, acc[i][ee]);
+            }
           }
+        }
+      }
+    } else if (ni == 1) {  // at most 8 tokens in the tile: warp ty's one row
+      for (int kk = 0; kk < chunk; kk += 4) {
+        const float4 xv = *reinterpret_cast<const float4*>(&xs[ty][kk]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float xe = j == 0 ? xv.x : j == 1 ? xv.y : j == 2 ? xv.z : xv.w;
+#pragma unroll
+          for (int ee = 0; ee < NE; ++ee)
+            acc[0][ee] = fmaf(xe, ws[kk + j][tx + 32 * ee], acc[0][ee]);
         }
       }
     }
