@@ -42,6 +42,9 @@ def test_launch_counts_match_the_profiled_launch_lists():
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE) == 6
     # up to 16 tokens GEMM1 reads x itself: no row gather
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE.with_T(8)) == 5
+    assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE.with_T(16)) == 5
+    assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE.with_T(17)) == 6
+    assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE.with_T(8), w8a8=True) == 7
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_DECODE, fp8=True) == 6
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_PREFILL) == 13
     assert bench.launches_per_forward(wl.QWEN3_30B_A3B_PREFILL, fp8=True) == 11

@@ -481,18 +481,21 @@ def test_forward_large_batch_gemm_regimes(cfg):
 
 
 @pytest.mark.parametrize("cfg", [wl.QWEN3_30B_A3B_DECODE.with_T(1),
+                                 wl.QWEN3_30B_A3B_DECODE.with_T(16),
+                                 wl.QWEN3_30B_A3B_DECODE.with_T(17),
                                  wl.QWEN3_30B_A3B_DECODE.with_T(64),
                                  wl.QWEN3_30B_A3B_DECODE.with_T(256),
                                  wl.MoEConfig("ragged-combine", T=37, d=320, E=6, k=3, f=128),
                                  wl.MoEConfig("ragged-direct", T=13, d=320, E=6, k=3, f=128)],
-                         ids=["T1", "T64", "T256", "ragged", "ragged-direct"])
+                         ids=["T1", "T16", "T17", "T64", "T256", "ragged", "ragged-direct"])
 def test_forward_equals_ffn_then_combine(cfg):
     """moe_forward's y equals moe_combine over moe_ffn's z on the layer's own
     dispatch bit for bit (the layer's gather, GEMMs and combine against the
     caller-offset FFN and the standalone combine), including a partial last
     128-column tile (d = 320), and again on a second call on the same
     workspace.  Up to 16 tokens the layer's GEMM1 reads x itself (no gather)
-    and maps rows in its epilogue (T = 1, T = 13)."""
+    and maps rows in its epilogue (T = 1, 13, 16; T = 17 is the first size
+    with the gather)."""
     x = wl.make_hidden(cfg, DEV, 4)
     w_g, bias = wl.make_router(cfg, DEV, 0)
     w13, w2 = wl.make_experts(cfg, DEV, 0)
