@@ -1578,15 +1578,14 @@ static cudaError_t swap_ffn_w8a8(const CUtensorMap& tW1, const CUtensorMap& tX1,
 }
 
 // Both GEMMs with E4M3 operands on both sides, at every batch size, and
-// between them the SwiGLU output quantised row by row: the swap-AB kernels
-// over the touched-expert list (T <= 64) or the 128-row tile list; for large
-// dense batches (the CTA-pair tile layout, pair_tiles) the CTA-pair kernels
-// over the tile pairs, with the lone-tile experts' leftover list on the
-// swap-AB kernels (their tokens fit one 128-row item).  The swap-AB GEMM2 of
-// the small-batch forms is an early launch (the quantisation kernel lets it
-// launch after its own wait; the work list precedes GEMM1); with at most 64
-// (token, expert) rows the quantisation runs per list entry beside GEMM1
-// instead, and GEMM2 waits per entry.
+// between them the SwiGLU output quantised: the swap-AB kernels over the
+// touched-expert list (T <= 64) or the 128-row tile list (swap_ffn_w8a8: the
+// quantisation per list entry beside GEMM1 when the entries are small or
+// many, else row by row between the GEMMs with GEMM2 an early launch); for
+// large dense batches (the CTA-pair tile layout, pair_tiles) the CTA-pair
+// kernels over the tile pairs, with the lone-tile experts' leftover list on
+// the swap-AB kernels (their tokens fit one 128-row item) and the row
+// quantiser between the GEMMs.
 int launch_expert_ffn_w8a8(const uint8_t* xq, const float* xs, long long x_rows,
                            const uint8_t* w13, const float* w13_scale, const uint8_t* w2,
                            const float* w2_scale, const moe_shape& s, const WsLayout& L,
