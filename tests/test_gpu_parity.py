@@ -111,8 +111,18 @@ def test_topk_on_router_logits_of_model_shapes(cfg):
                                  wl.MIXTRAL_8X7B.with_T(700),
                                  # E not a multiple of 4: the tensor-core epilogue's scalar stores
                                  wl.MoEConfig("router-odd-E", T=300, d=256, E=6, k=2, f=64,
+                                              zipf_s=1.0),
+                                 # cluster router: one token in a 32-token tile (the warps
+                                 # that multiply a single row), 448-deep K slices
+                                 wl.DEEPSEEK_V3_ROUTED.with_T(1),
+                                 # 64-expert tiles (the 32-expert grid would need 336 CTAs)
+                                 # with a partial last expert tile and an 8-token last tile
+                                 wl.MoEConfig("router-64-wide", T=200, d=1024, E=96, k=4, f=64,
+                                              zipf_s=1.0),
+                                 # 32-expert tiles, a partial expert tile, a 5-token last tile
+                                 wl.MoEConfig("router-partial", T=37, d=512, E=40, k=2, f=64,
                                               zipf_s=1.0)],
-                         ids=lambda c: c.name)
+                         ids=lambda c: f"{c.name}-T{c.T}")
 def test_router_within_fp32_error_bound(cfg):
     x = wl.make_hidden(cfg, "cpu", 0)
     w_g, bias = wl.make_router(cfg, "cpu", 0)
@@ -541,9 +551,12 @@ def test_forward_is_deterministic():
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
 
 
-def test_forward_matches_router_then_topk():
-    """moe_forward's routing equals moe_topk(moe_router(x)) bit for bit."""
-    cfg = wl.DEEPSEEK_V3_ROUTED.with_T(512)
+@pytest.mark.parametrize("T", [512, 64, 1])
+def test_forward_matches_router_then_topk(T):
+    """moe_forward's routing equals moe_topk(moe_router(x)) bit for bit (the
+    tensor-core router at T = 512; the cluster router with 64-expert tiles
+    at T = 64 and with single-row warps at T = 1)."""
+    cfg = wl.DEEPSEEK_V3_ROUTED.with_T(T)
     import dataclasses
     cfg = dataclasses.replace(cfg, f=64)
     x = wl.make_hidden(cfg, DEV, 0)

@@ -140,6 +140,10 @@ def test_ffn_w8a8_ragged_shapes():
     # widths, and experts of more than one tile (about 128 rows each)
     _ffn_case(wl.MoEConfig("ragged-tiles", T=300, d=320, E=20, k=2, f=192))
     _ffn_case(wl.MoEConfig("multi-tile-entries", T=256, d=256, E=16, k=8, f=384))
+    # the per-entry quantiser's register rows end at 1024 columns; 1088 takes
+    # the two-pass row quantisation
+    _ffn_case(wl.MoEConfig("quant-regs-1024", T=40, d=256, E=20, k=2, f=1024))
+    _ffn_case(wl.MoEConfig("quant-two-pass-1088", T=40, d=256, E=20, k=2, f=1088))
 
 
 @pytest.mark.parametrize("T,counts", [
