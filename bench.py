@@ -748,8 +748,10 @@ def run_ours(args):
     value = tokens / (total_ms / 1e3)
 
     # ---------------- end to end through the public API, host buffers
-    # MoELayer.forward_host: pinned x -> device, graph replay of the layer,
-    # device -> pinned y, every step; the host waits for y each step.
+    # MoELayer.forward_host, every step: one graph replay that copies the
+    # pinned x to the device (a library kernel) and runs the layer, whose
+    # combine writes the pinned y across the bus; the host waits for y each
+    # step.  The bytes crossing the bus are x's and y's, as with copies.
     x_host = x.cpu().pin_memory()
     y_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
     for _ in range(2):

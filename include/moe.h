@@ -79,7 +79,8 @@ MOE_API const char* moe_error_string(int status);
 /* Library ABI version (major * 100 + minor): 101 adds the EPLB calls and
  * moe_dispatch_dedup; 102 the FP8-weight calls; 103 moe_ep_recv_experts and
  * FP8 weights at every batch size; 104 the FP8-activation (W8A8) calls and
- * moe_quantise_rows_e4m3 (the workspace grows by their buffers). */
+ * moe_quantise_rows_e4m3 (the workspace grows by their buffers); 105
+ * moe_copy, and the layer calls' y may be pinned host memory. */
 MOE_API int moe_version(void);
 
 /* Bytes of scratch workspace `ws` that moe_dispatch / moe_ffn / moe_forward
@@ -173,7 +174,11 @@ MOE_API int moe_combine(const moe_bf16* z, const int32_t* row_of, const float* w
  * graph).  Inputs as above; y [T, d] bf16 out.  idx_out [T,k], w_out [T,k]
  * and counts_out [E] receive the routing decisions when non-NULL.  With
  * s->R > 1 the send-count matrix and rank offsets are computed too (in the
- * workspace).  ws: moe_workspace_size(s) bytes. */
+ * workspace).  ws: moe_workspace_size(s) bytes.  y may be device memory or
+ * host memory the device addresses directly (page-locked, e.g. from
+ * cudaHostAlloc): the combine then writes the result across the bus itself,
+ * so no separate device-to-host copy is needed; pageable host memory is
+ * rejected with MOE_ERR_INVALID_ARG (this and moe_forward_fp8 / _w8a8). */
 MOE_API int moe_forward(const moe_bf16* x, const float* w_g, const float* bias,
                 const moe_bf16* w13, const moe_bf16* w2, const moe_shape* s,
                 moe_bf16* y, int32_t* idx_out, float* w_out,
@@ -425,6 +430,17 @@ MOE_API int moe_forward_w8a8_staged(const moe_bf16* x, const float* w_g, const f
  * One warp per row; asynchronous on `stream`. */
 MOE_API int moe_quantise_rows_e4m3(const moe_bf16* a, int64_t rows, int32_t cols,
                                    uint8_t* codes, float* scales, void* stream);
+
+/* Copy of `bytes` bytes from src to dst by a kernel on `stream`, in the
+ * library's launch chain: the next library kernel may launch while it runs
+ * and waits for it (so a captured graph goes from the copy into the layer
+ * without a copy-engine node between them).  Either pointer may be device
+ * memory or host memory the device addresses directly (page-locked); both
+ * 16-byte aligned, bytes a multiple of 16.  Pageable host memory, a NULL or
+ * misaligned pointer or a size that is not a multiple of 16 give
+ * MOE_ERR_INVALID_ARG; overlapping ranges are undefined.  bytes == 0 does
+ * nothing. */
+MOE_API int moe_copy(void* dst, const void* src, int64_t bytes, void* stream);
 
 /* Self-test of the failure path every device-side wait uses: launches one
  * kernel that waits on a barrier nothing will ever complete, through the same

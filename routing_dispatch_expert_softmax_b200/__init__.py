@@ -16,5 +16,6 @@ from .binding import (EXPORTS, MOE_STAGE_EVENTS, STAGE_NAMES, MOE_ERR_CUDA, MOE_
                       moe_workspace_size_eplb, workspace_eplb, moe_forward_eplb,
                       moe_dispatch_dedup, moe_ffn_fp8, moe_forward_fp8,
                       moe_forward_fp8_staged, moe_ep_recv_experts, moe_ffn_w8a8,
-                      moe_forward_w8a8, moe_forward_w8a8_staged, moe_quantise_rows_e4m3)
+                      moe_forward_w8a8, moe_forward_w8a8_staged, moe_quantise_rows_e4m3,
+                      moe_copy)
 from .layer import MoELayer  # noqa: F401

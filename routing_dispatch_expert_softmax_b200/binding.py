@@ -2,7 +2,8 @@
 
 Argument marshalling only: every step of the layer runs in the library's CUDA
 kernels.  Tensors are torch CUDA tensors (PyTorch supplies device memory and
-streams); the functions keep the C names and raise :class:`MoEError` on a
+streams; the layer calls' y and moe_copy's operands may also be pinned host
+tensors); the functions keep the C names and raise :class:`MoEError` on a
 non-zero status.  There is no fallback: if the library is missing or the
 device is not an sm_100 GPU, calls raise.
 """
@@ -33,7 +34,7 @@ EXPORTS = ("moe_error_string", "moe_version", "moe_workspace_size", "moe_router"
            "moe_workspace_size_eplb", "moe_forward_eplb", "moe_dispatch_dedup",
            "moe_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_staged", "moe_ep_recv_experts",
            "moe_ffn_w8a8", "moe_forward_w8a8", "moe_forward_w8a8_staged",
-           "moe_quantise_rows_e4m3")
+           "moe_quantise_rows_e4m3", "moe_copy")
 
 
 class MoEError(RuntimeError):
@@ -124,6 +125,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_forward_w8a8_staged.argtypes = [_P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]
     lib.moe_quantise_rows_e4m3.restype = ctypes.c_int
     lib.moe_quantise_rows_e4m3.argtypes = [_P, ctypes.c_int64, ctypes.c_int32, _P, _P, _P]
+    lib.moe_copy.restype = ctypes.c_int
+    lib.moe_copy.argtypes = [_P, _P, ctypes.c_int64, _P]
     _lib = lib
     return lib
 
@@ -148,6 +151,20 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _ptr_dev_or_pinned(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    """A CUDA tensor, or a page-locked CPU tensor the device addresses
+    directly (the calls that accept host memory check it again)."""
+    if isinstance(t, torch.Tensor) and t.device.type == "cpu":
+        if not t.is_pinned():
+            raise ValueError(f"{name} must be a CUDA tensor or page-locked (pinned) host memory")
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        return ctypes.c_void_p(t.data_ptr())
+    return _ptr(t, dtype, name)
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -236,7 +253,8 @@ def moe_forward(x, w_g, bias, w13, w2, y, shape: MoEShape, ws, idx_out=None, w_o
     _check(load_library().moe_forward(
         _ptr(x, torch.bfloat16, "x"), _ptr(w_g, torch.float32, "w_g"),
         _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.bfloat16, "w13"),
-        _ptr(w2, torch.bfloat16, "w2"), ctypes.byref(shape), _ptr(y, torch.bfloat16, "y"),
+        _ptr(w2, torch.bfloat16, "w2"), ctypes.byref(shape),
+        _ptr_dev_or_pinned(y, torch.bfloat16, "y"),
         _ptr(idx_out, torch.int32, "idx_out"), _ptr(w_out, torch.float32, "w_out"),
         _ptr(counts_out, torch.int32, "counts_out"), _ptr(ws, torch.uint8, "ws"),
         _stream(stream)), "moe_forward")
@@ -369,7 +387,7 @@ def moe_forward_fp8(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoESha
         _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.uint8, "w13"),
         _ptr(w13_scale, torch.float32, "w13_scale"), _ptr(w2, torch.uint8, "w2"),
         _ptr(w2_scale, torch.float32, "w2_scale"), ctypes.byref(shape),
-        _ptr(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
+        _ptr_dev_or_pinned(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
         _ptr(w_out, torch.float32, "w_out"), _ptr(counts_out, torch.int32, "counts_out"),
         _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_forward_fp8")
 
@@ -394,7 +412,7 @@ def moe_forward_w8a8(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoESh
         _ptr(bias, torch.float32, "bias"), _ptr(w13, torch.uint8, "w13"),
         _ptr(w13_scale, torch.float32, "w13_scale"), _ptr(w2, torch.uint8, "w2"),
         _ptr(w2_scale, torch.float32, "w2_scale"), ctypes.byref(shape),
-        _ptr(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
+        _ptr_dev_or_pinned(y, torch.bfloat16, "y"), _ptr(idx_out, torch.int32, "idx_out"),
         _ptr(w_out, torch.float32, "w_out"), _ptr(counts_out, torch.int32, "counts_out"),
         _ptr(ws, torch.uint8, "ws"), _stream(stream)), "moe_forward_w8a8")
 
@@ -420,6 +438,17 @@ def moe_quantise_rows_e4m3(a, codes, scales, stream=None):
     _check(load_library().moe_quantise_rows_e4m3(
         _ptr(a, torch.bfloat16, "a"), rows, cols, _ptr(codes, torch.uint8, "codes"),
         _ptr(scales, torch.float32, "scales"), _stream(stream)), "moe_quantise_rows_e4m3")
+
+
+def moe_copy(dst, src, stream=None):
+    """Copies src's bytes into dst by a library kernel (either may be a pinned
+    host tensor); a multiple of 16 bytes, 16-byte aligned."""
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() < nbytes:
+        raise ValueError("dst is smaller than src")
+    _check(load_library().moe_copy(_ptr_dev_or_pinned(dst, None, "dst"),
+                                   _ptr_dev_or_pinned(src, None, "src"), nbytes,
+                                   _stream(stream)), "moe_copy")
 
 
 def moe_forward_fp8_staged(x, w_g, bias, w13, w13_scale, w2, w2_scale, y, shape: MoEShape, ws,

@@ -9,13 +9,25 @@ using namespace moe;
 
 namespace {
 
-constexpr int kVersion = 104;
+constexpr int kVersion = 105;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool ok16(const void* p) { return p != nullptr && aligned(p, 16); }
 bool ok4(const void* p) { return p != nullptr && aligned(p, 4); }
 
 bool shape_ok(const moe_shape* s) { return shape_valid(s); }
+
+// p can be read and written by the device as it is: device or managed
+// memory, or page-locked host memory mapped at the same address.
+bool device_addressable(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return true;
+  return a.type == cudaMemoryTypeHost && a.devicePointer == p;
+}
 
 // Current device: its SM count, and whether it is an sm_100 part.
 int device_check(int* num_sms) {
@@ -208,6 +220,7 @@ static int forward_impl(int mode, const moe_bf16* x, const float* w_g, const flo
   int sms = 0;
   int st = device_check(&sms);
   if (st != MOE_OK) return st;
+  if (!device_addressable(y)) return MOE_ERR_INVALID_ARG;  // y may be page-locked host memory
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t {
     if (!events || !events[i]) return cudaSuccess;
@@ -468,6 +481,17 @@ int moe_selftest_bounded_wait(long long limit_ns, void* ws, void* stream) {
   return cuda_status(launch_selftest_bounded_wait((unsigned long long)limit_ns,
                                                   static_cast<int*>(ws),
                                                   static_cast<cudaStream_t>(stream)));
+}
+
+int moe_copy(void* dst, const void* src, int64_t bytes, void* stream) {
+  if (bytes < 0 || bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (bytes == 0) return MOE_OK;
+  if (!ok16(dst) || !ok16(src)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  int st = device_check(&sms);
+  if (st != MOE_OK) return st;
+  if (!device_addressable(dst) || !device_addressable(src)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_copy(dst, src, bytes, sms, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_check(void* ws, void* stream) {

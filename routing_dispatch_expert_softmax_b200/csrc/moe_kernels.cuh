@@ -34,6 +34,10 @@ cudaError_t launch_gather(const __nv_bfloat16* x, const int* perm, long long P, 
                           int d, __nv_bfloat16* x_perm, int* err, cudaStream_t st);
 cudaError_t launch_selftest_bounded_wait(unsigned long long limit_ns, int* err,
                                          cudaStream_t st);
+// bytes (a multiple of 16) from src to dst, both 16-byte aligned and
+// addressable by the device.
+cudaError_t launch_copy(void* dst, const void* src, long long bytes, int num_sms,
+                        cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* z, const int* row_of, const float* w,
                            const moe_shape& s, __nv_bfloat16* y, cudaStream_t st);
 // early_gemm1: the kernel just before (the row gather) lets GEMM1 launch only

@@ -897,6 +897,29 @@ __global__ void __launch_bounds__(256) k_combine(
   }
 }
 
+// ============================================================== copy
+// dst[i] = src[i] for n 16-byte vectors, grid-stride.  It lets the next
+// kernel launch at once (that one waits for this one) and waits for a
+// previous kernel only before its reads.
+__global__ void __launch_bounds__(256) k_copy16(const uint4* __restrict__ src,
+                                                uint4* __restrict__ dst, long long n) {
+  pdl_trigger();
+  pdl_wait();
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
+cudaError_t launch_copy(void* dst, const void* src, long long bytes, int num_sms,
+                        cudaStream_t st) {
+  const long long n = bytes / 16;
+  if (n == 0) return cudaSuccess;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 4LL * num_sms) blocks = 4LL * num_sms;
+  return launch_kernel(k_copy16, dim3((unsigned)blocks), dim3(256), 0, st, 1,
+                       reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst), n);
+}
+
 // ============================================================== self-test
 // Waits on an mbarrier that nothing ever arrives on, through the same bounded
 // wait the GEMM pipeline uses, with a caller-chosen limit: the wait must give

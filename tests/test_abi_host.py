@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_error_strings(lib):
-    assert moe.moe_version() == 104
+    assert moe.moe_version() == 105
     for code in range(6):
         assert moe.moe_error_string(code).startswith("MOE_")
     assert "unknown" in moe.moe_error_string(99)
@@ -111,6 +111,12 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     assert _raw(lib, "moe_selftest_bounded_wait", ctypes.c_longlong(2 * 10 ** 9), _P(A16),
                 None) == INV
     assert _raw(lib, "moe_check", _P(A16 + 8), None) == INV
+    # moe_copy: sizes not a multiple of 16, misaligned or null pointers
+    assert _raw(lib, "moe_copy", _P(A16), _P(A16), ctypes.c_int64(24), None) == INV
+    assert _raw(lib, "moe_copy", _P(A16), _P(A16), ctypes.c_int64(-16), None) == INV
+    assert _raw(lib, "moe_copy", _P(A16 + 4), _P(A16), ctypes.c_int64(32), None) == INV
+    assert _raw(lib, "moe_copy", None, _P(A16), ctypes.c_int64(32), None) == INV
+    assert _raw(lib, "moe_copy", None, None, ctypes.c_int64(0), None) == B.MOE_OK
     # dedup dispatch: needs R >= 2 and a workspace
     s_r4 = ctypes.byref(B.MoEShape.of(**dict(VALID, R=4)))
     assert _raw(lib, "moe_dispatch_dedup", _P(A16), None, s, _P(A16), _P(A16), _P(A16),
@@ -200,6 +206,8 @@ def test_no_cpu_fallback_without_a_gpu(lib):
     assert _raw(lib, "moe_forward_w8a8", *[_P(A16)] * 7, s, _P(A16), None, None, None,
                 _P(A16), None) == B.MOE_ERR_CUDA
     assert _raw(lib, "moe_quantise_rows_e4m3", _P(A16), 4, 32, _P(A16), _P(A16),
+                None) == B.MOE_ERR_CUDA
+    assert _raw(lib, "moe_copy", _P(A16), _P(A16 + 64), ctypes.c_int64(32),
                 None) == B.MOE_ERR_CUDA
 
 
