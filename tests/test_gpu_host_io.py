@@ -108,6 +108,11 @@ def test_forward_host_direct_and_copy_paths_agree():
     torch.cuda.synchronize()
     assert torch.equal(y_pinned, y2_ref)
     assert layer.check() == moe.MOE_OK
+    # buffers above the in-place limit (4 MB each) keep the copy path
+    big = 1100  # 1100 x 2048 bf16 = 4.5 MB
+    x_big = torch.zeros(big, cfg.d, dtype=torch.bfloat16).pin_memory()
+    assert not layer._host_direct(x_big, torch.empty_like(x_big).pin_memory())
+    assert layer._host_direct(x_pinned, y_pinned)
     # the W8A8 layer
     from routing_dispatch_expert_softmax_b200 import workloads
     c13, s13, c2, s2 = workloads.make_experts_fp8(cfg, DEV, 0)
