@@ -148,6 +148,7 @@ class MoELayer:
         self._ws: Dict[int, torch.Tensor] = {}
         self._graphs: Dict[int, _Graphed] = {}
         self._host_graphs: Dict[tuple, _GraphedHost] = {}
+        self._host_refused: set = set()
         self._last_ws: Optional[torch.Tensor] = None
         self._eplb: Optional[dict] = None
         self._auto: Optional[dict] = None
@@ -317,18 +318,26 @@ class MoELayer:
         (T, x_host, y_host) buffer triple, the most recent few.  Other (and
         larger) buffers go through copies to and from a device-side graph."""
         T = int(x_host.shape[0])
-        if self._host_direct(x_host, y_host):
-            key = (T, x_host.data_ptr(), y_host.data_ptr())
+        key = (T, x_host.data_ptr(), y_host.data_ptr())
+        if key not in self._host_refused and self._host_direct(x_host, y_host):
             g = self._host_graphs.pop(key, None)
             if g is None:
-                g = _GraphedHost(self, T, x_host, y_host)
-            self._host_graphs[key] = g  # most recent last
-            while len(self._host_graphs) > self._MAX_HOST_GRAPHS:
-                self._host_graphs.pop(next(iter(self._host_graphs)))
-            g.graph.replay()
-            self._last_ws = g.ws
-            self._record_graphed(g)
-            return y_host
+                try:
+                    g = _GraphedHost(self, T, x_host, y_host)
+                except B.MoEError as err:
+                    # the library refused a host buffer (before any launch or
+                    # capture): these buffers take the copy path from now on
+                    if err.status != B.MOE_ERR_INVALID_ARG:
+                        raise
+                    self._host_refused.add(key)
+            if g is not None:
+                self._host_graphs[key] = g  # most recent last
+                while len(self._host_graphs) > self._MAX_HOST_GRAPHS:
+                    self._host_graphs.pop(next(iter(self._host_graphs)))
+                g.graph.replay()
+                self._last_ws = g.ws
+                self._record_graphed(g)
+                return y_host
         g = self.graphed(T)
         g.x.copy_(x_host, non_blocking=True)
         g.graph.replay()
