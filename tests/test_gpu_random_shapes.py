@@ -9,8 +9,13 @@ with E4M3 weights and activations."""
 
 import numpy as np
 import pytest
+import torch
 
+import oracle
+import routing_dispatch_expert_softmax_b200 as moe
 from routing_dispatch_expert_softmax_b200 import workloads as wl
+from routing_dispatch_expert_softmax_b200.binding import MoEShape
+from parity_utils import LazyExperts, assert_layer_close
 
 import test_gpu_parity as P
 import test_gpu_w8a8 as W
@@ -45,3 +50,49 @@ def test_forward_random_shape(cfg):
                          ids=lambda c: f"{c.name}-T{c.T}-d{c.d}-E{c.E}-k{c.k}-f{c.f}")
 def test_forward_w8a8_random_shape(cfg):
     W._forward_case(cfg, seed=3)
+
+
+def _offsets(rng, P, E):
+    """Per-expert row counts summing to P: skewed, with empty experts, and at
+    times one expert holding more rows than the batch has tokens (moe_ffn's
+    caller offsets allow it)."""
+    w = rng.pareto(1.0, E) + 1e-3
+    w[rng.random(E) < 0.3] = 0.0
+    if w.sum() == 0:
+        w[0] = 1.0
+    counts = np.floor(w / w.sum() * P).astype(np.int64)
+    counts[int(np.argmax(w))] += P - counts.sum()
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+
+
+def _ffn_shapes(seed, n):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        cfg = _shapes(seed * 7 + i, 1, f"rand-ffn-{i}-")[0]
+        out.append((cfg, _offsets(rng, cfg.T * cfg.k, cfg.E)))
+    return out
+
+
+@pytest.mark.parametrize("cfg,offsets", _ffn_shapes(20242, 16),
+                         ids=lambda v: v.name if hasattr(v, "name") else "")
+def test_ffn_random_offsets(cfg, offsets):
+    P = int(offsets[-1])
+    x_perm = wl.make_hidden(wl.MoEConfig("rows", T=P, d=cfg.d, E=1, k=1, f=64), "cuda", 5)
+    w13, w2 = wl.make_experts(cfg, "cuda", 5)
+    shape = MoEShape.from_config(cfg)
+    z = torch.empty(P, cfg.d, dtype=torch.bfloat16, device="cuda")
+    ws = moe.workspace(shape)
+    moe.moe_ffn(x_perm, torch.from_numpy(offsets).cuda(), w13, w2, z, shape, ws)
+    assert moe.moe_check(ws) == moe.MOE_OK
+    ref = oracle.expert_outputs(x_perm.double().cpu().numpy(), np.arange(P), offsets,
+                                LazyExperts(w13), LazyExperts(w2))
+    assert_layer_close(z, ref, f"moe_ffn {cfg.name} T={cfg.T}")
+
+
+@pytest.mark.parametrize("cfg,offsets", _ffn_shapes(20243, 10),
+                         ids=lambda v: v.name if hasattr(v, "name") else "")
+def test_ffn_w8a8_random_offsets(cfg, offsets):
+    P = int(offsets[-1])
+    x_perm = wl.make_hidden(wl.MoEConfig("rows", T=P, d=cfg.d, E=1, k=1, f=64), "cuda", 5)
+    W._ffn_case(cfg, seed=5, offsets=offsets, x_perm=x_perm)
