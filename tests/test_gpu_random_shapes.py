@@ -96,3 +96,24 @@ def test_ffn_w8a8_random_offsets(cfg, offsets):
     P = int(offsets[-1])
     x_perm = wl.make_hidden(wl.MoEConfig("rows", T=P, d=cfg.d, E=1, k=1, f=64), "cuda", 5)
     W._ffn_case(cfg, seed=5, offsets=offsets, x_perm=x_perm)
+
+
+def _dispatch_cases(seed, n):
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        T = int(rng.choice([1, 7, 64, 255, 256, 257, 1000, 1025, 3000, 9000]))
+        R = int(rng.choice([0, 2, 4, 8, 16, 64]))
+        E = (R if R > 1 else 1) * int(rng.integers(1, 17))      # a multiple of R, <= 1024
+        k = int(rng.integers(1, min(E, 32) + 1))
+        d = 64 * int(rng.integers(1, 5))
+        out.append((T, d, E, k, R))
+    return out
+
+
+@pytest.mark.parametrize("T,d,E,k,R", _dispatch_cases(20244, 20))
+def test_dispatch_random_shape(T, d, E, k, R):
+    """Counts, offsets, permutation, row map, gathered rows and the virtual
+    EP layout bit for bit against the oracle (both routing-table kernels: the
+    fused one up to 1024 tokens, the four-kernel form above)."""
+    P.test_dispatch_bit_exact(T, d, E, k, R)
