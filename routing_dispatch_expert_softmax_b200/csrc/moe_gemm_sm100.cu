@@ -486,11 +486,16 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
+// Arrives on the barrier at the same offset in CTA `cta` of the cluster.  The
+// default (CTA-scope) release is enough for its one use, the accumulator-free
+// signal: the TMEM loads it guards have completed (tcgen05.wait::ld) before it,
+// and the MMA issuer reads nothing else this thread wrote.  A cluster-scope
+// release would also wait for the epilogue's global stores of the tile.
 __device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar, uint32_t cta) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
       "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+      "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
       "r"(cta)
       : "memory");
 }
