@@ -509,9 +509,14 @@ struct PairCfg {
   static constexpr int kBBytes = 128 * kGemmBK * 2;  // this CTA's 128 weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 512;  // two 128 x 256 fp32 accumulators
+  // Epilogue warps: two per 32-lane TMEM quarter, each taking half of the
+  // tile's columns, so that draining an accumulator keeps pace with the
+  // MMAs of the next tile (short-K GEMM2 tiles especially).
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   // Per epilogue warp: 32 rows x 128 bytes of output staged for full-line
   // stores (the plain-store epilogue only).
-  static constexpr int kOutStageBytes = EPI == kEpiStore ? 4 * 32 * 128 : 0;
+  static constexpr int kOutStageBytes = EPI == kEpiStore ? kEpiWarps * 32 * 128 : 0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kOutStageBytes + 1024 + 256;
 };
 
@@ -519,7 +524,7 @@ struct PairCfg {
 // rows then hold 128 K elements (kind::f8f6f4 MMAs), and the epilogue
 // multiplies each accumulator by args.a_scale[row] * args.b_scale[weight row].
 template <int EPI, bool F8 = false>
-__global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
+__global__ void __launch_bounds__(PairCfg<EPI>::kThreads, 1) k_grouped_gemm_2sm(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const GemmArgs args) {
   using C = PairCfg<EPI>;
@@ -549,7 +554,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
+      mbar_init(&tempty[a], 2 * 32 * C::kEpiWarps);  // every epilogue thread of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -670,13 +675,17 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
       }
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
-    // Each warp owns TMEM lanes q*32.. (32 output rows).  GEMM2: a 64-column
-    // slice is packed to bf16, written row by row into the warp's staging
-    // tile (16-byte chunks XOR-swizzled by row: no bank conflicts either way)
-    // and read back so that every store instruction writes 4 full 128-byte
-    // rows instead of half sectors of 32 rows.
+    // ------------------------------------------------ epilogue (warps 2.., both CTAs)
+    // Each warp owns TMEM lanes q*32.. (32 output rows; a warp reaches the
+    // lanes of its index mod 4) and half of the accumulator's columns (hc).
+    // GEMM2: a 64-column slice is packed to bf16, written row by row into the
+    // warp's staging tile (16-byte chunks XOR-swizzled by row: no bank
+    // conflicts either way) and read back so that every store instruction
+    // writes 4 full 128-byte rows instead of half sectors of 32 rows.
+    static_assert(C::kEpiWarps == 4 || C::kEpiWarps == 8, "one or two warps per lane quarter");
+    constexpr int kColParts = C::kEpiWarps / 4;
     const int q = warp & 3;
+    const int hc = (warp - 2) >> 2;
     uint4* st_tile = out_stage + (size_t)(warp - 2) * 32 * 8;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
     int it = 0;
@@ -720,7 +729,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
         const bool row_ok = row < rowend;
         const float sa = (F8 && row_ok) ? __ldg(args.a_scale + row) : 1.0f;
 #pragma unroll 1
-        for (int c = 0; c < H; c += 32) {
+        for (int c = hc * (H / kColParts); c < (hc + 1) * (H / kColParts); c += 32) {
           uint32_t g[32], u[32];
           tmem_ld_32x32b_x32(t_addr + c, g);
           tmem_ld_32x32b_x32(t_addr + H + c, u);
@@ -753,7 +762,7 @@ __global__ void __launch_bounds__(192, 1) k_grouped_gemm_2sm(
         const int row = row_base + lane;
         const float sa = (F8 && row < rowend) ? __ldg(args.a_scale + row) : 1.0f;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 64) {
+        for (int c = hc * (BN / kColParts); c < (hc + 1) * (BN / kColParts); c += 64) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t a[32];
@@ -1529,8 +1538,8 @@ static cudaError_t launch_gemm_2sm(const CUtensorMap& ta, const CUtensorMap& tb,
   }
   int clusters = max_pairs_work < num_sms / 2 ? max_pairs_work : num_sms / 2;
   if (clusters < 1) clusters = 1;
-  return launch_kernel(k_grouped_gemm_2sm<EPI, F8>, dim3(2 * clusters), dim3(192), C::kSmemBytes,
-                       st, 2, ta, tb, args);
+  return launch_kernel(k_grouped_gemm_2sm<EPI, F8>, dim3(2 * clusters), dim3(C::kThreads),
+                       C::kSmemBytes, st, 2, ta, tb, args);
 }
 
 // The W8A8 expert GEMMs in the swap-AB form over the touched-expert list
